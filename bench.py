@@ -1,0 +1,398 @@
+"""WTConv layer fwd+bwd benchmark on B200 (prints one JSON line on rank 0).
+
+A step is one pass of the whole layer hot path over one batch: forward,
+backward-data and backward-weight (the fused kernels of libwtconv) on the
+ConvNeXt-T stage-1 shape (N=32, C=96, 56x56, k=5, L=3, fp32) by default.
+
+  python bench.py --gpus N --steps K --warmup W [--impl reference]
+
+Timing: W untimed warm-up steps; then a barrier + synchronize, K timed steps
+with CUDA events on the launching stream (each step preceded by an L2 flush
+that writes a buffer larger than L2, outside the events), a synchronize +
+barrier, and the max over ranks.  Multi-GPU runs are data parallel with
+weak scaling: every rank runs the full per-GPU batch and the parameter
+gradients are summed over ranks with one NCCL all-reduce inside the step.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+import torch.distributed as dist
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from depthwise_convolution_wtconv_b200.configs import WORKLOADS, BENCH_WORKLOAD  # noqa: E402
+from depthwise_convolution_wtconv_b200.inputs import make_inputs  # noqa: E402
+
+METRIC = "WTConv layer fwd+bwd steps/s and achieved HBM GB/s (% of B200 peak)"
+PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_HBM_GBS = 6650.0
+SM_COUNT_NOMINAL = 148
+FP32_LANES_PER_SM = 128
+L2_FLUSH_BYTES = 256 << 20
+
+
+def algorithmic_counts(wl):
+    """Per-launch algorithmic FMAs and bytes of each pass (fp32 arithmetic).
+
+    FMAs: P*k^2*(1 + (4/3)(1 - 4^-L)) per pass (base conv plus the level-l
+    convs on 4C channels at 4^-l of the pixels).  Bytes: forward reads x and
+    writes y; backward-data reads dy, writes dx; backward-weight reads x and
+    dy; parameters (and gradients) are counted once per pass they touch.
+    """
+    P = wl.P
+    k2 = wl.k * wl.k
+    fma = P * k2 * (1.0 + (4.0 / 3.0) * (1.0 - 4.0 ** (-wl.L)))
+    S = P * wl.io_bytes
+    params = 4 * (wl.C * k2 + 2 * wl.C + wl.L * wl.C * 4 * (k2 + 1))
+    return dict(
+        fwd=dict(fma=fma, bytes=2 * S + params),
+        bwd_data=dict(fma=fma, bytes=2 * S + params),
+        bwd_weight=dict(fma=fma, bytes=2 * S + 2 * params),
+    )
+
+
+def load_peaks():
+    try:
+        with open(PEAKS_PATH) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return {"hbm_gbs": FALLBACK_HBM_GBS, "sm_max_mhz": 1965.0}, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = [r.split(",") for r in out.strip().splitlines() if r.strip()]
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                smax.append(float(r[2]))
+                for name, v in zip(names, r[5:9]):
+                    if v.strip().lower() == "active":
+                        reasons.add(name)
+            except (IndexError, ValueError):
+                continue
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def setup_dist():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1 and not dist.is_initialized():
+        from datetime import timedelta
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=timedelta(seconds=120))
+    return world, rank, local
+
+
+def max_over_ranks(value, world, device):
+    if world == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def grads_flat_views(wl, device):
+    """One flat fp32 buffer with views for every parameter gradient (so the
+    data-parallel all-reduce is a single collective)."""
+    k2 = wl.k * wl.k
+    sizes = [wl.C * k2, wl.C, wl.C, wl.L * wl.C * 4 * k2, wl.L * wl.C * 4]
+    flat = torch.empty(sum(sizes), dtype=torch.float32, device=device)
+    views, o = [], 0
+    for s in sizes:
+        views.append(flat[o:o + s])
+        o += s
+    g = dict(dw0=views[0].view(wl.C, wl.k, wl.k), db0=views[1], ds0=views[2],
+             dwl=views[3].view(wl.L, wl.C, 4, wl.k, wl.k) if wl.L else None,
+             dsl=views[4].view(wl.L, wl.C, 4) if wl.L else None)
+    return flat, g
+
+
+def run_ours(args, wl, world, rank, local):
+    import depthwise_convolution_wtconv_b200 as wt
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    dt = torch.float32 if wl.io == "f32" else torch.bfloat16
+    inp = make_inputs(wl, seed=rank)
+    X = inp["X"].to(dt).to(device)
+    dY = inp["dY"].to(dt).to(device)
+    p = {k: inp[k].to(device) for k in ("W0", "b0", "s0")}
+    Wl = inp["Wl"].to(device) if wl.L else None
+    sl = inp["sl"].to(device) if wl.L else None
+    Y = torch.empty_like(X)
+    dX = torch.empty_like(X)
+    gflat, grads = grads_flat_views(wl, device)
+    desc = wt.make_desc(wl.N, wl.C, wl.H, wl.W, wl.k, wl.L, wl.io)
+    ws = torch.empty(max(16, wt.workspace_size(desc, 2)), dtype=torch.uint8, device=device)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step(ev=None, x=X, dy=dY, y=Y, dx=dX):
+        if ev is not None:
+            ev[0].record(stream)
+        wt.forward(x, p["W0"], p["b0"], p["s0"], Wl, sl, y=y, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        wt.backward_data(dy, p["W0"], p["s0"], Wl, sl, dx=dx, stream=stream)
+        if ev is not None:
+            ev[2].record(stream)
+        wt.backward_weight(x, dy, p["W0"], p["b0"], p["s0"], Wl, sl, grads=grads, ws=ws, stream=stream)
+        if ev is not None:
+            ev[3].record(stream)
+        if world > 1:
+            dist.all_reduce(gflat)
+        if ev is not None:
+            ev[4].record(stream)
+
+    for _ in range(args.warmup):
+        flush.fill_(0.0)
+        step()
+    torch.cuda.synchronize(device)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(device)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    sampler = ClockSampler(local)
+    sampler.start()
+    t_wall = time.perf_counter()
+    for i in range(args.steps):
+        flush.fill_(0.0)
+        step(evs[i])
+    torch.cuda.synchronize(device)
+    t_wall = time.perf_counter() - t_wall
+    clocks = sampler.stop()
+    if world > 1:
+        dist.barrier()
+    per_step = [e[0].elapsed_time(e[4]) for e in evs]
+    t_fwd = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
+    t_bd = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
+    t_bw = sum(e[2].elapsed_time(e[3]) for e in evs) / args.steps
+    total_ms = max_over_ranks(sum(per_step), world, device)
+    ms_per_step = total_ms / args.steps
+
+    # end to end through the public API: pinned host inputs in, results out
+    hX = inp["X"].to(dt).pin_memory()
+    hdY = inp["dY"].to(dt).pin_memory()
+    hY = torch.empty_like(hX).pin_memory()
+    hdX = torch.empty_like(hX).pin_memory()
+    hg = torch.empty_like(gflat, device="cpu").pin_memory()
+    e2e_steps = max(3, min(args.steps, 20))
+
+    def e2e_step():
+        x = hX.to(device, non_blocking=True)
+        dy = hdY.to(device, non_blocking=True)
+        step(None, x, dy, Y, dX)
+        hY.copy_(Y, non_blocking=True)
+        hdX.copy_(dX, non_blocking=True)
+        hg.copy_(gflat, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(device)
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, device) / e2e_steps
+    h2d = 2 * X.numel() * X.element_size()
+    d2h = 2 * X.numel() * X.element_size() + gflat.numel() * 4
+
+    counts = algorithmic_counts(wl)
+    peaks, peak_src = load_peaks()
+    sms = torch.cuda.get_device_properties(device).multi_processor_count
+    sm_max = float(peaks.get("sm_max_mhz", 1965.0))
+    fp32_peak_tflops = sms * FP32_LANES_PER_SM * 2 * sm_max * 1e6 / 1e12
+    hbm_peak = float(peaks["hbm_gbs"])
+    kernels = {"fwd": t_fwd, "bwd_data": t_bd, "bwd_weight": t_bw}
+    dom = max(kernels, key=kernels.get)
+    dom_ms = kernels[dom]
+    achieved_tflops = 2 * counts[dom]["fma"] / (dom_ms * 1e-3) / 1e12
+    step_bytes = sum(c["bytes"] for c in counts.values())
+    hbm_gbs = step_bytes / (ms_per_step * 1e-3) / 1e9
+    traffic = load_traffic(dom, wl.name)
+    line = {
+        "metric": METRIC,
+        "value": world * 1000.0 / ms_per_step,
+        "unit": "steps/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_per_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f32" if wl.io == "f32" else "bf16-io/f32",
+        "data": "synthetic (seeded N(0,1) activations, N(0,1/k^2) weights, U(0.5,1.5) scales)",
+        "config": {"workload": wl.name, **{k: v for k, v in wl.as_dict().items() if k != "name"},
+                   "global_batch": wl.N * world, "parallelism": f"dp{world}",
+                   "l2": "flushed before every timed step (256 MiB write)"},
+        "roofline": {"bound": "alu", "kernel": dom, "achieved": achieved_tflops,
+                     "peak": fp32_peak_tflops, "unit": "TFLOP/s", "frac": achieved_tflops / fp32_peak_tflops,
+                     "traffic": traffic,
+                     "peak_source": f"{sms} SMs x {FP32_LANES_PER_SM} FP32 lanes x 2 x {sm_max:.0f} MHz"},
+        "hbm": {"achieved_gbs": hbm_gbs, "peak_gbs": hbm_peak, "frac": hbm_gbs / hbm_peak,
+                "algorithmic_bytes_per_step": step_bytes, "peak_source": peak_src},
+        "kernels_ms": kernels,
+        "e2e": {"value": world * 1000.0 / e2e_ms, "unit": "steps/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": 4 * args.steps,
+        "clocks": clocks,
+        "wall_s_timed_region": t_wall,
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl, args.cpu_sample_n)
+    return line
+
+
+def load_traffic(kernel, workload):
+    """DRAM bytes per launch from the committed ncu summary, if present."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d.get(workload, {}).get(kernel)
+    except (OSError, ValueError):
+        return None
+
+
+def oracle_step(p):
+    import oracle
+    oracle.forward(p["X"], p["W0"], p["b0"], p["s0"], p["Wl"], p["sl"])
+    oracle.backward(p["X"], p["dY"], p["W0"], p["b0"], p["s0"], p["Wl"], p["sl"])
+
+
+def cpu_baseline(wl, sample_n):
+    """The float64 oracle, as it stands, timed on the host on a bounded
+    sample (the first `sample_n` batch entries of the same workload)."""
+    import dataclasses
+    from depthwise_convolution_wtconv_b200.inputs import as_float64
+    n = max(1, min(sample_n, wl.N))
+    sub = dataclasses.replace(wl, N=n)
+    p = as_float64(make_inputs(sub, 0))
+    t = time.perf_counter()
+    oracle_step(p)
+    dt = time.perf_counter() - t
+    return {"value": (n / wl.N) / dt, "unit": "steps/s", "cores": 1, "kind": "oracle",
+            "sample": f"N={n} of {wl.N} (same C, H, W, k, L), one fwd+bwd in numpy float64, "
+                      f"single-threaded; host has {os.cpu_count()} cores; scaled by {n}/{wl.N}",
+            "seconds": dt}
+
+
+def _plane_sample(wl, planes):
+    """Sub-workload of `planes` (n, c) planes: the first channels of the
+    first batch entries, with every other dimension unchanged."""
+    import dataclasses
+    planes = max(1, min(planes, wl.N * wl.C))
+    if planes >= wl.C:
+        return dataclasses.replace(wl, N=planes // wl.C), (planes // wl.C) * wl.C
+    return dataclasses.replace(wl, N=1, C=planes), planes
+
+
+def run_reference(args, wl, world, rank):
+    """The oracle as the reference arm: rank 0 only, on the host cores.
+    Each step runs the oracle on a bounded plane sample sized so that the
+    whole run stays near two minutes; the rate is scaled to the workload."""
+    if rank != 0:
+        return None
+    from depthwise_convolution_wtconv_b200.inputs import as_float64
+    cal, cal_planes = _plane_sample(wl, min(8, wl.N * wl.C))
+    pc = as_float64(make_inputs(cal, 0))
+    t = time.perf_counter()
+    oracle_step(pc)
+    tau = (time.perf_counter() - t) / cal_planes
+    planes = int(120.0 / max(1e-9, (args.steps + args.warmup) * tau))
+    sub, planes = _plane_sample(wl, planes)
+    p = as_float64(make_inputs(sub, 0))
+    for _ in range(args.warmup):
+        oracle_step(p)
+    t = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_step(p)
+    dt = (time.perf_counter() - t) / args.steps
+    frac = planes / (wl.N * wl.C)
+    value = frac / dt
+    sample = (f"{planes} of {wl.N * wl.C} (n, c) planes per step ({sub.N}x{sub.C}x{wl.H}x{wl.W}), numpy float64, "
+              f"single-threaded, rate scaled by {planes}/{wl.N * wl.C}")
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 / value, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, **{k: v for k, v in wl.as_dict().items() if k != "name"}},
+        "cpu_baseline": {"value": value, "unit": "steps/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=BENCH_WORKLOAD, choices=list(WORKLOADS))
+    ap.add_argument("--cpu-sample-n", type=int, default=32)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    wl = WORKLOADS[args.workload]
+    world, rank, local = setup_dist()
+    try:
+        if args.impl == "reference":
+            line = run_reference(args, wl, world, rank)
+        else:
+            line = run_ours(args, wl, world, rank, local)
+        if rank == 0 and line is not None:
+            print(json.dumps(line), flush=True)
+    finally:
+        if dist.is_initialized():
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

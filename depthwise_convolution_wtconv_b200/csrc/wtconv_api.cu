@@ -1,0 +1,423 @@
+// C ABI of libwtconv: argument checks, shared-memory plans and launches.
+// The operations and their definitions are documented in include/wtconv.h.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <initializer_list>
+
+#include "wtconv.h"
+#include "wtconv_kernels.cuh"
+
+namespace wt {
+namespace {
+
+inline int rup(int a, int b) { return (a + b - 1) / b * b; }
+
+struct TileShape {
+  int R, CW;
+};
+
+// Shifted buffer able to serve register tiles of every listed shape.
+BufDesc make_shifted(int& cur, int h, int w, int r, std::initializer_list<TileShape> shapes, int nb) {
+  int rows = h + 2 * r, ld = w + 2 * r;
+  for (const TileShape& s : shapes) {
+    const int nv = (s.CW + 2 * r + 3) / 4;
+    rows = std::max(rows, rup(h, s.R) + 2 * r);
+    ld = std::max(ld, rup(w, s.CW) - s.CW + nv * 4);
+  }
+  ld = rup(ld, 4);
+  BufDesc d{cur, ld, rows, 0};
+  cur += rup(ld * rows * nb, 4);
+  return d;
+}
+
+BufDesc make_plain(int& cur, int h, int w, std::initializer_list<TileShape> shapes, int nb) {
+  int rows = h, ld = w;
+  for (const TileShape& s : shapes) {
+    rows = std::max(rows, rup(h, s.R));
+    ld = std::max(ld, rup(w, s.CW));
+  }
+  ld = rup(ld, 4);
+  BufDesc d{cur, ld, rows, 0};
+  cur += rup(ld * rows * nb, 4);
+  return d;
+}
+
+void relocate(BufDesc& d, int base, int slab) {
+  d.off += base;
+  d.ps = slab;
+}
+
+int io_bytes(const wtconv_desc* d) { return d->io == WTCONV_BF16 ? 2 : 4; }
+
+void fill_common(Plan& P, const wtconv_desc* d) {
+  P = Plan{};
+  P.N = d->N;
+  P.C = d->C;
+  P.H = d->H;
+  P.W = d->W;
+  P.K = d->k;
+  P.r = d->k / 2;
+  P.L = d->L;
+  P.H1 = d->L >= 1 ? d->H / 2 : d->H;
+  P.W1 = d->L >= 1 ? d->W / 2 : d->W;
+  P.kk4 = rup(d->k * d->k, 4);
+  P.vec_in = (d->W % 4) == 0;
+  P.vec_out = d->io == WTCONV_BF16 ? (d->W % 8) == 0 : (d->W % 4) == 0;
+  P.V = d->k * d->k * (1 + 4 * d->L) + 1;
+}
+
+// Per-plane slab of the forward / backward-data kernel.
+int forward_slab(Plan& P) {
+  const int r = P.r, L = P.L;
+  int cur = 0;
+  P.xf = make_shifted(cur, P.H, P.W, r, {{P.R3, C3_CW}}, 1);
+  if (L >= 1) P.s1 = make_shifted(cur, P.H1, P.W1, r, {{C2_R, C2_CW}, {2, 2}}, 4);
+  if (L >= 2) P.t1 = make_plain(cur, P.H1, P.W1, {{C2_R, C2_CW}, {2 * DP_R, 2 * DP_CW}}, 1);
+  const int region = cur;
+  if (L >= 1) P.zb = make_plain(cur, P.H1, P.W1, {{C2_R, C2_CW}, {P.R3 / 2, C3_CW / 2}}, 4);
+  const int end1 = cur;
+  cur = region;
+  if (L >= 2) {
+    for (int l = 2; l <= L; ++l) P.sd[l] = make_shifted(cur, P.H >> l, P.W >> l, r, {{DP_R, DP_CW}, {2, 2}}, 4);
+    for (int l = 3; l <= L; ++l) P.zd[l] = make_plain(cur, P.H >> l, P.W >> l, {{DP_R, DP_CW}}, 4);
+    if (L >= 3) P.t2 = make_plain(cur, P.H >> 2, P.W >> 2, {{DP_R, DP_CW}}, 1);
+  }
+  P.deep_off = region;
+  P.deep_floats = cur - region;
+  return rup(std::max(end1, cur), 4);
+}
+
+void finish_forward_plan(Plan& P, int PB) {
+  const int slab = forward_slab(P);
+  P.PB = PB;
+  P.nbatch = (P.N + PB - 1) / PB;
+  P.w_off = 0;
+  const int base = rup((1 + 4 * P.L) * P.kk4 + 4, 4);
+  for (BufDesc* b : {&P.xf, &P.s1, &P.t1, &P.zb, &P.t2}) relocate(*b, base, slab);
+  for (int l = 0; l <= MAXL; ++l) {
+    relocate(P.sd[l], base, slab);
+    relocate(P.zd[l], base, slab);
+  }
+  P.deep_off += base;
+  P.smem_floats = base + PB * slab;
+}
+
+// Tiles of the output pass per plane, for the batch-size choice.
+int output_items(const Plan& P, int R3) { return ((P.H + R3 - 1) / R3) * ((P.W + C3_CW - 1) / C3_CW); }
+
+void build_forward_plan(Plan& P, const wtconv_desc* d, int max_smem) {
+  fill_common(P, d);
+  P.R3 = output_items(P, 4) >= NT / 2 ? 4 : 2;
+  const int items = output_items(P, P.R3);
+  int PB = std::max(1, std::min(d->N, (NT + items - 1) / items));
+  for (;;) {
+    finish_forward_plan(P, PB);
+    if (PB == 1 || (size_t)P.smem_floats * 4 <= (size_t)max_smem / 2) break;
+    --PB;
+  }
+}
+
+int bwdw_slab(Plan& P) {
+  const int r = P.r, L = P.L;
+  int cur = 0;
+  P.xf = make_shifted(cur, P.H, P.W, r, {{BW_R, BW_CW}}, 1);
+  P.gf = make_plain(cur, P.H, P.W, {{BW_R, BW_CW}}, 1);
+  if (L >= 1) {
+    P.s1 = make_shifted(cur, P.H1, P.W1, r, {{B1_R, B1_CW}, {2, 2}}, 4);
+    P.g1 = make_plain(cur, P.H1, P.W1, {{B1_R, B1_CW}, {2, 2}}, 4);
+  }
+  for (int l = 2; l <= L; ++l) {
+    P.sd[l] = make_shifted(cur, P.H >> l, P.W >> l, r, {{DP_R, DP_CW}, {2, 2}}, 4);
+    P.gd[l] = make_plain(cur, P.H >> l, P.W >> l, {{DP_R, DP_CW}, {2, 2}}, 4);
+  }
+  return rup(cur, 4);
+}
+
+void finish_bwdw_plan(Plan& P, int PB) {
+  const int slab = bwdw_slab(P);
+  P.PB = PB;
+  const int ndeep = P.L >= 2 ? (P.L - 1) * 4 : 0;
+  P.gdeep_off = 0;
+  P.dpart_off = ndeep * P.kk4;
+  const int base = rup(P.dpart_off + ndeep * DSLOTS * P.kk4, 4);
+  for (BufDesc* b : {&P.xf, &P.gf, &P.s1, &P.g1}) relocate(*b, base, slab);
+  for (int l = 0; l <= MAXL; ++l) {
+    relocate(P.sd[l], base, slab);
+    relocate(P.gd[l], base, slab);
+  }
+  P.red_off = base;
+  P.smem_floats = std::max(base + PB * slab, base + NT * P.kk4 + NT);
+}
+
+void build_bwdw_plan(Plan& P, const wtconv_desc* d, int max_smem) {
+  fill_common(P, d);
+  P.R3 = 2;
+  const int items = ((P.H + BW_R - 1) / BW_R) * ((P.W + BW_CW - 1) / BW_CW);
+  const int nbase = P.L >= 1 ? 128 : NT;
+  int PB = std::max(1, std::min(d->N, (nbase + items - 1) / items));
+  for (;;) {
+    finish_bwdw_plan(P, PB);
+    if (PB == 1 || (size_t)P.smem_floats * 4 <= (size_t)max_smem / 2) break;
+    --PB;
+  }
+}
+
+wtconv_status check_desc(const wtconv_desc* d) {
+  if (!d) return WTCONV_ERR_ARG;
+  if (d->k < 1 || d->k > WTCONV_MAX_K || (d->k % 2) == 0) return WTCONV_ERR_ARG;
+  if (d->L < 0 || d->L > WTCONV_MAX_LEVELS) return WTCONV_ERR_ARG;
+  if (d->N <= 0 || d->C <= 0 || d->H <= 0 || d->W <= 0) return WTCONV_ERR_ARG;
+  if (d->io != WTCONV_F32 && d->io != WTCONV_BF16) return WTCONV_ERR_ARG;
+  if ((long long)d->H * d->W > (1LL << 30) || (long long)d->N * d->C > (1LL << 30)) return WTCONV_ERR_ARG;
+  const int m = 1 << d->L;
+  if ((d->H % m) != 0 || (d->W % m) != 0) return WTCONV_ERR_SHAPE;
+  return WTCONV_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+wtconv_status check_params(const wtconv_desc* d, const float* w0, const float* b0, const float* s0,
+                           const float* wl, const float* sl, bool need_b0) {
+  if (!w0 || !s0 || (need_b0 && !b0)) return WTCONV_ERR_ARG;
+  if (d->L > 0 && (!wl || !sl)) return WTCONV_ERR_ARG;
+  if (!aligned4(w0) || !aligned4(s0) || (b0 && !aligned4(b0))) return WTCONV_ERR_ALIGN;
+  if (d->L > 0 && (!aligned4(wl) || !aligned4(sl))) return WTCONV_ERR_ALIGN;
+  return WTCONV_OK;
+}
+
+struct Device {
+  int sms = 0, max_smem = 0;
+};
+
+wtconv_status query_device(Device& dev) {
+  int id = 0;
+  if (cudaGetDevice(&id) != cudaSuccess) return WTCONV_ERR_CUDA;
+  if (cudaDeviceGetAttribute(&dev.sms, cudaDevAttrMultiProcessorCount, id) != cudaSuccess) return WTCONV_ERR_CUDA;
+  if (cudaDeviceGetAttribute(&dev.max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, id) != cudaSuccess)
+    return WTCONV_ERR_CUDA;
+  return WTCONV_OK;
+}
+
+template <typename F>
+wtconv_status prepare(F kern, size_t smem, int& occ) {
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return WTCONV_ERR_CUDA;
+  occ = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, NT, smem) != cudaSuccess) return WTCONV_ERR_CUDA;
+  if (occ < 1) return WTCONV_ERR_UNSUPPORTED;
+  return WTCONV_OK;
+}
+
+template <int K, int R3, typename IO>
+wtconv_status launch_fwd_t(const Plan& P, const Device& dev, const void* x, const float* w0, const float* b0,
+                           const float* s0, const float* wl, const float* sl, void* y, int flip,
+                           cudaStream_t st) {
+  auto kern = wtconv_fwd_kernel<K, R3, IO>;
+  const size_t smem = (size_t)P.smem_floats * 4;
+  int occ = 0;
+  wtconv_status e = prepare(kern, smem, occ);
+  if (e != WTCONV_OK) return e;
+  const int units = P.C * P.nbatch;
+  const int grid = std::min(units, dev.sms * occ);
+  kern<<<grid, NT, smem, st>>>(P, static_cast<const IO*>(x), w0, b0, s0, wl, sl, static_cast<IO*>(y), flip);
+  return cudaGetLastError() == cudaSuccess ? WTCONV_OK : WTCONV_ERR_CUDA;
+}
+
+template <int K>
+wtconv_status launch_fwd_k(const Plan& P, const Device& dev, wtconv_dtype io, const void* x, const float* w0,
+                           const float* b0, const float* s0, const float* wl, const float* sl, void* y, int flip,
+                           cudaStream_t st) {
+  if (io == WTCONV_F32) {
+    if (P.R3 == 4) return launch_fwd_t<K, 4, float>(P, dev, x, w0, b0, s0, wl, sl, y, flip, st);
+    return launch_fwd_t<K, 2, float>(P, dev, x, w0, b0, s0, wl, sl, y, flip, st);
+  }
+  if (P.R3 == 4) return launch_fwd_t<K, 4, __nv_bfloat16>(P, dev, x, w0, b0, s0, wl, sl, y, flip, st);
+  return launch_fwd_t<K, 2, __nv_bfloat16>(P, dev, x, w0, b0, s0, wl, sl, y, flip, st);
+}
+
+wtconv_status run_forward(const wtconv_desc* d, const void* x, const float* w0, const float* b0, const float* s0,
+                          const float* wl, const float* sl, void* y, int flip, cudaStream_t st) {
+  Device dev;
+  wtconv_status e = query_device(dev);
+  if (e != WTCONV_OK) return e;
+  Plan P;
+  build_forward_plan(P, d, dev.max_smem);
+  if ((size_t)P.smem_floats * 4 > (size_t)dev.max_smem) return WTCONV_ERR_UNSUPPORTED;
+  switch (d->k) {
+    case 1: return launch_fwd_k<1>(P, dev, d->io, x, w0, b0, s0, wl, sl, y, flip, st);
+    case 3: return launch_fwd_k<3>(P, dev, d->io, x, w0, b0, s0, wl, sl, y, flip, st);
+    case 5: return launch_fwd_k<5>(P, dev, d->io, x, w0, b0, s0, wl, sl, y, flip, st);
+    default: return launch_fwd_k<7>(P, dev, d->io, x, w0, b0, s0, wl, sl, y, flip, st);
+  }
+}
+
+size_t bwdw_ws_bytes(const wtconv_desc* d) {
+  const size_t V = (size_t)d->k * d->k * (1 + 4 * d->L) + 1;
+  return (size_t)d->N * d->C * V * sizeof(float);
+}
+
+template <int K, typename IO>
+wtconv_status launch_bwdw_t(Plan& P, const Device& dev, const void* x, const void* dy, const float* w0,
+                            const float* b0, const float* s0, const float* wl, const float* sl, float* dw0,
+                            float* db0, float* ds0, float* dwl, float* dsl, float* part, cudaStream_t st) {
+  auto kern = wtconv_bwdw_kernel<K, IO>;
+  const size_t smem = (size_t)P.smem_floats * 4;
+  int occ = 0;
+  wtconv_status e = prepare(kern, smem, occ);
+  if (e != WTCONV_OK) return e;
+  const int slots = dev.sms * occ;
+  int groups = std::max(1, std::min(P.N, slots / P.C));
+  P.planes_per_cta = (P.N + groups - 1) / groups;
+  P.ngroups = (P.N + P.planes_per_cta - 1) / P.planes_per_cta;
+  kern<<<P.C * P.ngroups, NT, smem, st>>>(P, static_cast<const IO*>(x), static_cast<const IO*>(dy), part);
+  if (cudaGetLastError() != cudaSuccess) return WTCONV_ERR_CUDA;
+  const size_t fsmem = (size_t)P.V * sizeof(float);
+  auto fin = wtconv_bwdw_finalize<K>;
+  if (fsmem > 48 * 1024 &&
+      cudaFuncSetAttribute(fin, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fsmem) != cudaSuccess)
+    return WTCONV_ERR_CUDA;
+  fin<<<P.C, 128, fsmem, st>>>(P, part, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl);
+  return cudaGetLastError() == cudaSuccess ? WTCONV_OK : WTCONV_ERR_CUDA;
+}
+
+template <int K>
+wtconv_status launch_bwdw_k(Plan& P, const Device& dev, wtconv_dtype io, const void* x, const void* dy,
+                            const float* w0, const float* b0, const float* s0, const float* wl, const float* sl,
+                            float* dw0, float* db0, float* ds0, float* dwl, float* dsl, float* part,
+                            cudaStream_t st) {
+  if (io == WTCONV_F32)
+    return launch_bwdw_t<K, float>(P, dev, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, part, st);
+  return launch_bwdw_t<K, __nv_bfloat16>(P, dev, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, part, st);
+}
+
+wtconv_status run_bwdw(const wtconv_desc* d, const void* x, const void* dy, const float* w0, const float* b0,
+                       const float* s0, const float* wl, const float* sl, float* dw0, float* db0, float* ds0,
+                       float* dwl, float* dsl, void* ws, cudaStream_t st) {
+  Device dev;
+  wtconv_status e = query_device(dev);
+  if (e != WTCONV_OK) return e;
+  Plan P;
+  build_bwdw_plan(P, d, dev.max_smem);
+  if ((size_t)P.smem_floats * 4 > (size_t)dev.max_smem) return WTCONV_ERR_UNSUPPORTED;
+  float* part = static_cast<float*>(ws);
+  switch (d->k) {
+    case 1: return launch_bwdw_k<1>(P, dev, d->io, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, part, st);
+    case 3: return launch_bwdw_k<3>(P, dev, d->io, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, part, st);
+    case 5: return launch_bwdw_k<5>(P, dev, d->io, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, part, st);
+    default: return launch_bwdw_k<7>(P, dev, d->io, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, part, st);
+  }
+}
+
+wtconv_status check_ws(void* ws, size_t ws_bytes, size_t need) {
+  if (need == 0) return WTCONV_OK;
+  if (!ws || ws_bytes < need) return WTCONV_ERR_WORKSPACE;
+  if (!aligned16(ws)) return WTCONV_ERR_ALIGN;
+  return WTCONV_OK;
+}
+
+wtconv_status check_grad_outputs(const wtconv_desc* d, const float* dw0, const float* db0, const float* ds0,
+                                 const float* dwl, const float* dsl) {
+  if (!dw0 || !db0 || !ds0) return WTCONV_ERR_ARG;
+  if (d->L > 0 && (!dwl || !dsl)) return WTCONV_ERR_ARG;
+  if (!aligned4(dw0) || !aligned4(db0) || !aligned4(ds0)) return WTCONV_ERR_ALIGN;
+  if (d->L > 0 && (!aligned4(dwl) || !aligned4(dsl))) return WTCONV_ERR_ALIGN;
+  return WTCONV_OK;
+}
+
+}  // namespace
+}  // namespace wt
+
+using namespace wt;
+
+extern "C" {
+
+size_t wtconv_workspace_size(const wtconv_desc* desc, int op) {
+  if (check_desc(desc) != WTCONV_OK) return 0;
+  switch (op) {
+    case WTCONV_OP_FORWARD:
+    case WTCONV_OP_BACKWARD_DATA:
+      return 0;
+    case WTCONV_OP_BACKWARD_WEIGHT:
+    case WTCONV_OP_BACKWARD:
+      return bwdw_ws_bytes(desc);
+    default:
+      return 0;
+  }
+}
+
+wtconv_status wtconv_forward(const wtconv_desc* desc, const void* x, const float* w0, const float* b0,
+                             const float* s0, const float* wl, const float* sl, void* y, void* ws,
+                             size_t ws_bytes, void* stream) {
+  wtconv_status e = check_desc(desc);
+  if (e != WTCONV_OK) return e;
+  if (!x || !y) return WTCONV_ERR_ARG;
+  if ((e = check_params(desc, w0, b0, s0, wl, sl, true)) != WTCONV_OK) return e;
+  if (!aligned16(x) || !aligned16(y)) return WTCONV_ERR_ALIGN;
+  (void)ws;
+  (void)ws_bytes;
+  return run_forward(desc, x, w0, b0, s0, wl, sl, y, 0, static_cast<cudaStream_t>(stream));
+}
+
+wtconv_status wtconv_backward_data(const wtconv_desc* desc, const void* dy, const float* w0, const float* s0,
+                                   const float* wl, const float* sl, void* dx, void* ws, size_t ws_bytes,
+                                   void* stream) {
+  wtconv_status e = check_desc(desc);
+  if (e != WTCONV_OK) return e;
+  if (!dy || !dx) return WTCONV_ERR_ARG;
+  if ((e = check_params(desc, w0, nullptr, s0, wl, sl, false)) != WTCONV_OK) return e;
+  if (!aligned16(dy) || !aligned16(dx)) return WTCONV_ERR_ALIGN;
+  (void)ws;
+  (void)ws_bytes;
+  return run_forward(desc, dy, w0, nullptr, s0, wl, sl, dx, 1, static_cast<cudaStream_t>(stream));
+}
+
+wtconv_status wtconv_backward_weight(const wtconv_desc* desc, const void* x, const void* dy, const float* w0,
+                                     const float* b0, const float* s0, const float* wl, const float* sl,
+                                     float* dw0, float* db0, float* ds0, float* dwl, float* dsl, void* ws,
+                                     size_t ws_bytes, void* stream) {
+  wtconv_status e = check_desc(desc);
+  if (e != WTCONV_OK) return e;
+  if (!x || !dy) return WTCONV_ERR_ARG;
+  if ((e = check_params(desc, w0, b0, s0, wl, sl, true)) != WTCONV_OK) return e;
+  if ((e = check_grad_outputs(desc, dw0, db0, ds0, dwl, dsl)) != WTCONV_OK) return e;
+  if (!aligned16(x) || !aligned16(dy)) return WTCONV_ERR_ALIGN;
+  if ((e = check_ws(ws, ws_bytes, bwdw_ws_bytes(desc))) != WTCONV_OK) return e;
+  return run_bwdw(desc, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, ws,
+                  static_cast<cudaStream_t>(stream));
+}
+
+wtconv_status wtconv_backward(const wtconv_desc* desc, const void* x, const void* dy, const float* w0,
+                              const float* b0, const float* s0, const float* wl, const float* sl, void* dx,
+                              float* dw0, float* db0, float* ds0, float* dwl, float* dsl, void* ws,
+                              size_t ws_bytes, void* stream) {
+  wtconv_status e = check_desc(desc);
+  if (e != WTCONV_OK) return e;
+  if (!x || !dy || !dx) return WTCONV_ERR_ARG;
+  if ((e = check_params(desc, w0, b0, s0, wl, sl, true)) != WTCONV_OK) return e;
+  if ((e = check_grad_outputs(desc, dw0, db0, ds0, dwl, dsl)) != WTCONV_OK) return e;
+  if (!aligned16(x) || !aligned16(dy) || !aligned16(dx)) return WTCONV_ERR_ALIGN;
+  if ((e = check_ws(ws, ws_bytes, bwdw_ws_bytes(desc))) != WTCONV_OK) return e;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  e = run_forward(desc, dy, w0, nullptr, s0, wl, sl, dx, 1, st);
+  if (e != WTCONV_OK) return e;
+  return run_bwdw(desc, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, ws, st);
+}
+
+const char* wtconv_status_string(wtconv_status s) {
+  switch (s) {
+    case WTCONV_OK: return "ok";
+    case WTCONV_ERR_ARG: return "invalid argument";
+    case WTCONV_ERR_SHAPE: return "H or W not divisible by 2^L";
+    case WTCONV_ERR_ALIGN: return "pointer not aligned (16 bytes for tensors and workspace)";
+    case WTCONV_ERR_WORKSPACE: return "workspace missing or too small";
+    case WTCONV_ERR_CUDA: return "CUDA error at launch";
+    case WTCONV_ERR_UNSUPPORTED: return "shape needs more shared memory than one SM offers";
+    default: return "unknown status";
+  }
+}
+
+}  // extern "C"

@@ -1,0 +1,149 @@
+/*
+ * wtconv.h -- C ABI of the B200 (sm_100a) WTConv layer library (libwtconv.so).
+ *
+ * The layer (source: "I/O-aware reformulation of wavelet convolution",
+ * arXiv:2608.10805, abstract): a multi-level 2-D Haar wavelet decomposition
+ * of each input channel, a k x k depthwise convolution with a learned
+ * per-channel scale on every subband at every level, the multi-level
+ * synthesis cascade back to full resolution, added to a scaled base k x k
+ * depthwise convolution of the input.  With L = 0 it is a plain depthwise
+ * convolution (with bias and per-channel scale).
+ *
+ * Definitions (all entry points follow them exactly, up to fp32 rounding):
+ *   dwconv(A, W)[c,i,j] = sum_{u,v<k} W[c,u,v] * A[c, i+u-r, j+v-r],
+ *       r = (k-1)/2, zero outside the image (cross-correlation, 'same').
+ *   Haar of the 2x2 block a=(2i,2j) b=(2i,2j+1) c=(2i+1,2j) d=(2i+1,2j+1):
+ *       LL=(a+b+c+d)/2  LH=(a+b-c-d)/2  HL=(a-b+c-d)/2  HH=(a-b-c+d)/2
+ *   IWT is its inverse (and transpose).
+ *   Ybase = s0[c] * (dwconv(X, W0)[c] + b0[c])
+ *   cur = X; for l = 1..L: sub_l = Haar(cur) (bands LL,LH,HL,HH);
+ *       Z_l[c,s] = sl[l][c][s] * dwconv(sub_l[c,s], Wl[l][c][s]); cur = raw LL.
+ *   t = 0; for l = L..1: t = IWT(Z_l with t added to its LL band)
+ *   Y = Ybase + t
+ *
+ * Layouts (all contiguous, row-major):
+ *   x, y, dy, dx : [N][C][H][W] in the I/O dtype (fp32 or bf16)
+ *   w0 : [C][k][k] fp32      b0, s0 : [C] fp32
+ *   wl : [L][C][4][k][k] fp32 (band order LL, LH, HL, HH)
+ *   sl : [L][C][4] fp32
+ *
+ * Conventions shared by every entry point:
+ *   - Every tensor pointer is caller-owned DEVICE memory; the library never
+ *     allocates, frees or keeps state between calls.  Calls are asynchronous
+ *     on `stream` (a cudaStream_t; NULL = legacy default stream) and never
+ *     synchronise.
+ *   - Arithmetic is fp32 throughout; bf16 I/O is rounded to nearest even on
+ *     output.  Results are deterministic run to run (fixed reduction order).
+ *   - Gradients are overwritten, not accumulated.
+ *   - Argument checks happen on the host before any launch:
+ *       WTCONV_ERR_ARG       null desc/pointer, k even or outside 1..7,
+ *                            L < 0 or L > WTCONV_MAX_LEVELS, N,C,H,W <= 0,
+ *                            element counts that overflow 32-bit indexing
+ *       WTCONV_ERR_SHAPE     H or W not divisible by 2^L
+ *       WTCONV_ERR_ALIGN     a tensor pointer not 16-byte aligned
+ *       WTCONV_ERR_WORKSPACE ws_bytes < wtconv_workspace_size(desc, op)
+ *       WTCONV_ERR_UNSUPPORTED  the shape needs more on-chip memory than
+ *                            one SM offers
+ *     and WTCONV_ERR_CUDA reports a launch failure (cudaGetLastError).
+ *     Nothing is launched when a check fails.  No device-side trap exists.
+ *   - With L = 0, wl and sl may be NULL.
+ */
+#ifndef WTCONV_H
+#define WTCONV_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define WTCONV_MAX_LEVELS 8
+#define WTCONV_MAX_K 7
+
+typedef enum { WTCONV_F32 = 0, WTCONV_BF16 = 1 } wtconv_dtype;
+
+/* Layer shape: batch N, channels C, image H x W, kernel size k (odd),
+ * levels L, I/O dtype of x, y, dy, dx. */
+typedef struct {
+  int N, C, H, W, k, L;
+  wtconv_dtype io;
+} wtconv_desc;
+
+typedef enum {
+  WTCONV_OK = 0,
+  WTCONV_ERR_ARG = 1,
+  WTCONV_ERR_SHAPE = 2,
+  WTCONV_ERR_ALIGN = 3,
+  WTCONV_ERR_WORKSPACE = 4,
+  WTCONV_ERR_CUDA = 5,
+  WTCONV_ERR_UNSUPPORTED = 6
+} wtconv_status;
+
+/* Operation codes for wtconv_workspace_size. */
+enum {
+  WTCONV_OP_FORWARD = 0,
+  WTCONV_OP_BACKWARD_DATA = 1,
+  WTCONV_OP_BACKWARD_WEIGHT = 2,
+  WTCONV_OP_BACKWARD = 3
+};
+
+/* Bytes of device workspace the operation `op` needs for `desc` (0 when it
+ * needs none, or when desc is invalid).  The weight-gradient pass keeps its
+ * per-CTA partial sums there before the fixed-order second stage. */
+size_t wtconv_workspace_size(const wtconv_desc* desc, int op);
+
+/* Forward pass: y = WTConv(x).  Source: arXiv:2608.10805, abstract (the
+ * layer; reformulations (1) on-chip Haar analysis, (2) single-pass
+ * synthesis indexed by output-coordinate bits, (3) scales folded into the
+ * convolution weights).  b0, s0 and w0 are required; wl, sl when L > 0.
+ * ws may be NULL when wtconv_workspace_size(desc, 0) == 0. */
+wtconv_status wtconv_forward(const wtconv_desc* desc, const void* x,
+                             const float* w0, const float* b0, const float* s0,
+                             const float* wl, const float* sl, void* y,
+                             void* ws, size_t ws_bytes, void* stream);
+
+/* Backward data pass: dx = J^T dy, the adjoint of the forward map in x.
+ * The adjoint of the +-1/2 Haar analysis is the synthesis and vice versa,
+ * and the adjoint of each depthwise conv is the correlation with its
+ * spatially flipped kernel, so this is the forward pass run on dy with
+ * flipped kernels and no bias (arXiv:2608.10805, abstract: training). */
+wtconv_status wtconv_backward_data(const wtconv_desc* desc, const void* dy,
+                                   const float* w0, const float* s0,
+                                   const float* wl, const float* sl, void* dx,
+                                   void* ws, size_t ws_bytes, void* stream);
+
+/* Backward weight pass: gradients of <y, dy> with respect to every
+ * parameter, with G_0[c,u,v] = sum_{n,i,j} dy[n,c,i,j] x[n,c,i+u-r,j+v-r]
+ * and G_l[c,s,u,v] = sum dZ_l[c,s](i,j) sub_l[c,s](i+u-r,j+v-r), where
+ * dZ_l = Haar pyramid of dy and sub_l = Haar pyramid of x:
+ *   dw0 = s0 G_0   db0 = s0 sum(dy)   ds0 = sum_uv w0 G_0 + b0 sum(dy)
+ *   dwl = sl G_l   dsl = sum_uv wl G_l
+ * Outputs dw0 [C][k][k], db0 [C], ds0 [C], dwl [L][C][4][k][k], dsl [L][C][4]
+ * (fp32, overwritten).  Needs wtconv_workspace_size(desc, 2) bytes of ws. */
+wtconv_status wtconv_backward_weight(const wtconv_desc* desc, const void* x,
+                                     const void* dy, const float* w0,
+                                     const float* b0, const float* s0,
+                                     const float* wl, const float* sl,
+                                     float* dw0, float* db0, float* ds0,
+                                     float* dwl, float* dsl, void* ws,
+                                     size_t ws_bytes, void* stream);
+
+/* Both backward passes in one call (dx and every parameter gradient), as
+ * wtconv_backward_data followed by wtconv_backward_weight but sharing the
+ * reads of x and dy where the shape allows.  Needs
+ * wtconv_workspace_size(desc, 3) bytes of ws. */
+wtconv_status wtconv_backward(const wtconv_desc* desc, const void* x,
+                              const void* dy, const float* w0, const float* b0,
+                              const float* s0, const float* wl, const float* sl,
+                              void* dx, float* dw0, float* db0, float* ds0,
+                              float* dwl, float* dsl, void* ws, size_t ws_bytes,
+                              void* stream);
+
+/* Static description of a status code (never NULL). */
+const char* wtconv_status_string(wtconv_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* WTCONV_H */

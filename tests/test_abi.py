@@ -1,0 +1,127 @@
+"""C-ABI checks that need no GPU: the library loads, exports every declared
+entry point, and rejects bad arguments on the host before any launch."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+import depthwise_convolution_wtconv_b200 as wt
+from depthwise_convolution_wtconv_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "wtconv.h")
+
+OK, ARG, SHAPE, ALIGN, WS = 0, 1, 2, 3, 4
+FAKE = 0x10000          # 16-byte aligned address that is never dereferenced
+FAKE_MIS = 0x10004      # misaligned
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return wt.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^\s*(?:const char\*|size_t|wtconv_status)\s+(wtconv_\w+)\s*\(", text, re.M)))
+
+
+def test_header_declares_the_binding_exports():
+    assert declared_functions() == sorted(_lib.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(lib):
+    for s in range(7):
+        assert lib.wtconv_status_string(s)
+    assert lib.wtconv_status_string(99) == b"unknown status"
+
+
+def _desc(N=2, C=3, H=16, W=16, k=5, L=2, io=0):
+    return _lib.WTConvDesc(N, C, H, W, k, L, io)
+
+
+def test_workspace_sizes(lib):
+    d = _desc()
+    V = 25 * (1 + 4 * 2) + 1
+    assert lib.wtconv_workspace_size(ctypes.byref(d), 0) == 0
+    assert lib.wtconv_workspace_size(ctypes.byref(d), 1) == 0
+    assert lib.wtconv_workspace_size(ctypes.byref(d), 2) == 2 * 3 * V * 4
+    assert lib.wtconv_workspace_size(ctypes.byref(d), 3) == 2 * 3 * V * 4
+    assert lib.wtconv_workspace_size(ctypes.byref(_desc(k=4)), 2) == 0
+    assert lib.wtconv_workspace_size(None, 2) == 0
+
+
+def _fwd(lib, d, x=FAKE, y=FAKE, w0=FAKE, b0=FAKE, s0=FAKE, wl=FAKE, sl=FAKE):
+    return lib.wtconv_forward(ctypes.byref(d) if d is not None else None, x, w0, b0, s0, wl, sl, y, None, 0, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(k=4), ARG), (dict(k=9), ARG), (dict(k=0), ARG), (dict(L=-1), ARG), (dict(L=9), ARG),
+    (dict(N=0), ARG), (dict(C=-1), ARG), (dict(H=0), ARG), (dict(io=7), ARG),
+    (dict(H=18, L=2), SHAPE), (dict(W=20, L=3), SHAPE), (dict(H=3, W=4, L=1), SHAPE),
+])
+def test_forward_rejects_bad_descriptors(lib, kw, status):
+    assert _fwd(lib, _desc(**kw)) == status
+
+
+def test_forward_rejects_null_and_misaligned(lib):
+    assert _fwd(lib, None) == ARG
+    assert _fwd(lib, _desc(), x=None) == ARG
+    assert _fwd(lib, _desc(), w0=None) == ARG
+    assert _fwd(lib, _desc(), b0=None) == ARG
+    assert _fwd(lib, _desc(), wl=None) == ARG
+    assert _fwd(lib, _desc(), x=FAKE_MIS) == ALIGN
+    assert _fwd(lib, _desc(), y=FAKE + 8) == ALIGN
+    assert _fwd(lib, _desc(), w0=FAKE + 2) == ALIGN
+
+
+def test_level0_allows_null_level_params(lib):
+    # L = 0 with NULL wl/sl passes every host check; with the fake pointers a
+    # compute call would follow, so only a bad descriptor is tried here.
+    assert _fwd(lib, _desc(L=0, k=2), wl=None, sl=None) == ARG
+
+
+def test_backward_data_checks(lib):
+    d = _desc()
+    f = lib.wtconv_backward_data
+    assert f(ctypes.byref(d), None, FAKE, FAKE, FAKE, FAKE, FAKE, None, 0, None) == ARG
+    assert f(ctypes.byref(d), FAKE_MIS, FAKE, FAKE, FAKE, FAKE, FAKE, None, 0, None) == ALIGN
+    assert f(ctypes.byref(_desc(W=10, L=2)), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, 0, None) == SHAPE
+
+
+def test_backward_weight_checks_workspace(lib):
+    d = _desc()
+    need = lib.wtconv_workspace_size(ctypes.byref(d), 2)
+    f = lib.wtconv_backward_weight
+    args = [FAKE] * 12
+    assert f(ctypes.byref(d), *args, None, need, None) == WS
+    assert f(ctypes.byref(d), *args, FAKE, need - 4, None) == WS
+    assert f(ctypes.byref(d), *args, FAKE + 4, need, None) == ALIGN
+    bad = list(args)
+    bad[7] = None  # dw0
+    assert f(ctypes.byref(d), *bad, FAKE, need, None) == ARG
+
+
+def test_backward_checks(lib):
+    d = _desc()
+    need = lib.wtconv_workspace_size(ctypes.byref(d), 3)
+    f = lib.wtconv_backward
+    args = [FAKE] * 13
+    assert f(ctypes.byref(d), *args, None, need, None) == WS
+    bad = list(args)
+    bad[7] = None  # dx
+    assert f(ctypes.byref(d), *bad, FAKE, need, None) == ARG
+
+
+def test_python_binding_refuses_cpu_tensors():
+    x = torch.zeros(1, 1, 4, 4)
+    w = torch.zeros(1, 3, 3)
+    with pytest.raises(TypeError):
+        wt.forward(x, w, torch.zeros(1), torch.ones(1))

@@ -1,0 +1,189 @@
+"""Parity of the CUDA library (through its C ABI) with the float64 oracle.
+
+Tolerances (per tensor, normwise): fp32 I/O max|gpu - oracle| / max|oracle|
+<= 1e-4; bf16 I/O <= 2e-2 of the oracle's max-abs.  The oracle sees the
+exact bf16 values of bf16 inputs.
+"""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import depthwise_convolution_wtconv_b200 as wt
+from depthwise_convolution_wtconv_b200.configs import WORKLOADS, Workload
+from depthwise_convolution_wtconv_b200.inputs import make_inputs, as_float64
+
+pytestmark = pytest.mark.gpu
+
+TOL = {"f32": 1e-4, "bf16": 2e-2}
+
+
+def _dev(inp, io):
+    dt = torch.float32 if io == "f32" else torch.bfloat16
+    d = {}
+    for k, v in inp.items():
+        if k in ("X", "dY"):
+            d[k] = v.to(dt).cuda().contiguous()
+        else:
+            d[k] = v.cuda().contiguous()
+    if d["Wl"].numel() == 0:
+        d["Wl"] = None
+        d["sl"] = None
+    return d
+
+
+def _rel(gpu, ref):
+    gpu = np.asarray(gpu, dtype=np.float64)
+    scale = max(np.max(np.abs(ref)), 1e-30)
+    return float(np.max(np.abs(gpu - ref)) / scale)
+
+
+def _np(t):
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def run_gpu(d):
+    y = wt.forward(d["X"], d["W0"], d["b0"], d["s0"], d["Wl"], d["sl"])
+    dx = wt.backward_data(d["dY"], d["W0"], d["s0"], d["Wl"], d["sl"])
+    g = wt.backward_weight(d["X"], d["dY"], d["W0"], d["b0"], d["s0"], d["Wl"], d["sl"])
+    torch.cuda.synchronize()
+    out = dict(Y=y, dX=dx, dW0=g["dw0"], db0=g["db0"], ds0=g["ds0"])
+    if d["Wl"] is not None:
+        out.update(dWl=g["dwl"], dsl=g["dsl"])
+    return out
+
+
+def run_oracle(p):
+    Y = oracle.forward(p["X"], p["W0"], p["b0"], p["s0"], p["Wl"], p["sl"])
+    g = oracle.backward(p["X"], p["dY"], p["W0"], p["b0"], p["s0"], p["Wl"], p["sl"])
+    out = dict(Y=Y, dX=g["dX"], dW0=g["dW0"], db0=g["db0"], ds0=g["ds0"])
+    if p["Wl"] is not None:
+        out.update(dWl=g["dWl"], dsl=g["dsl"])
+    return out
+
+
+def check_all(wl, seed=0):
+    inp = make_inputs(wl, seed)
+    gpu = run_gpu(_dev(inp, wl.io))
+    ref = run_oracle(as_float64(inp))
+    errs = {k: _rel(_np(gpu[k]), ref[k]) for k in ref}
+    bad = {k: e for k, e in errs.items() if not e <= TOL[wl.io]}
+    assert not bad, (wl, errs)
+    return errs
+
+
+EDGE = [
+    Workload("tiny", 1, 8, 16, 16, 5, 2, "f32"),
+    Workload("ragged_L3", 3, 5, 24, 40, 3, 3, "f32"),
+    Workload("deepest_1x1", 2, 3, 8, 8, 5, 3, "f32"),
+    Workload("k7_L1", 2, 3, 16, 12, 7, 1, "f32"),
+    Workload("k1_L2", 2, 4, 16, 16, 1, 2, "f32"),
+    Workload("odd_L0", 2, 3, 7, 13, 5, 0, "f32"),
+    Workload("odd_L0_bf16", 2, 3, 9, 11, 3, 0, "bf16"),
+    Workload("bf16_w12", 2, 3, 12, 12, 5, 2, "bf16"),
+    Workload("min_2x2", 1, 1, 2, 2, 3, 1, "f32"),
+    Workload("w20", 2, 2, 20, 20, 5, 2, "f32"),
+    Workload("tall", 1, 2, 64, 8, 5, 3, "f32"),
+    Workload("multi_tile_L4", 2, 3, 64, 64, 5, 4, "f32"),
+    Workload("L4_bf16", 3, 2, 48, 32, 5, 4, "bf16"),
+    Workload("batchy_small", 37, 3, 14, 14, 5, 1, "f32"),
+]
+
+
+@pytest.mark.parametrize("wl", EDGE, ids=[w.name for w in EDGE])
+def test_parity_edge_cases(cuda_ok, wl):
+    check_all(wl)
+
+
+SMALL = {name: dataclasses.replace(w, N=min(w.N, 2)) for name, w in WORKLOADS.items()}
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_parity_workload_shapes_small_batch(cuda_ok, name):
+    """Every workload's plane shape, k, L and dtype at batch 2: all outputs."""
+    check_all(SMALL[name])
+
+
+FULL = ["stage1_f32_k5_L3", "stage2_bf16_k5_L2", "dw_k3_112_f32", "dw_k5_14_f32"]
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name", FULL)
+def test_parity_full_size(cuda_ok, name):
+    """Full workload size, every output element against the oracle."""
+    check_all(WORKLOADS[name])
+
+
+@pytest.mark.slow
+def test_parity_deep_full_size_sampled(cuda_ok):
+    """256x256 planes with 5 levels at full batch: y and dx on sampled batch
+    entries (the layer is independent across n); parameter gradients on a
+    sub-batch of the same planes."""
+    wl = WORKLOADS["deep_bf16_k5_L5"]
+    inp = make_inputs(wl, 0)
+    d = _dev(inp, wl.io)
+    y = wt.forward(d["X"], d["W0"], d["b0"], d["s0"], d["Wl"], d["sl"])
+    dx = wt.backward_data(d["dY"], d["W0"], d["s0"], d["Wl"], d["sl"])
+    torch.cuda.synchronize()
+    for n in (0, wl.N - 1):
+        p = as_float64({k: (v[n:n + 1] if k in ("X", "dY") else v) for k, v in inp.items()})
+        ref = run_oracle(p)
+        assert _rel(_np(y[n:n + 1]), ref["Y"]) <= TOL["bf16"]
+        assert _rel(_np(dx[n:n + 1]), ref["dX"]) <= TOL["bf16"]
+    sub = dataclasses.replace(wl, N=2)
+    check_all(sub)
+
+
+def test_weight_gradients_deterministic(cuda_ok):
+    wl = Workload("det", 4, 6, 32, 32, 5, 3, "f32")
+    d = _dev(make_inputs(wl, 1), wl.io)
+    a = run_gpu(d)
+    b = run_gpu(d)
+    for k in a:
+        assert torch.equal(a[k], b[k]), k
+
+
+def test_fused_backward_matches_separate_calls(cuda_ok):
+    wl = Workload("fused", 3, 4, 32, 32, 5, 2, "f32")
+    d = _dev(make_inputs(wl, 2), wl.io)
+    sep = run_gpu(d)
+    dx, g = wt.backward(d["X"], d["dY"], d["W0"], d["b0"], d["s0"], d["Wl"], d["sl"])
+    torch.cuda.synchronize()
+    assert torch.equal(dx, sep["dX"])
+    for k, kk in (("dw0", "dW0"), ("db0", "db0"), ("ds0", "ds0"), ("dwl", "dWl"), ("dsl", "dsl")):
+        assert torch.allclose(g[k], sep[kk], rtol=1e-6, atol=1e-6), k
+
+
+def test_delta_kernels_on_gpu(cuda_ok):
+    """Closed form Y = s0 X + sum_l s_l U_{l-1}(X) through the CUDA path."""
+    N, C, H, W, k, L = 2, 3, 32, 32, 5, 3
+    g = torch.Generator().manual_seed(5)
+    X = torch.randn(N, C, H, W, generator=g)
+    W0 = torch.zeros(C, k, k); W0[:, 2, 2] = 1
+    Wl = torch.zeros(L, C, 4, k, k); Wl[..., 2, 2] = 1
+    s0 = torch.rand(C, generator=g) + 0.5
+    sc = torch.rand(L, C, generator=g) + 0.5
+    sl = sc[:, :, None].repeat(1, 1, 4).contiguous()
+    y = wt.forward(X.cuda(), W0.cuda(), torch.zeros(C).cuda(), s0.cuda(), Wl.cuda(), sl.cuda()).cpu()
+    ref = s0.view(1, C, 1, 1) * X
+    for l in range(1, L + 1):
+        b = 1 << (l - 1)
+        m = torch.nn.functional.avg_pool2d(X, b) if b > 1 else X
+        m = m.repeat_interleave(b, 2).repeat_interleave(b, 3)
+        ref = ref + sc[l - 1].view(1, C, 1, 1) * m
+    assert (y - ref).abs().max().item() <= 1e-5 * ref.abs().max().item()
+
+
+def test_stream_argument_and_preallocated_outputs(cuda_ok):
+    wl = Workload("stream", 2, 3, 16, 16, 3, 2, "f32")
+    d = _dev(make_inputs(wl, 3), wl.io)
+    s = torch.cuda.Stream()
+    y = torch.empty_like(d["X"])
+    with torch.cuda.stream(s):
+        wt.forward(d["X"], d["W0"], d["b0"], d["s0"], d["Wl"], d["sl"], y=y, stream=s)
+    s.synchronize()
+    ref = wt.forward(d["X"], d["W0"], d["b0"], d["s0"], d["Wl"], d["sl"])
+    torch.cuda.synchronize()
+    assert torch.equal(y, ref)
