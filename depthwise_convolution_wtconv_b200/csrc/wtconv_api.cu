@@ -14,6 +14,23 @@ namespace wt {
 namespace {
 
 inline int rup(int a, int b) { return (a + b - 1) / b * b; }
+inline int cdiv_h(int a, int b) { return (a + b - 1) / b; }
+
+// Magic numbers for FDiv: x / d == umulhi(x, m) >> s for 0 <= x < 2^31.
+FDiv make_fdiv(int d) {
+  FDiv f;
+  f.d = d < 1 ? 1 : d;
+  f.m = 0;
+  f.s = 0;
+  if (f.d > 1) {
+    int lg = 0;
+    while ((1LL << lg) < f.d) ++lg;  // ceil(log2 d)
+    const unsigned long long p = 31 + lg;
+    f.m = (unsigned)(((1ULL << p) + (unsigned long long)f.d - 1) / (unsigned long long)f.d);
+    f.s = (int)(p - 32);
+  }
+  return f;
+}
 
 struct TileShape {
   int R, CW;
@@ -66,58 +83,113 @@ void fill_common(Plan& P, const wtconv_desc* d) {
   P.kk4 = rup(d->k * d->k, 4);
   P.vec_in = (d->W % 4) == 0;
   P.vec_out = d->io == WTCONV_BF16 ? (d->W % 8) == 0 : (d->W % 4) == 0;
+  P.prefetch_ok = ((size_t)d->H * d->W * io_bytes(d)) % 16 == 0;
+  P.io_bytes = io_bytes(d);
+  P.nthreads = NT;
   P.V = d->k * d->k * (1 + 4 * d->L) + 1;
 }
 
 // Per-plane slab of the forward / backward-data kernel.
 int forward_slab(Plan& P) {
-  const int r = P.r, L = P.L;
+  const int r = P.r, L = P.L, RB = P.R3 / 2;
   int cur = 0;
   P.xf = make_shifted(cur, P.H, P.W, r, {{P.R3, C3_CW}}, 1);
-  if (L >= 1) P.s1 = make_shifted(cur, P.H1, P.W1, r, {{C2_R, C2_CW}, {2, 2}}, 4);
-  if (L >= 2) P.t1 = make_plain(cur, P.H1, P.W1, {{C2_R, C2_CW}, {2 * DP_R, 2 * DP_CW}}, 1);
-  const int region = cur;
-  if (L >= 1) P.zb = make_plain(cur, P.H1, P.W1, {{C2_R, C2_CW}, {P.R3 / 2, C3_CW / 2}}, 4);
-  const int end1 = cur;
-  cur = region;
+  if (L >= 1) P.s1 = make_shifted(cur, P.H1, P.W1, r, {{RB, 4}, {2, 2}}, 4);
   if (L >= 2) {
+    P.t1 = make_plain(cur, P.H1, P.W1, {{RB, 4}, {1, 4}}, 1);
     for (int l = 2; l <= L; ++l) P.sd[l] = make_shifted(cur, P.H >> l, P.W >> l, r, {{DP_R, DP_CW}, {2, 2}}, 4);
-    for (int l = 3; l <= L; ++l) P.zd[l] = make_plain(cur, P.H >> l, P.W >> l, {{DP_R, DP_CW}}, 4);
-    if (L >= 3) P.t2 = make_plain(cur, P.H >> 2, P.W >> 2, {{DP_R, DP_CW}}, 1);
+    for (int l = 2; l <= L; ++l) P.zd[l] = make_plain(cur, P.H >> l, P.W >> l, {{DP_R, DP_CW}}, 4);
   }
-  P.deep_off = region;
-  P.deep_floats = cur - region;
-  return rup(std::max(end1, cur), 4);
+  P.deep_off = 0;
+  P.deep_floats = 0;
+  return rup(cur, 4);
 }
+
+void forward_items(Plan& P) {
+  const int L = P.L;
+  int per, xdiv;
+  if (L >= 2) {
+    xdiv = P.W >> 2;
+    per = (P.H >> 2) * xdiv;
+  } else if (L == 1) {
+    xdiv = cdiv_h(P.W, 4);
+    per = P.H1 * xdiv;
+  } else {
+    xdiv = cdiv_h(P.W, 4);
+    per = P.H * xdiv;
+  }
+  P.f_stage_per = make_fdiv(per);
+  P.f_stage_x = make_fdiv(xdiv);
+  int first = 0;
+  for (int l = 0; l <= MAXL + 1; ++l) P.deep_first[l] = 0;
+  for (int l = 2; l <= L; ++l) {
+    const int tx = cdiv_h(P.W >> l, DP_CW), tiles = cdiv_h(P.H >> l, DP_R) * tx;
+    P.f_l_tiles[l] = make_fdiv(tiles);
+    P.f_l_tx[l] = make_fdiv(tx);
+    P.deep_first[l] = first;
+    first += 4 * tiles;
+  }
+  P.deep_items = first;
+  if (L >= 2) P.deep_first[L + 1] = first;
+  P.f_deep_per = make_fdiv(first > 0 ? first : 1);
+  const int tq = cdiv_h(P.W1, 4);
+  P.f_t1_x = make_fdiv(tq);
+  P.f_t1_per = make_fdiv(P.H1 * tq);
+  const int ox = cdiv_h(P.W, C3_CW);
+  P.f_out_x = make_fdiv(ox);
+  P.f_out_per = make_fdiv(cdiv_h(P.H, P.R3) * ox);
+}
+
+// Shared-memory header: mbarrier (8 bytes) and abort flag, 16 bytes.
+constexpr int HEADER_FLOATS = 4;
 
 void finish_forward_plan(Plan& P, int PB) {
   const int slab = forward_slab(P);
   P.PB = PB;
   P.nbatch = (P.N + PB - 1) / PB;
-  P.w_off = 0;
-  const int base = rup((1 + 4 * P.L) * P.kk4 + 4, 4);
+  P.w_off = HEADER_FLOATS;
+  P.use_bulk = P.prefetch_ok;
+  P.raw_off = rup(P.w_off + (1 + 4 * P.L) * P.kk4 + 4, 4);
+  const int raw_floats = P.use_bulk ? rup((int)((size_t)PB * P.H * P.W * P.io_bytes / 4), 4) : 0;
+  const int base = P.raw_off + raw_floats;
   for (BufDesc* b : {&P.xf, &P.s1, &P.t1, &P.zb, &P.t2}) relocate(*b, base, slab);
   for (int l = 0; l <= MAXL; ++l) {
     relocate(P.sd[l], base, slab);
     relocate(P.zd[l], base, slab);
   }
-  P.deep_off += base;
   P.smem_floats = base + PB * slab;
+  forward_items(P);
 }
 
 // Tiles of the output pass per plane, for the batch-size choice.
 int output_items(const Plan& P, int R3) { return ((P.H + R3 - 1) / R3) * ((P.W + C3_CW - 1) / C3_CW); }
 
+// Threads per CTA of the forward kernel: 128 when one plane has few
+// output tiles, so that a batch of one plane still keeps most threads busy.
+int forward_threads(const Plan& P) { return output_items(P, P.H >= 8 ? 4 : 2) <= 128 ? 128 : 256; }
+
 void build_forward_plan(Plan& P, const wtconv_desc* d, int max_smem) {
   fill_common(P, d);
-  P.R3 = output_items(P, 4) >= NT / 2 ? 4 : 2;
+  P.R3 = (P.H >= 8) ? 4 : 2;
+  P.nthreads = forward_threads(P);
   const int items = output_items(P, P.R3);
-  int PB = std::max(1, std::min(d->N, (NT + items - 1) / items));
+  int PB = std::max(1, std::min(d->N, P.nthreads / items));
+  const size_t budget = (size_t)max_smem / 2;
   for (;;) {
     finish_forward_plan(P, PB);
-    if (PB == 1 || (size_t)P.smem_floats * 4 <= (size_t)max_smem / 2) break;
+    if (PB == 1 || (size_t)P.smem_floats * 4 <= budget) break;
     --PB;
   }
+}
+
+void bwdw_items(Plan& P) {
+  forward_items(P);  // staging and deep-level decompositions are shared
+  const int bx = cdiv_h(P.W, BW_CW);
+  P.f_bw_x = make_fdiv(bx);
+  P.f_bw_per = make_fdiv(cdiv_h(P.H, BW_R) * bx);
+  const int b1 = cdiv_h(P.W1, B1_CW);
+  P.f_b1_x = make_fdiv(b1);
+  P.f_b1_per = make_fdiv(cdiv_h(P.H1, B1_R) * b1);
 }
 
 int bwdw_slab(Plan& P) {
@@ -140,9 +212,13 @@ void finish_bwdw_plan(Plan& P, int PB) {
   const int slab = bwdw_slab(P);
   P.PB = PB;
   const int ndeep = P.L >= 2 ? (P.L - 1) * 4 : 0;
-  P.gdeep_off = 0;
-  P.dpart_off = ndeep * P.kk4;
-  const int base = rup(P.dpart_off + ndeep * DSLOTS * P.kk4, 4);
+  P.gdeep_off = HEADER_FLOATS;
+  P.dpart_off = P.gdeep_off + ndeep * P.kk4;
+  P.use_bulk = P.prefetch_ok;
+  const int raw_floats = P.use_bulk ? rup((int)((size_t)PB * P.H * P.W * P.io_bytes / 4), 4) : 0;
+  P.raw_off = rup(P.dpart_off + ndeep * DSLOTS * P.kk4, 4);
+  P.rawg_off = P.raw_off + raw_floats;
+  const int base = P.rawg_off + raw_floats;
   for (BufDesc* b : {&P.xf, &P.gf, &P.s1, &P.g1}) relocate(*b, base, slab);
   for (int l = 0; l <= MAXL; ++l) {
     relocate(P.sd[l], base, slab);
@@ -150,6 +226,7 @@ void finish_bwdw_plan(Plan& P, int PB) {
   }
   P.red_off = base;
   P.smem_floats = std::max(base + PB * slab, base + NT * P.kk4 + NT);
+  bwdw_items(P);
 }
 
 void build_bwdw_plan(Plan& P, const wtconv_desc* d, int max_smem) {
@@ -203,44 +280,46 @@ wtconv_status query_device(Device& dev) {
 }
 
 template <typename F>
-wtconv_status prepare(F kern, size_t smem, int& occ) {
+wtconv_status prepare(F kern, size_t smem, int& occ, int nthreads = NT) {
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return WTCONV_ERR_CUDA;
   occ = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, NT, smem) != cudaSuccess) return WTCONV_ERR_CUDA;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, nthreads, smem) != cudaSuccess)
+    return WTCONV_ERR_CUDA;
   if (occ < 1) return WTCONV_ERR_UNSUPPORTED;
   return WTCONV_OK;
 }
 
 template <int K, int R3, typename IO>
 wtconv_status launch_fwd_t(const Plan& P, const Device& dev, const void* x, const float* w0, const float* b0,
-                           const float* s0, const float* wl, const float* sl, void* y, int flip,
+                           const float* s0, const float* wl, const float* sl, void* y, int flip, int* status,
                            cudaStream_t st) {
   auto kern = wtconv_fwd_kernel<K, R3, IO>;
   const size_t smem = (size_t)P.smem_floats * 4;
   int occ = 0;
-  wtconv_status e = prepare(kern, smem, occ);
+  wtconv_status e = prepare(kern, smem, occ, P.nthreads);
   if (e != WTCONV_OK) return e;
   const int units = P.C * P.nbatch;
   const int grid = std::min(units, dev.sms * occ);
-  kern<<<grid, NT, smem, st>>>(P, static_cast<const IO*>(x), w0, b0, s0, wl, sl, static_cast<IO*>(y), flip);
+  kern<<<grid, P.nthreads, smem, st>>>(P, static_cast<const IO*>(x), w0, b0, s0, wl, sl, static_cast<IO*>(y), flip,
+                                       status);
   return cudaGetLastError() == cudaSuccess ? WTCONV_OK : WTCONV_ERR_CUDA;
 }
 
 template <int K>
 wtconv_status launch_fwd_k(const Plan& P, const Device& dev, wtconv_dtype io, const void* x, const float* w0,
                            const float* b0, const float* s0, const float* wl, const float* sl, void* y, int flip,
-                           cudaStream_t st) {
+                           int* status, cudaStream_t st) {
   if (io == WTCONV_F32) {
-    if (P.R3 == 4) return launch_fwd_t<K, 4, float>(P, dev, x, w0, b0, s0, wl, sl, y, flip, st);
-    return launch_fwd_t<K, 2, float>(P, dev, x, w0, b0, s0, wl, sl, y, flip, st);
+    if (P.R3 == 4) return launch_fwd_t<K, 4, float>(P, dev, x, w0, b0, s0, wl, sl, y, flip, status, st);
+    return launch_fwd_t<K, 2, float>(P, dev, x, w0, b0, s0, wl, sl, y, flip, status, st);
   }
-  if (P.R3 == 4) return launch_fwd_t<K, 4, __nv_bfloat16>(P, dev, x, w0, b0, s0, wl, sl, y, flip, st);
-  return launch_fwd_t<K, 2, __nv_bfloat16>(P, dev, x, w0, b0, s0, wl, sl, y, flip, st);
+  if (P.R3 == 4) return launch_fwd_t<K, 4, __nv_bfloat16>(P, dev, x, w0, b0, s0, wl, sl, y, flip, status, st);
+  return launch_fwd_t<K, 2, __nv_bfloat16>(P, dev, x, w0, b0, s0, wl, sl, y, flip, status, st);
 }
 
 wtconv_status run_forward(const wtconv_desc* d, const void* x, const float* w0, const float* b0, const float* s0,
-                          const float* wl, const float* sl, void* y, int flip, cudaStream_t st) {
+                          const float* wl, const float* sl, void* y, int flip, int* status, cudaStream_t st) {
   Device dev;
   wtconv_status e = query_device(dev);
   if (e != WTCONV_OK) return e;
@@ -248,32 +327,50 @@ wtconv_status run_forward(const wtconv_desc* d, const void* x, const float* w0, 
   build_forward_plan(P, d, dev.max_smem);
   if ((size_t)P.smem_floats * 4 > (size_t)dev.max_smem) return WTCONV_ERR_UNSUPPORTED;
   switch (d->k) {
-    case 1: return launch_fwd_k<1>(P, dev, d->io, x, w0, b0, s0, wl, sl, y, flip, st);
-    case 3: return launch_fwd_k<3>(P, dev, d->io, x, w0, b0, s0, wl, sl, y, flip, st);
-    case 5: return launch_fwd_k<5>(P, dev, d->io, x, w0, b0, s0, wl, sl, y, flip, st);
-    default: return launch_fwd_k<7>(P, dev, d->io, x, w0, b0, s0, wl, sl, y, flip, st);
+    case 1: return launch_fwd_k<1>(P, dev, d->io, x, w0, b0, s0, wl, sl, y, flip, status, st);
+    case 3: return launch_fwd_k<3>(P, dev, d->io, x, w0, b0, s0, wl, sl, y, flip, status, st);
+    case 5: return launch_fwd_k<5>(P, dev, d->io, x, w0, b0, s0, wl, sl, y, flip, status, st);
+    default: return launch_fwd_k<7>(P, dev, d->io, x, w0, b0, s0, wl, sl, y, flip, status, st);
   }
 }
 
+// Workspace: a 16-byte header whose first int is the device status word,
+// then (weight gradients) the per-CTA partial sums.
+constexpr size_t WS_HEADER = 16;
+
 size_t bwdw_ws_bytes(const wtconv_desc* d) {
   const size_t V = (size_t)d->k * d->k * (1 + 4 * d->L) + 1;
-  return (size_t)d->N * d->C * V * sizeof(float);
+  return WS_HEADER + (size_t)d->N * d->C * V * sizeof(float);
 }
 
 template <int K, typename IO>
 wtconv_status launch_bwdw_t(Plan& P, const Device& dev, const void* x, const void* dy, const float* w0,
                             const float* b0, const float* s0, const float* wl, const float* sl, float* dw0,
-                            float* db0, float* ds0, float* dwl, float* dsl, float* part, cudaStream_t st) {
+                            float* db0, float* ds0, float* dwl, float* dsl, float* part, int* status,
+                            cudaStream_t st) {
   auto kern = wtconv_bwdw_kernel<K, IO>;
   const size_t smem = (size_t)P.smem_floats * 4;
   int occ = 0;
   wtconv_status e = prepare(kern, smem, occ);
   if (e != WTCONV_OK) return e;
+  // planes per CTA: fewest sequential batches per CTA slot (waves x batches
+  // per CTA), ties broken towards longer CTAs (fewer partial sums)
   const int slots = dev.sms * occ;
-  int groups = std::max(1, std::min(P.N, slots / P.C));
-  P.planes_per_cta = (P.N + groups - 1) / groups;
+  long best = -1;
+  for (int ppc = P.PB; ppc < P.N + P.PB; ppc += P.PB) {
+    const int p = std::min(ppc, P.N);
+    const int groups = (P.N + p - 1) / p;
+    const long ctas = (long)P.C * groups;
+    const long cost = ((ctas + slots - 1) / slots) * ((p + P.PB - 1) / P.PB);
+    if (best < 0 || cost <= best) {
+      best = cost;
+      P.planes_per_cta = p;
+    }
+    if (p == P.N) break;
+  }
   P.ngroups = (P.N + P.planes_per_cta - 1) / P.planes_per_cta;
-  kern<<<P.C * P.ngroups, NT, smem, st>>>(P, static_cast<const IO*>(x), static_cast<const IO*>(dy), part);
+  kern<<<P.C * P.ngroups, NT, smem, st>>>(P, static_cast<const IO*>(x), static_cast<const IO*>(dy), part,
+                                          status);
   if (cudaGetLastError() != cudaSuccess) return WTCONV_ERR_CUDA;
   const size_t fsmem = (size_t)P.V * sizeof(float);
   auto fin = wtconv_bwdw_finalize<K>;
@@ -287,11 +384,12 @@ wtconv_status launch_bwdw_t(Plan& P, const Device& dev, const void* x, const voi
 template <int K>
 wtconv_status launch_bwdw_k(Plan& P, const Device& dev, wtconv_dtype io, const void* x, const void* dy,
                             const float* w0, const float* b0, const float* s0, const float* wl, const float* sl,
-                            float* dw0, float* db0, float* ds0, float* dwl, float* dsl, float* part,
+                            float* dw0, float* db0, float* ds0, float* dwl, float* dsl, float* part, int* status,
                             cudaStream_t st) {
   if (io == WTCONV_F32)
-    return launch_bwdw_t<K, float>(P, dev, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, part, st);
-  return launch_bwdw_t<K, __nv_bfloat16>(P, dev, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, part, st);
+    return launch_bwdw_t<K, float>(P, dev, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, part, status, st);
+  return launch_bwdw_t<K, __nv_bfloat16>(P, dev, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, part, status,
+                                         st);
 }
 
 wtconv_status run_bwdw(const wtconv_desc* d, const void* x, const void* dy, const float* w0, const float* b0,
@@ -303,12 +401,17 @@ wtconv_status run_bwdw(const wtconv_desc* d, const void* x, const void* dy, cons
   Plan P;
   build_bwdw_plan(P, d, dev.max_smem);
   if ((size_t)P.smem_floats * 4 > (size_t)dev.max_smem) return WTCONV_ERR_UNSUPPORTED;
-  float* part = static_cast<float*>(ws);
+  int* status = static_cast<int*>(ws);
+  float* part = reinterpret_cast<float*>(static_cast<char*>(ws) + WS_HEADER);
   switch (d->k) {
-    case 1: return launch_bwdw_k<1>(P, dev, d->io, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, part, st);
-    case 3: return launch_bwdw_k<3>(P, dev, d->io, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, part, st);
-    case 5: return launch_bwdw_k<5>(P, dev, d->io, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, part, st);
-    default: return launch_bwdw_k<7>(P, dev, d->io, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, part, st);
+    case 1:
+      return launch_bwdw_k<1>(P, dev, d->io, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, part, status, st);
+    case 3:
+      return launch_bwdw_k<3>(P, dev, d->io, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, part, status, st);
+    case 5:
+      return launch_bwdw_k<5>(P, dev, d->io, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, part, status, st);
+    default:
+      return launch_bwdw_k<7>(P, dev, d->io, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, part, status, st);
   }
 }
 
@@ -340,7 +443,7 @@ size_t wtconv_workspace_size(const wtconv_desc* desc, int op) {
   switch (op) {
     case WTCONV_OP_FORWARD:
     case WTCONV_OP_BACKWARD_DATA:
-      return 0;
+      return WS_HEADER;
     case WTCONV_OP_BACKWARD_WEIGHT:
     case WTCONV_OP_BACKWARD:
       return bwdw_ws_bytes(desc);
@@ -357,9 +460,9 @@ wtconv_status wtconv_forward(const wtconv_desc* desc, const void* x, const float
   if (!x || !y) return WTCONV_ERR_ARG;
   if ((e = check_params(desc, w0, b0, s0, wl, sl, true)) != WTCONV_OK) return e;
   if (!aligned16(x) || !aligned16(y)) return WTCONV_ERR_ALIGN;
-  (void)ws;
-  (void)ws_bytes;
-  return run_forward(desc, x, w0, b0, s0, wl, sl, y, 0, static_cast<cudaStream_t>(stream));
+  if (ws && !aligned16(ws)) return WTCONV_ERR_ALIGN;
+  int* status = (ws && ws_bytes >= WS_HEADER) ? static_cast<int*>(ws) : nullptr;
+  return run_forward(desc, x, w0, b0, s0, wl, sl, y, 0, status, static_cast<cudaStream_t>(stream));
 }
 
 wtconv_status wtconv_backward_data(const wtconv_desc* desc, const void* dy, const float* w0, const float* s0,
@@ -370,9 +473,9 @@ wtconv_status wtconv_backward_data(const wtconv_desc* desc, const void* dy, cons
   if (!dy || !dx) return WTCONV_ERR_ARG;
   if ((e = check_params(desc, w0, nullptr, s0, wl, sl, false)) != WTCONV_OK) return e;
   if (!aligned16(dy) || !aligned16(dx)) return WTCONV_ERR_ALIGN;
-  (void)ws;
-  (void)ws_bytes;
-  return run_forward(desc, dy, w0, nullptr, s0, wl, sl, dx, 1, static_cast<cudaStream_t>(stream));
+  if (ws && !aligned16(ws)) return WTCONV_ERR_ALIGN;
+  int* status = (ws && ws_bytes >= WS_HEADER) ? static_cast<int*>(ws) : nullptr;
+  return run_forward(desc, dy, w0, nullptr, s0, wl, sl, dx, 1, status, static_cast<cudaStream_t>(stream));
 }
 
 wtconv_status wtconv_backward_weight(const wtconv_desc* desc, const void* x, const void* dy, const float* w0,
@@ -402,7 +505,7 @@ wtconv_status wtconv_backward(const wtconv_desc* desc, const void* x, const void
   if (!aligned16(x) || !aligned16(dy) || !aligned16(dx)) return WTCONV_ERR_ALIGN;
   if ((e = check_ws(ws, ws_bytes, bwdw_ws_bytes(desc))) != WTCONV_OK) return e;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  e = run_forward(desc, dy, w0, nullptr, s0, wl, sl, dx, 1, st);
+  e = run_forward(desc, dy, w0, nullptr, s0, wl, sl, dx, 1, static_cast<int*>(ws), st);
   if (e != WTCONV_OK) return e;
   return run_bwdw(desc, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, ws, st);
 }

@@ -39,7 +39,7 @@ __device__ void load_weights(const Plan& P, float* sw, int c, const float* __res
   constexpr int KK = K * K;
   const int kk4 = P.kk4;
   const int total = (1 + 4 * P.L) * kk4;
-  for (int i = threadIdx.x; i < total; i += NT) {
+  for (int i = threadIdx.x; i < total; i += blockDim.x) {
     const int blk = i / kk4, t = i - blk * kk4;
     float v = 0.f;
     if (t < KK) {
@@ -57,69 +57,12 @@ __device__ void load_weights(const Plan& P, float* sw, int c, const float* __res
   if (threadIdx.x < 4) sw[kk4 + threadIdx.x] = (threadIdx.x == 0 && !flip) ? s0[c] * b0[c] : 0.f;
 }
 
-// ------------------------------------------------------------ staging
-// Reads plane `xp` (H x W, I/O dtype) into the shifted fp32 buffer xf and,
-// when L >= 1, writes its level-1 Haar subbands into the shifted 4-band
-// buffer s1.  Only the image interior is written; borders stay zero.
-// Optionally accumulates the sum of all values read into *sum.
-template <typename IO, bool SUM>
-__device__ void stage_plane(const Plan& P, const IO* __restrict__ xp, float* xf, int ldx, float* s1, int ld1,
-                            int bs1, bool shifted, float* sum) {
-  const int r = shifted ? P.r : 0;
-  const int Q = (P.W + 3) >> 2;
-  if (P.L >= 1) {
-    const int items = P.H1 * Q;
-    for (int it = threadIdx.x; it < items; it += NT) {
-      const int i = it / Q, q = it - i * Q;
-      const int x0 = q << 2;
-      const IO* p0 = xp + (size_t)(2 * i) * P.W + x0;
-      const float4 a = load4(p0, x0, P.W, P.vec_in);
-      const float4 b = load4(p0 + P.W, x0, P.W, P.vec_in);
-      if (SUM) *sum += ((a.x + a.y) + (a.z + a.w)) + ((b.x + b.y) + (b.z + b.w));
-      float* d0 = xf + (2 * i + r) * ldx + x0 + r;
-      float* d1 = d0 + ldx;
-      const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e)
-        if (x0 + e < P.W) {
-          d0[e] = av[e];
-          d1[e] = bv[e];
-        }
-      float* o = s1 + (i + r) * ld1 + (x0 >> 1) + r;
-#pragma unroll
-      for (int bk = 0; bk < 2; ++bk) {
-        if (x0 + 2 * bk < P.W) {
-          float ll, lh, hl, hh;
-          haar4(av[2 * bk], av[2 * bk + 1], bv[2 * bk], bv[2 * bk + 1], ll, lh, hl, hh);
-          o[bk] = ll;
-          o[bs1 + bk] = lh;
-          o[2 * bs1 + bk] = hl;
-          o[3 * bs1 + bk] = hh;
-        }
-      }
-    }
-  } else {
-    const int items = P.H * Q;
-    for (int it = threadIdx.x; it < items; it += NT) {
-      const int y = it / Q, q = it - y * Q;
-      const int x0 = q << 2;
-      const float4 a = load4(xp + (size_t)y * P.W + x0, x0, P.W, P.vec_in);
-      if (SUM) *sum += (a.x + a.y) + (a.z + a.w);
-      float* d0 = xf + (y + r) * ldx + x0 + r;
-      const float av[4] = {a.x, a.y, a.z, a.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e)
-        if (x0 + e < P.W) d0[e] = av[e];
-    }
-  }
-}
-
 // Haar analysis of the LL band of level l-1 into the 4 bands of level l
 // for every plane of the batch.  src: LL of level l-1 at interior origin.
 __device__ void pyramid_level(int npb, int hl, int wlv, const float* src0, int lds, int src_ps, float* dst0,
                               int ldd, int bsd, int dst_ps) {
   const int per = hl * wlv;
-  for (int it = threadIdx.x; it < npb * per; it += NT) {
+  for (int it = threadIdx.x; it < npb * per; it += blockDim.x) {
     const int pb = it / per, rem = it - pb * per;
     const int i = rem / wlv, j = rem - i * wlv;
     const float* q = src0 + pb * src_ps + (2 * i) * lds + 2 * j;
@@ -135,211 +78,366 @@ __device__ void pyramid_level(int npb, int hl, int wlv, const float* src0, int l
 
 __device__ __forceinline__ int cdiv(int a, int b) { return (a + b - 1) / b; }
 
+// ------------------------------------------------------ vector smem stores
+// 4 floats at p = row + x0 + RB with x0 % 4 == 0 (RB = column offset).
+template <int RB>
+__device__ __forceinline__ void sts4(float* p, const float4 v) {
+  if constexpr (RB % 4 == 0) {
+    *reinterpret_cast<float4*>(p) = v;
+  } else if constexpr (RB % 2 == 0) {
+    reinterpret_cast<float2*>(p)[0] = make_float2(v.x, v.y);
+    reinterpret_cast<float2*>(p)[1] = make_float2(v.z, v.w);
+  } else {
+    p[0] = v.x;
+    p[1] = v.y;
+    p[2] = v.z;
+    p[3] = v.w;
+  }
+}
+// 2 floats at p = row + x0 + RB with x0 even.
+template <int RB>
+__device__ __forceinline__ void sts2(float* p, float a, float b) {
+  if constexpr (RB % 2 == 0) {
+    *reinterpret_cast<float2*>(p) = make_float2(a, b);
+  } else {
+    p[0] = a;
+    p[1] = b;
+  }
+}
+
+// ------------------------------------------------------------ staging
+// Loads 4 consecutive elements of a staged row (smem, I/O dtype): vector
+// loads when `vec` (row start and x 16/8-byte aligned), else scalar with
+// zero past w.
+__device__ __forceinline__ float4 lds4(const float* p, int x, int w, bool vec) {
+  if (vec && x + 3 < w) return *reinterpret_cast<const float4*>(p);
+  return make_float4(x + 0 < w ? p[0] : 0.f, x + 1 < w ? p[1] : 0.f, x + 2 < w ? p[2] : 0.f,
+                     x + 3 < w ? p[3] : 0.f);
+}
+__device__ __forceinline__ float4 lds4(const __nv_bfloat16* p, int x, int w, bool vec) {
+  if (vec && x + 3 < w) {
+    const uint2 raw = *reinterpret_cast<const uint2*>(p);
+    return make_float4(__uint_as_float(raw.x << 16), __uint_as_float(raw.x & 0xffff0000u),
+                       __uint_as_float(raw.y << 16), __uint_as_float(raw.y & 0xffff0000u));
+  }
+  const unsigned short* q = reinterpret_cast<const unsigned short*>(p);
+  return make_float4(x + 0 < w ? __uint_as_float((unsigned)q[0] << 16) : 0.f,
+                     x + 1 < w ? __uint_as_float((unsigned)q[1] << 16) : 0.f,
+                     x + 2 < w ? __uint_as_float((unsigned)q[2] << 16) : 0.f,
+                     x + 3 < w ? __uint_as_float((unsigned)q[3] << 16) : 0.f);
+}
+template <bool SMEM, typename IO>
+__device__ __forceinline__ float4 src4(const IO* p, int x, int w, bool vec) {
+  if constexpr (SMEM) return lds4(p, x, w, vec);
+  else return load4(p, x, w, vec);
+}
+
+// Stages the npb planes of a batch: the plane into the fp32 buffer xf, its
+// level-1 subbands into s1 and, when L >= 2, its level-2 subbands into s2
+// (4x4 blocks of x per item; the Haar butterflies run in registers).  The
+// source is either the raw copy of the batch in shared memory (SMEM, planes
+// packed back to back) or global memory.  SH selects the shifted layout
+// (border r, read by the register tiles at x0 - r) or the plain layout (read
+// at x0).  SUM accumulates every value read.
+template <int K, typename IO, bool SH, bool SUM, bool SMEM>
+__device__ void stage_planes(const Plan& P, float* sm, const IO* __restrict__ src0, size_t pstride, int npb,
+                             const BufDesc& bx, const BufDesc& b1, const BufDesc& b2, float* sum) {
+  constexpr int r = SH ? K / 2 : 0;
+  const int ldx = bx.ld;
+  const bool vec = P.vec_in != 0;
+  if (P.L >= 2) {
+    const int bw = P.W >> 2, per = (P.H >> 2) * bw, n = npb * per;
+    const int ld1 = b1.ld, bs1 = b1.ld * b1.rows, ld2 = b2.ld, bs2 = b2.ld * b2.rows;
+    for (int it = threadIdx.x; it < n; it += blockDim.x) {
+      const int pb = P.f_stage_per.div(it);
+      const int rem = it - pb * per;
+      const int by = P.f_stage_x.div(rem);
+      const int bxi = rem - by * bw;
+      const int x0 = bxi << 2, y0 = by << 2;
+      const IO* src = src0 + pb * pstride + (size_t)y0 * P.W + x0;
+      float4 v[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) v[i] = src4<SMEM>(src + (size_t)i * P.W, x0, P.W, true);
+      if (SUM) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) *sum += (v[i].x + v[i].y) + (v[i].z + v[i].w);
+      }
+      float* xf = sm + bx.off + pb * bx.ps + (y0 + r) * ldx + x0 + r;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) sts4<r>(xf + i * ldx, v[i]);
+      float* s1 = sm + b1.off + pb * b1.ps + (2 * by + r) * ld1 + 2 * bxi + r;
+      float ll[2][2];
+#pragma unroll
+      for (int a = 0; a < 2; ++a) {
+        float l0, h0, g0, k0, l1, h1, g1, k1;
+        haar4(v[2 * a].x, v[2 * a].y, v[2 * a + 1].x, v[2 * a + 1].y, l0, h0, g0, k0);
+        haar4(v[2 * a].z, v[2 * a].w, v[2 * a + 1].z, v[2 * a + 1].w, l1, h1, g1, k1);
+        sts2<r>(s1 + a * ld1, l0, l1);
+        sts2<r>(s1 + bs1 + a * ld1, h0, h1);
+        sts2<r>(s1 + 2 * bs1 + a * ld1, g0, g1);
+        sts2<r>(s1 + 3 * bs1 + a * ld1, k0, k1);
+        ll[a][0] = l0;
+        ll[a][1] = l1;
+      }
+      float L2, H2, G2, K2;
+      haar4(ll[0][0], ll[0][1], ll[1][0], ll[1][1], L2, H2, G2, K2);
+      float* s2 = sm + b2.off + pb * b2.ps + (by + r) * ld2 + bxi + r;
+      s2[0] = L2;
+      s2[bs2] = H2;
+      s2[2 * bs2] = G2;
+      s2[3 * bs2] = K2;
+    }
+  } else if (P.L == 1) {
+    const int Q = (P.W + 3) >> 2, per = P.H1 * Q, n = npb * per;
+    const int ld1 = b1.ld, bs1 = b1.ld * b1.rows;
+    for (int it = threadIdx.x; it < n; it += blockDim.x) {
+      const int pb = P.f_stage_per.div(it);
+      const int rem = it - pb * per;
+      const int i = P.f_stage_x.div(rem);
+      const int x0 = (rem - i * Q) << 2;
+      const IO* src = src0 + pb * pstride + (size_t)(2 * i) * P.W + x0;
+      const float4 a = src4<SMEM>(src, x0, P.W, vec);
+      const float4 b = src4<SMEM>(src + P.W, x0, P.W, vec);
+      if (SUM) *sum += ((a.x + a.y) + (a.z + a.w)) + ((b.x + b.y) + (b.z + b.w));
+      float* d0 = sm + bx.off + pb * bx.ps + (2 * i + r) * ldx + x0 + r;
+      float* s1 = sm + b1.off + pb * b1.ps + (i + r) * ld1 + (x0 >> 1) + r;
+      float l0, h0, g0, k0, l1, h1, g1, k1;
+      haar4(a.x, a.y, b.x, b.y, l0, h0, g0, k0);
+      haar4(a.z, a.w, b.z, b.w, l1, h1, g1, k1);
+      if (x0 + 3 < P.W) {
+        sts4<r>(d0, a);
+        sts4<r>(d0 + ldx, b);
+        sts2<r>(s1, l0, l1);
+        sts2<r>(s1 + bs1, h0, h1);
+        sts2<r>(s1 + 2 * bs1, g0, g1);
+        sts2<r>(s1 + 3 * bs1, k0, k1);
+      } else {  // W % 4 == 2: one 2-wide block left in the row
+        d0[0] = a.x;
+        d0[1] = a.y;
+        d0[ldx] = b.x;
+        d0[ldx + 1] = b.y;
+        s1[0] = l0;
+        s1[bs1] = h0;
+        s1[2 * bs1] = g0;
+        s1[3 * bs1] = k0;
+      }
+    }
+  } else {
+    const int Q = (P.W + 3) >> 2, per = P.H * Q, n = npb * per;
+    for (int it = threadIdx.x; it < n; it += blockDim.x) {
+      const int pb = P.f_stage_per.div(it);
+      const int rem = it - pb * per;
+      const int yy = P.f_stage_x.div(rem);
+      const int x0 = (rem - yy * Q) << 2;
+      const float4 a = src4<SMEM>(src0 + pb * pstride + (size_t)yy * P.W + x0, x0, P.W, vec);
+      if (SUM) *sum += (a.x + a.y) + (a.z + a.w);
+      float* d0 = sm + bx.off + pb * bx.ps + (yy + r) * ldx + x0 + r;
+      if (x0 + 3 < P.W) {
+        sts4<r>(d0, a);
+      } else {
+        const float av[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          if (x0 + e < P.W) d0[e] = av[e];
+      }
+    }
+  }
+}
+
+// ------------------------------------------------ TMA bulk copies of planes
+// The issuing thread first announces the bytes of one batch on the CTA's
+// mbarrier (one arrival per phase), then issues 1-D bulk copies of whole
+// planes (each H*W elements, contiguous in global memory, a multiple of 16
+// bytes) into a raw shared-memory buffer; the phase completes when they land.
+__device__ __forceinline__ void bulk_expect(uint64_t* mbar, unsigned bytes) {
+  const unsigned bar = (unsigned)__cvta_generic_to_shared(mbar);
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+template <typename IO>
+__device__ __forceinline__ void bulk_copies(uint64_t* mbar, void* raw, const IO* src, size_t pstride, int npb,
+                                            unsigned bytes) {
+  const unsigned bar = (unsigned)__cvta_generic_to_shared(mbar);
+  const unsigned dst = (unsigned)__cvta_generic_to_shared(raw);
+  for (int pb = 0; pb < npb; ++pb) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            dst + pb * bytes),
+        "l"(src + pb * pstride), "r"(bytes), "r"(bar)
+        : "memory");
+  }
+}
+
+// Waits for the mbarrier phase `parity` with an iteration limit.  Returns
+// false when the limit ran out (the copy never completed).
+__device__ __forceinline__ bool mbar_wait(uint64_t* mbar, unsigned parity) {
+  const unsigned bar = (unsigned)__cvta_generic_to_shared(mbar);
+  for (int i = 0; i < (1 << 22); ++i) {
+    unsigned done;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(done)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    if (done) return true;
+  }
+  return false;
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* mbar) {
+  const unsigned bar = (unsigned)__cvta_generic_to_shared(mbar);
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar) : "memory");
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // ------------------------------------------------------------ deep levels
-// Levels 2..L of the batch: pyramid, level convs, closed-form synthesis of
-// levels >= 3 at level-2 resolution (t2), then the level-2 conv fused with
-// its synthesis butterfly into t1 (level-1 resolution).  Ends synchronised.
+// Levels 2..L of the batch: the rest of the pyramid (levels >= 3), every
+// level conv in one parallel pass (folded weights 2^-l s_l W_l), then the
+// closed-form synthesis of all levels >= 2 at level-1 resolution:
+//   t1(i,j) = sum_{l>=2} sum_s sigma_s(bit_{l-2}(i), bit_{l-2}(j)) Zd_l^s(i >> (l-1), j >> (l-1))
+// Ends synchronised.
 template <int K>
 __device__ void deep_forward(const Plan& P, float* sm, const float* sw, int npb) {
-  const int r = P.r;
+  constexpr int r = K / 2;
   const int kk4 = P.kk4;
-  // the deep region aliases the level-1 conv buffer: clear borders first
-  for (int pb = 0; pb < npb; ++pb) {
-    float4* z = reinterpret_cast<float4*>(sm + P.deep_off + pb * P.xf.ps);
-    for (int i = threadIdx.x; i < (P.deep_floats >> 2); i += NT) z[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int l = 3; l <= P.L; ++l) {
+    const BufDesc& s = P.sd[l - 1];
+    const BufDesc& d = P.sd[l];
+    pyramid_level(npb, P.H >> l, P.W >> l, sm + s.off + r * s.ld + r, s.ld, s.ps, sm + d.off + r * d.ld + r, d.ld,
+                  d.ld * d.rows, d.ps);
+    __syncthreads();
+  }
+  const int per = P.deep_items;
+  for (int it = threadIdx.x; it < npb * per; it += blockDim.x) {
+    const int pb = P.f_deep_per.div(it);
+    int rem = it - pb * per;
+    int l = 2;
+    while (rem >= P.deep_first[l + 1]) ++l;
+    rem -= P.deep_first[l];
+    const int tpb = P.f_l_tiles[l].d;
+    const int s = P.f_l_tiles[l].div(rem);
+    rem -= s * tpb;
+    const int ti = P.f_l_tx[l].div(rem);
+    const int tj = rem - ti * P.f_l_tx[l].d;
+    const BufDesc& d = P.sd[l];
+    const BufDesc& z = P.zd[l];
+    float acc[DP_R][DP_CW];
+#pragma unroll
+    for (int a = 0; a < DP_R; ++a)
+#pragma unroll
+      for (int b = 0; b < DP_CW; ++b) acc[a][b] = 0.f;
+    conv_tile<K, DP_R, DP_CW>(sm + d.off + pb * d.ps + s * d.ld * d.rows + ti * DP_R * d.ld + tj * DP_CW, d.ld,
+                              sw + wl_off(kk4, l, s), acc);
+    float* o = sm + z.off + pb * z.ps + s * z.ld * z.rows + ti * DP_R * z.ld + tj * DP_CW;
+#pragma unroll
+    for (int a = 0; a < DP_R; ++a)
+      reinterpret_cast<float4*>(o + a * z.ld)[0] = make_float4(acc[a][0], acc[a][1], acc[a][2], acc[a][3]);
   }
   __syncthreads();
-  for (int l = 2; l <= P.L; ++l) {
-    const BufDesc& d = P.sd[l];
-    const float* src;
-    int lds;
-    if (l == 2) {
-      src = sm + P.s1.off + r * P.s1.ld + r;
-      lds = P.s1.ld;
-    } else {
-      src = sm + P.sd[l - 1].off + r * P.sd[l - 1].ld + r;
-      lds = P.sd[l - 1].ld;
-    }
-    pyramid_level(npb, P.H >> l, P.W >> l, src, lds, P.xf.ps, sm + d.off + r * d.ld + r, d.ld, d.ld * d.rows,
-                  P.xf.ps);
-    __syncthreads();
-  }
-  if (P.L >= 3) {
-    // level convs l = 3..L (folded weights); items (pb, l, s, tile)
-    int per_plane = 0;
-    for (int l = 3; l <= P.L; ++l) per_plane += 4 * cdiv(P.H >> l, DP_R) * cdiv(P.W >> l, DP_CW);
-    for (int it = threadIdx.x; it < npb * per_plane; it += NT) {
-      const int pb = it / per_plane;
-      int rem = it - pb * per_plane;
-      int l = 3;
-      for (;;) {
-        const int n = 4 * cdiv(P.H >> l, DP_R) * cdiv(P.W >> l, DP_CW);
-        if (rem < n) break;
-        rem -= n;
-        ++l;
-      }
-      const int tx = cdiv(P.W >> l, DP_CW), tpb = cdiv(P.H >> l, DP_R) * tx;
-      const int s = rem / tpb;
-      rem -= s * tpb;
-      const int ti = rem / tx, tj = rem - ti * tx;
-      const BufDesc& d = P.sd[l];
-      const BufDesc& z = P.zd[l];
-      float acc[DP_R][DP_CW];
-#pragma unroll
-      for (int a = 0; a < DP_R; ++a)
-#pragma unroll
-        for (int b = 0; b < DP_CW; ++b) acc[a][b] = 0.f;
-      conv_tile<K, DP_R, DP_CW>(sm + d.off + pb * d.ps + s * d.ld * d.rows + ti * DP_R * d.ld + tj * DP_CW, d.ld,
-                                sw + wl_off(kk4, l, s), acc);
-      float* o = sm + z.off + pb * z.ps + s * z.ld * z.rows + ti * DP_R * z.ld + tj * DP_CW;
-#pragma unroll
-      for (int a = 0; a < DP_R; ++a)
-        reinterpret_cast<float4*>(o + a * z.ld)[0] = make_float4(acc[a][0], acc[a][1], acc[a][2], acc[a][3]);
-    }
-    __syncthreads();
-    // t2(i,j) = sum_{l>=3} sum_s sigma_s(bit_{l-3}(i), bit_{l-3}(j)) Zd_l^s(i >> (l-2), j >> (l-2))
-    const int h2 = P.H >> 2, w2 = P.W >> 2;
-    for (int it = threadIdx.x; it < npb * h2 * w2; it += NT) {
-      const int pb = it / (h2 * w2), rem = it - pb * h2 * w2;
-      const int i = rem / w2, j = rem - i * w2;
-      float acc = 0.f;
+  {
+    const int tq = P.f_t1_x.d, per1 = P.f_t1_per.d;
+    const BufDesc& z2 = P.zd[2];
+    const int bz2 = z2.ld * z2.rows;
+    for (int it = threadIdx.x; it < npb * per1; it += blockDim.x) {
+      const int pb = P.f_t1_per.div(it);
+      const int rem = it - pb * per1;
+      const int i = P.f_t1_x.div(rem);
+      const int j0 = (rem - i * tq) << 2;
+      // level 2: positions (i >> 1, (j0 >> 1) + {0, 1}), sign bits bit0(i), bit0(j)
+      const float* q = sm + z2.off + pb * z2.ps + (i >> 1) * z2.ld + (j0 >> 1);
+      const float2 zl = *reinterpret_cast<const float2*>(q);
+      const float2 zh = *reinterpret_cast<const float2*>(q + bz2);
+      const float2 zg = *reinterpret_cast<const float2*>(q + 2 * bz2);
+      const float2 zk = *reinterpret_cast<const float2*>(q + 3 * bz2);
+      const float sy = (i & 1) ? -1.f : 1.f;
+      // sum_s sigma_s z_s = (ll + sy lh) + sx (hl + sy hh)
+      const float a0 = fmaf(sy, zh.x, zl.x), b0 = fmaf(sy, zk.x, zg.x);
+      const float a1 = fmaf(sy, zh.y, zl.y), b1 = fmaf(sy, zk.y, zg.y);
+      float o0 = a0 + b0, o1 = a0 - b0, o2 = a1 + b1, o3 = a1 - b1;
       for (int l = 3; l <= P.L; ++l) {
         const BufDesc& z = P.zd[l];
         const int bz = z.ld * z.rows;
-        const float* q = sm + z.off + pb * z.ps + (i >> (l - 2)) * z.ld + (j >> (l - 2));
-        const int by = (i >> (l - 3)) & 1, bx = (j >> (l - 3)) & 1;
-        const float zlh = q[bz], zhl = q[2 * bz], zhh = q[3 * bz];
-        acc += q[0] + (by ? -zlh : zlh) + (bx ? -zhl : zhl) + ((by ^ bx) ? -zhh : zhh);
-      }
-      sm[P.t2.off + pb * P.t2.ps + i * P.t2.ld + j] = acc;
-    }
-    __syncthreads();
-  }
-  {
-    // level 2: conv of the 4 bands + t2 on LL, synthesis butterfly into t1
-    const int h2 = P.H >> 2, w2 = P.W >> 2;
-    const int tx = cdiv(w2, DP_CW), per = cdiv(h2, DP_R) * tx;
-    const BufDesc& d = P.sd[2];
-    const int bs = d.ld * d.rows;
-    for (int it = threadIdx.x; it < npb * per; it += NT) {
-      const int pb = it / per, rem = it - pb * per;
-      const int ti = rem / tx, tj = rem - ti * tx;
-      const int i0 = ti * DP_R, j0 = tj * DP_CW;
-      float acc[4][DP_R][DP_CW];
-#pragma unroll
-      for (int s = 0; s < 4; ++s)
-#pragma unroll
-        for (int a = 0; a < DP_R; ++a)
-#pragma unroll
-          for (int b = 0; b < DP_CW; ++b) acc[s][a][b] = 0.f;
-      const float* in = sm + d.off + pb * d.ps + i0 * d.ld + j0;
-#pragma unroll
-      for (int s = 0; s < 4; ++s) conv_tile<K, DP_R, DP_CW>(in + s * bs, d.ld, sw + wl_off(kk4, 2, s), acc[s]);
-      if (P.L >= 3) {
-        const float* t2 = sm + P.t2.off + pb * P.t2.ps + i0 * P.t2.ld + j0;
-#pragma unroll
-        for (int a = 0; a < DP_R; ++a) {
-          const float4 t = reinterpret_cast<const float4*>(t2 + a * P.t2.ld)[0];
-          acc[0][a][0] += t.x;
-          acc[0][a][1] += t.y;
-          acc[0][a][2] += t.z;
-          acc[0][a][3] += t.w;
+        const float* p = sm + z.off + pb * z.ps + (i >> (l - 1)) * z.ld + (j0 >> (l - 1));
+        const float syl = ((i >> (l - 2)) & 1) ? -1.f : 1.f;
+        const float A = fmaf(syl, p[bz], p[0]), B = fmaf(syl, p[3 * bz], p[2 * bz]);
+        if (l == 3) {  // bit1 of j: 0 for j0, j0+1 and 1 for j0+2, j0+3
+          o0 += A + B;
+          o1 += A + B;
+          o2 += A - B;
+          o3 += A - B;
+        } else {
+          const float sxl = ((j0 >> (l - 2)) & 1) ? -1.f : 1.f;
+          const float v = fmaf(sxl, B, A);
+          o0 += v;
+          o1 += v;
+          o2 += v;
+          o3 += v;
         }
       }
-      float* t1 = sm + P.t1.off + pb * P.t1.ps;
-#pragma unroll
-      for (int a = 0; a < DP_R; ++a)
-#pragma unroll
-        for (int b = 0; b < DP_CW; ++b) {
-          if (i0 + a < h2 && j0 + b < w2) {
-            float o00, o01, o10, o11;
-            synth4(acc[0][a][b], acc[1][a][b], acc[2][a][b], acc[3][a][b], o00, o01, o10, o11);
-            float* q = t1 + 2 * (i0 + a) * P.t1.ld + 2 * (j0 + b);
-            q[0] = o00;
-            q[1] = o01;
-            q[P.t1.ld] = o10;
-            q[P.t1.ld + 1] = o11;
-          }
-        }
+      *reinterpret_cast<float4*>(sm + P.t1.off + pb * P.t1.ps + i * P.t1.ld + j0) = make_float4(o0, o1, o2, o3);
     }
-    __syncthreads();
   }
+  __syncthreads();
 }
 
-// Level-1 band convs of the batch into zb (t1 added to the LL band).
-template <int K>
-__device__ void level1_conv(const Plan& P, float* sm, const float* sw, int npb) {
-  const int tx = cdiv(P.W1, C2_CW), per_band = cdiv(P.H1, C2_R) * tx, per = 4 * per_band;
-  const int bs1 = P.s1.ld * P.s1.rows, bsz = P.zb.ld * P.zb.rows;
-  for (int it = threadIdx.x; it < npb * per; it += NT) {
-    const int pb = it / per;
-    int rem = it - pb * per;
-    const int s = rem / per_band;
-    rem -= s * per_band;
-    const int ti = rem / tx, tj = rem - ti * tx;
-    const int i0 = ti * C2_R, j0 = tj * C2_CW;
-    float acc[C2_R][C2_CW];
-#pragma unroll
-    for (int a = 0; a < C2_R; ++a)
-#pragma unroll
-      for (int b = 0; b < C2_CW; ++b) acc[a][b] = 0.f;
-    conv_tile<K, C2_R, C2_CW>(sm + P.s1.off + pb * P.s1.ps + s * bs1 + i0 * P.s1.ld + j0, P.s1.ld,
-                              sw + wl_off(P.kk4, 1, s), acc);
-    if (s == 0 && P.L >= 2) {
-      const float* t1 = sm + P.t1.off + pb * P.t1.ps + i0 * P.t1.ld + j0;
-#pragma unroll
-      for (int a = 0; a < C2_R; ++a) {
-        const float4 t = reinterpret_cast<const float4*>(t1 + a * P.t1.ld)[0];
-        acc[a][0] += t.x;
-        acc[a][1] += t.y;
-        acc[a][2] += t.z;
-        acc[a][3] += t.w;
-      }
-    }
-    float* o = sm + P.zb.off + pb * P.zb.ps + s * bsz + i0 * P.zb.ld + j0;
-#pragma unroll
-    for (int a = 0; a < C2_R; ++a)
-      reinterpret_cast<float4*>(o + a * P.zb.ld)[0] = make_float4(acc[a][0], acc[a][1], acc[a][2], acc[a][3]);
-  }
-}
-
-// Base conv + level-1 synthesis + bias; writes the output rows.
+// --------------------------------------------------------------- output pass
+// Per R3 x 8 tile: the four level-1 band convs ((R3/2) x 4 each, folded
+// weights), t1 added to the LL band, the synthesis signs applied straight
+// into the accumulators, then the base conv; y is written once.
 template <int K, int R3, typename IO>
 __device__ void output_pass(const Plan& P, float* sm, const float* sw, IO* __restrict__ y, int c, int nb0,
                             int npb) {
-  const int tx = cdiv(P.W, C3_CW), per = cdiv(P.H, R3) * tx;
-  const int bsz = P.zb.ld * P.zb.rows;
+  constexpr int RB = R3 / 2;
+  const int tx = P.f_out_x.d, per = P.f_out_per.d;
+  const int bs1 = P.s1.ld * P.s1.rows;
   const float bias = sw[P.kk4];
-  for (int it = threadIdx.x; it < npb * per; it += NT) {
-    const int pb = it / per, rem = it - pb * per;
-    const int ti = rem / tx, tj = rem - ti * tx;
+  for (int it = threadIdx.x; it < npb * per; it += blockDim.x) {
+    const int pb = P.f_out_per.div(it);
+    const int rem = it - pb * per;
+    const int ti = P.f_out_x.div(rem);
+    const int tj = rem - ti * tx;
     const int yy0 = ti * R3, xx0 = tj * C3_CW;
     float acc[R3][C3_CW];
+#pragma unroll
+    for (int a = 0; a < R3; ++a)
+#pragma unroll
+      for (int b = 0; b < C3_CW; ++b) acc[a][b] = bias;
     if (P.L >= 1) {
+      const float* s1 = sm + P.s1.off + pb * P.s1.ps + (yy0 >> 1) * P.s1.ld + (xx0 >> 1);
 #pragma unroll
-      for (int bi = 0; bi < R3 / 2; ++bi) {
-        const float* z = sm + P.zb.off + pb * P.zb.ps + ((yy0 >> 1) + bi) * P.zb.ld + (xx0 >> 1);
-        const float4 zll = reinterpret_cast<const float4*>(z)[0];
-        const float4 zlh = reinterpret_cast<const float4*>(z + bsz)[0];
-        const float4 zhl = reinterpret_cast<const float4*>(z + 2 * bsz)[0];
-        const float4 zhh = reinterpret_cast<const float4*>(z + 3 * bsz)[0];
-        const float a0[4] = {zll.x, zll.y, zll.z, zll.w}, a1[4] = {zlh.x, zlh.y, zlh.z, zlh.w};
-        const float a2[4] = {zhl.x, zhl.y, zhl.z, zhl.w}, a3[4] = {zhh.x, zhh.y, zhh.z, zhh.w};
+      for (int s = 0; s < 4; ++s) {
+        float z[RB][4];
 #pragma unroll
-        for (int bj = 0; bj < 4; ++bj) {
-          float o00, o01, o10, o11;
-          synth4(a0[bj], a1[bj], a2[bj], a3[bj], o00, o01, o10, o11);
-          acc[2 * bi][2 * bj] = bias + o00;
-          acc[2 * bi][2 * bj + 1] = bias + o01;
-          acc[2 * bi + 1][2 * bj] = bias + o10;
-          acc[2 * bi + 1][2 * bj + 1] = bias + o11;
+        for (int a = 0; a < RB; ++a)
+#pragma unroll
+          for (int b = 0; b < 4; ++b) z[a][b] = 0.f;
+        conv_tile<K, RB, 4>(s1 + s * bs1, P.s1.ld, sw + wl_off(P.kk4, 1, s), z);
+        if (s == 0 && P.L >= 2) {
+          const float* t1 = sm + P.t1.off + pb * P.t1.ps + (yy0 >> 1) * P.t1.ld + (xx0 >> 1);
+#pragma unroll
+          for (int a = 0; a < RB; ++a) {
+            const float4 t = reinterpret_cast<const float4*>(t1 + a * P.t1.ld)[0];
+            z[a][0] += t.x;
+            z[a][1] += t.y;
+            z[a][2] += t.z;
+            z[a][3] += t.w;
+          }
         }
+        // sigma_s(py, px): LL +,+,+,+  LH +,+,-,-  HL +,-,+,-  HH +,-,-,+
+        const float s01 = (s == 2 || s == 3) ? -1.f : 1.f;
+        const float s10 = (s == 1 || s == 3) ? -1.f : 1.f;
+        const float s11 = (s == 1 || s == 2) ? -1.f : 1.f;
+#pragma unroll
+        for (int a = 0; a < RB; ++a)
+#pragma unroll
+          for (int b = 0; b < 4; ++b) {
+            const float v = z[a][b];
+            acc[2 * a][2 * b] += v;
+            acc[2 * a][2 * b + 1] = fmaf(s01, v, acc[2 * a][2 * b + 1]);
+            acc[2 * a + 1][2 * b] = fmaf(s10, v, acc[2 * a + 1][2 * b]);
+            acc[2 * a + 1][2 * b + 1] = fmaf(s11, v, acc[2 * a + 1][2 * b + 1]);
+          }
       }
-    } else {
-#pragma unroll
-      for (int a = 0; a < R3; ++a)
-#pragma unroll
-        for (int b = 0; b < C3_CW; ++b) acc[a][b] = bias;
     }
     conv_tile<K, R3, C3_CW>(sm + P.xf.off + pb * P.xf.ps + yy0 * P.xf.ld + xx0, P.xf.ld, sw, acc);
     const int n = P.W - xx0 < C3_CW ? P.W - xx0 : C3_CW;
@@ -351,36 +449,73 @@ __device__ void output_pass(const Plan& P, float* sm, const float* sw, IO* __res
 }
 
 // Forward / backward-data kernel.  Work unit: (channel c, batch of PB
-// consecutive n); grid-strided over C * nbatch units.
+// consecutive n); grid-strided over C * nbatch units.  When the planes can
+// be bulk-copied, the raw copy of unit u+1 is in flight while unit u runs
+// its deep levels and output pass.
 template <int K, int R3, typename IO>
-__global__ void __launch_bounds__(NT) wtconv_fwd_kernel(const Plan P, const IO* __restrict__ x,
-                                                        const float* __restrict__ w0, const float* __restrict__ b0,
-                                                        const float* __restrict__ s0, const float* __restrict__ wl,
-                                                        const float* __restrict__ sl, IO* __restrict__ y, int flip) {
+__global__ void __launch_bounds__(NT, 2) wtconv_fwd_kernel(const Plan P, const IO* __restrict__ x,
+                                                           const float* __restrict__ w0, const float* __restrict__ b0,
+                                                           const float* __restrict__ s0,
+                                                           const float* __restrict__ wl,
+                                                           const float* __restrict__ sl, IO* __restrict__ y,
+                                                           int flip, int* __restrict__ status) {
   extern __shared__ float4 smem4[];
   float* sm = reinterpret_cast<float*>(smem4);
-  for (int i = threadIdx.x; i < (P.smem_floats >> 2); i += NT) smem4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  uint64_t* mbar = reinterpret_cast<uint64_t*>(sm);
+  int* abort_flag = reinterpret_cast<int*>(sm + 2);
+  for (int i = threadIdx.x + 1; i < (P.smem_floats >> 2); i += blockDim.x)
+    smem4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (threadIdx.x == 0) {
+    smem4[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+    mbar_init(mbar);
+  }
   __syncthreads();
   const int units = P.C * P.nbatch;
+  const size_t plane = (size_t)P.H * P.W;
+  const size_t pstride = (size_t)P.C * plane;
   float* sw = sm + P.w_off;
+  IO* raw = reinterpret_cast<IO*>(sm + P.raw_off);
+  unsigned parity = 0;
+  if (P.use_bulk && threadIdx.x == 0 && (int)blockIdx.x < units) {
+    const int u = blockIdx.x, bt = u / P.C, c = u - bt * P.C, nb0 = bt * P.PB;
+    const int cnt = min(P.PB, P.N - nb0);
+    const unsigned bytes = (unsigned)(plane * sizeof(IO));
+    bulk_expect(mbar, bytes * cnt);
+    bulk_copies(mbar, raw, x + ((size_t)nb0 * P.C + c) * plane, pstride, cnt, bytes);
+  }
   for (int u = blockIdx.x; u < units; u += gridDim.x) {
-    const int c = u % P.C, bt = u / P.C;
+    const int bt = u / P.C;
+    const int c = u - bt * P.C;
     const int nb0 = bt * P.PB;
     const int npb = (P.N - nb0) < P.PB ? (P.N - nb0) : P.PB;
     load_weights<K>(P, sw, c, w0, b0, s0, wl, sl, flip);
-    for (int pb = 0; pb < npb; ++pb) {
-      const IO* xp = x + ((size_t)(nb0 + pb) * P.C + c) * P.H * P.W;
-      stage_plane<IO, false>(P, xp, sm + P.xf.off + pb * P.xf.ps, P.xf.ld, sm + P.s1.off + pb * P.s1.ps, P.s1.ld,
-                             P.s1.ld * P.s1.rows, true, nullptr);
-    }
-    __syncthreads();
-    if (P.L >= 2) deep_forward<K>(P, sm, sw, npb);
-    if (P.L >= 1) {
-      level1_conv<K>(P, sm, sw, npb);
+    if (P.use_bulk) {
+      if (threadIdx.x == 0 && !mbar_wait(mbar, parity)) *abort_flag = 1;
+      parity ^= 1u;
+      __syncthreads();
+      if (*abort_flag) break;
+      stage_planes<K, IO, true, false, true>(P, sm, raw, plane, npb, P.xf, P.s1, P.sd[2], nullptr);
+      __syncthreads();
+      const int un = u + gridDim.x;
+      if (threadIdx.x == 0 && un < units) {
+        const int btn = un / P.C, cn = un - btn * P.C, nbn = btn * P.PB;
+        const int cnt = min(P.PB, P.N - nbn);
+        const unsigned bytes = (unsigned)(plane * sizeof(IO));
+        bulk_expect(mbar, bytes * cnt);
+        bulk_copies(mbar, raw, x + ((size_t)nbn * P.C + cn) * plane, pstride, cnt, bytes);
+      }
+    } else {
+      stage_planes<K, IO, true, false, false>(P, sm, x + ((size_t)nb0 * P.C + c) * plane, pstride, npb, P.xf,
+                                              P.s1, P.sd[2], nullptr);
       __syncthreads();
     }
+    if (P.L >= 2) deep_forward<K>(P, sm, sw, npb);
     output_pass<K, R3, IO>(P, sm, sw, y, c, nb0, npb);
     __syncthreads();
+  }
+  if (*abort_flag && threadIdx.x == 0) {
+    if (status) atomicExch(status, 1);
+    mbar_wait(mbar, parity ^ 1u);  // let a late copy land before the CTA exits
   }
 }
 
@@ -396,62 +531,98 @@ __device__ __forceinline__ void zero_taps(float (&G)[K * K]) {
 // [G0: K*K][G1: 4*K*K] ... [GL: 4*K*K][sum dy].
 template <int K, typename IO>
 __global__ void __launch_bounds__(NT) wtconv_bwdw_kernel(const Plan P, const IO* __restrict__ x,
-                                                         const IO* __restrict__ dy, float* __restrict__ part) {
+                                                         const IO* __restrict__ dy, float* __restrict__ part,
+                                                         int* __restrict__ status) {
   constexpr int KK = K * K;
+  constexpr int r = K / 2;
   extern __shared__ float4 smem4[];
   float* sm = reinterpret_cast<float*>(smem4);
-  for (int i = threadIdx.x; i < (P.smem_floats >> 2); i += NT) smem4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  uint64_t* mbar = reinterpret_cast<uint64_t*>(sm);
+  int* abort_flag = reinterpret_cast<int*>(sm + 2);
+  for (int i = threadIdx.x + 1; i < (P.smem_floats >> 2); i += NT) smem4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (threadIdx.x == 0) {
+    smem4[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+    mbar_init(mbar);
+  }
   __syncthreads();
-  const int r = P.r;
   const int kk4 = P.kk4;
   const int c = blockIdx.x % P.C, g = blockIdx.x / P.C;
   const int n_begin = g * P.planes_per_cta;
   const int n_end = min(P.N, n_begin + P.planes_per_cta);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nbase = P.L >= 1 ? 128 : NT;   // threads on the base taps
+  const size_t plane = (size_t)P.H * P.W;
+  const size_t pstride = (size_t)P.C * plane;
+  IO* rawx = reinterpret_cast<IO*>(sm + P.raw_off);
+  IO* rawg = reinterpret_cast<IO*>(sm + P.rawg_off);
   float G[KK];
   zero_taps<K>(G);
   float sumdy = 0.f;
   const int ndeep = P.L >= 2 ? (P.L - 1) * 4 : 0;
+  unsigned parity = 0;
+  if (P.use_bulk && threadIdx.x == 0 && n_begin < n_end) {
+    const int cnt = min(P.PB, n_end - n_begin);
+    const unsigned bytes = (unsigned)(plane * sizeof(IO));
+    bulk_expect(mbar, 2 * bytes * cnt);
+    bulk_copies(mbar, rawx, x + ((size_t)n_begin * P.C + c) * plane, pstride, cnt, bytes);
+    bulk_copies(mbar, rawg, dy + ((size_t)n_begin * P.C + c) * plane, pstride, cnt, bytes);
+  }
 
   for (int nb0 = n_begin; nb0 < n_end; nb0 += P.PB) {
     const int npb = (n_end - nb0) < P.PB ? (n_end - nb0) : P.PB;
-    for (int pb = 0; pb < npb; ++pb) {
-      const size_t po = ((size_t)(nb0 + pb) * P.C + c) * P.H * P.W;
-      stage_plane<IO, false>(P, x + po, sm + P.xf.off + pb * P.xf.ps, P.xf.ld, sm + P.s1.off + pb * P.s1.ps,
-                             P.s1.ld, P.s1.ld * P.s1.rows, true, nullptr);
-      stage_plane<IO, true>(P, dy + po, sm + P.gf.off + pb * P.gf.ps, P.gf.ld, sm + P.g1.off + pb * P.g1.ps,
-                            P.g1.ld, P.g1.ld * P.g1.rows, false, &sumdy);
+    if (P.use_bulk) {
+      if (threadIdx.x == 0 && !mbar_wait(mbar, parity)) *abort_flag = 1;
+      parity ^= 1u;
+      __syncthreads();
+      if (*abort_flag) break;
+      stage_planes<K, IO, true, false, true>(P, sm, rawx, plane, npb, P.xf, P.s1, P.sd[2], nullptr);
+      stage_planes<K, IO, false, true, true>(P, sm, rawg, plane, npb, P.gf, P.g1, P.gd[2], &sumdy);
+      __syncthreads();
+      const int nn = nb0 + P.PB;
+      if (threadIdx.x == 0 && nn < n_end) {
+        const int cnt = min(P.PB, n_end - nn);
+        const unsigned bytes = (unsigned)(plane * sizeof(IO));
+        bulk_expect(mbar, 2 * bytes * cnt);
+        bulk_copies(mbar, rawx, x + ((size_t)nn * P.C + c) * plane, pstride, cnt, bytes);
+        bulk_copies(mbar, rawg, dy + ((size_t)nn * P.C + c) * plane, pstride, cnt, bytes);
+      }
+    } else {
+      stage_planes<K, IO, true, false, false>(P, sm, x + ((size_t)nb0 * P.C + c) * plane, pstride, npb, P.xf,
+                                              P.s1, P.sd[2], nullptr);
+      stage_planes<K, IO, false, true, false>(P, sm, dy + ((size_t)nb0 * P.C + c) * plane, pstride, npb, P.gf,
+                                              P.g1, P.gd[2], &sumdy);
+      __syncthreads();
     }
-    __syncthreads();
-    for (int l = 2; l <= P.L; ++l) {
-      const BufDesc& d = P.sd[l];
-      const BufDesc& e = P.gd[l];
-      const float* srcx = (l == 2) ? sm + P.s1.off + r * P.s1.ld + r : sm + P.sd[l - 1].off + r * P.sd[l - 1].ld + r;
-      const int ldsx = (l == 2) ? P.s1.ld : P.sd[l - 1].ld;
-      const float* srcg = (l == 2) ? sm + P.g1.off : sm + P.gd[l - 1].off;
-      const int ldsg = (l == 2) ? P.g1.ld : P.gd[l - 1].ld;
-      pyramid_level(npb, P.H >> l, P.W >> l, srcx, ldsx, P.xf.ps, sm + d.off + r * d.ld + r, d.ld, d.ld * d.rows,
-                    P.xf.ps);
-      pyramid_level(npb, P.H >> l, P.W >> l, srcg, ldsg, P.xf.ps, sm + e.off, e.ld, e.ld * e.rows, P.xf.ps);
+    for (int l = 3; l <= P.L; ++l) {
+      const BufDesc& sx = P.sd[l - 1];
+      const BufDesc& dx = P.sd[l];
+      const BufDesc& sg = P.gd[l - 1];
+      const BufDesc& dg = P.gd[l];
+      pyramid_level(npb, P.H >> l, P.W >> l, sm + sx.off + r * sx.ld + r, sx.ld, sx.ps, sm + dx.off + r * dx.ld + r,
+                    dx.ld, dx.ld * dx.rows, dx.ps);
+      pyramid_level(npb, P.H >> l, P.W >> l, sm + sg.off, sg.ld, sg.ps, sm + dg.off, dg.ld, dg.ld * dg.rows, dg.ps);
       __syncthreads();
     }
     // base and level-1 taps: register accumulation across planes
-    if (threadIdx.x < nbase) {
-      const int tx = cdiv(P.W, BW_CW), per = cdiv(P.H, BW_R) * tx;
+    if ((int)threadIdx.x < nbase) {
+      const int tx = P.f_bw_x.d, per = P.f_bw_per.d;
       for (int it = threadIdx.x; it < npb * per; it += nbase) {
-        const int pb = it / per, rem = it - pb * per;
-        const int ti = rem / tx, tj = rem - ti * tx;
+        const int pb = P.f_bw_per.div(it);
+        const int rem = it - pb * per;
+        const int ti = P.f_bw_x.div(rem);
+        const int tj = rem - ti * tx;
         const int y0 = ti * BW_R, x0 = tj * BW_CW;
         corr_tile<K, BW_R, BW_CW>(sm + P.xf.off + pb * P.xf.ps + y0 * P.xf.ld + x0, P.xf.ld,
                                   sm + P.gf.off + pb * P.gf.ps + y0 * P.gf.ld + x0, P.gf.ld, G);
       }
     } else {
       const int s = warp - 4;
-      const int tx = cdiv(P.W1, B1_CW), per = cdiv(P.H1, B1_R) * tx;
+      const int tx = P.f_b1_x.d, per = P.f_b1_per.d;
       for (int it = lane; it < npb * per; it += 32) {
-        const int pb = it / per, rem = it - pb * per;
-        const int ti = rem / tx, tj = rem - ti * tx;
+        const int pb = P.f_b1_per.div(it);
+        const int rem = it - pb * per;
+        const int ti = P.f_b1_x.div(rem);
+        const int tj = rem - ti * tx;
         const int i0 = ti * B1_R, j0 = tj * B1_CW;
         corr_tile<K, B1_R, B1_CW>(
             sm + P.s1.off + pb * P.s1.ps + s * P.s1.ld * P.s1.rows + i0 * P.s1.ld + j0, P.s1.ld,
@@ -464,15 +635,16 @@ __global__ void __launch_bounds__(NT) wtconv_bwdw_kernel(const Plan P, const IO*
       for (int it = threadIdx.x; it < ndeep * DSLOTS; it += NT) {
         const int br = it / DSLOTS, slot = it - br * DSLOTS;
         const int l = 2 + (br >> 2), s = br & 3;
-        const int hl = P.H >> l, wlv = P.W >> l;
-        const int tx = cdiv(wlv, DP_CW), per = cdiv(hl, DP_R) * tx;
+        const int tx = P.f_l_tx[l].d, per = P.f_l_tiles[l].d;
         const BufDesc& d = P.sd[l];
         const BufDesc& e = P.gd[l];
         float Gd[KK];
         zero_taps<K>(Gd);
         for (int t = slot; t < npb * per; t += DSLOTS) {
-          const int pb = t / per, rem = t - pb * per;
-          const int ti = rem / tx, tj = rem - ti * tx;
+          const int pb = P.f_l_tiles[l].div(t);
+          const int rem = t - pb * per;
+          const int ti = P.f_l_tx[l].div(rem);
+          const int tj = rem - ti * tx;
           const int i0 = ti * DP_R, j0 = tj * DP_CW;
           corr_tile<K, DP_R, DP_CW>(sm + d.off + pb * d.ps + s * d.ld * d.rows + i0 * d.ld + j0, d.ld,
                                     sm + e.off + pb * e.ps + s * e.ld * e.rows + i0 * e.ld + j0, e.ld, Gd);
@@ -492,6 +664,13 @@ __global__ void __launch_bounds__(NT) wtconv_bwdw_kernel(const Plan P, const IO*
       }
     }
     __syncthreads();
+  }
+  if (*abort_flag) {
+    if (threadIdx.x == 0) {
+      if (status) atomicExch(status, 1);
+      mbar_wait(mbar, parity ^ 1u);  // let a late copy land before the CTA exits
+    }
+    return;
   }
   // final fixed-order reduction of the register partials
   float* red = sm + P.red_off;

@@ -29,6 +29,23 @@ constexpr int BW_R = 4, BW_CW = 8;  // weight-gradient correlation, full resolut
 constexpr int B1_R = 4, B1_CW = 4;  // weight-gradient correlation, level 1
 constexpr int DSLOTS = 8;           // threads per deep (level, band) in the correlation pass
 
+// Division by a runtime divisor d >= 1 without an integer divide:
+// x / d == umulhi(x, m) >> s for 0 <= x < 2^31 (m, s set on the host).
+struct FDiv {
+  int d;
+  unsigned m;
+  int s;
+#ifdef __CUDACC__
+  __host__ __device__
+#endif
+  FDiv() : d(1), m(0), s(0) {}
+#ifdef __CUDACC__
+  __device__ __forceinline__ int div(int x) const {
+    return d == 1 ? x : (int)(__umulhi((unsigned)x, m) >> s);
+  }
+#endif
+};
+
 struct BufDesc {
   int off, ld, rows;   // rows allocated; band stride = ld * rows
   int ps;              // stride between the copies of consecutive planes of a batch
@@ -40,6 +57,11 @@ struct Plan {
   int R3;              // rows of the full-resolution register tile (2 or 4)
   int kk4;             // K*K rounded up to 4
   int vec_in, vec_out; // global rows allow 16-byte vector access
+  int prefetch_ok;     // plane bytes are a multiple of 16 (TMA bulk copies allowed)
+  int use_bulk;        // stage through TMA bulk copies into the raw buffer(s)
+  int raw_off, rawg_off;  // raw copies of x (and dy) of one batch, I/O dtype
+  int nthreads;        // threads per CTA of the forward kernel
+  int io_bytes;        // bytes per element of x, y, dy, dx
   // weights (folded): w0 [kk4], b0 [4], wl[l][s] [kk4] for l = 1..L
   int w_off;
   BufDesc xf;          // shifted: input plane (fp32)
@@ -57,6 +79,17 @@ struct Plan {
   int red_off;         // per-thread partial sums for the final reduction
   int gdeep_off;       // deep-level accumulators [L-1][4][kk4]
   int dpart_off;       // deep-level per-slot partials [L-1][4][DSLOTS][kk4]
+  // item decompositions of the forward phases (divisors per plane)
+  FDiv f_stage_per, f_stage_x;   // staging items per plane, per block row
+  FDiv f_deep_per;               // deep conv items per plane
+  FDiv f_t1_per, f_t1_x;         // t1 items per plane, per row
+  FDiv f_out_per, f_out_x;       // output tiles per plane, per tile row
+  FDiv f_bw_per, f_bw_x;         // weight-gradient base tiles per plane, per row
+  FDiv f_b1_per, f_b1_x;         // weight-gradient level-1 tiles per band, per row
+  FDiv f_l_tiles[MAXL + 1];      // deep conv tiles per band of level l
+  FDiv f_l_tx[MAXL + 1];         // deep conv tiles per tile row of level l
+  int deep_items;                // deep conv items per plane (levels 2..L)
+  int deep_first[MAXL + 2];      // first item of level l within a plane
   int PB;              // planes of one channel processed together (a batch)
   int nbatch;          // batches per channel: ceil(N / PB)
   int planes_per_cta;  // weight-gradient kernel: consecutive n per CTA

@@ -50,10 +50,10 @@ def _desc(N=2, C=3, H=16, W=16, k=5, L=2, io=0):
 def test_workspace_sizes(lib):
     d = _desc()
     V = 25 * (1 + 4 * 2) + 1
-    assert lib.wtconv_workspace_size(ctypes.byref(d), 0) == 0
-    assert lib.wtconv_workspace_size(ctypes.byref(d), 1) == 0
-    assert lib.wtconv_workspace_size(ctypes.byref(d), 2) == 2 * 3 * V * 4
-    assert lib.wtconv_workspace_size(ctypes.byref(d), 3) == 2 * 3 * V * 4
+    assert lib.wtconv_workspace_size(ctypes.byref(d), 0) == 16
+    assert lib.wtconv_workspace_size(ctypes.byref(d), 1) == 16
+    assert lib.wtconv_workspace_size(ctypes.byref(d), 2) == 16 + 2 * 3 * V * 4
+    assert lib.wtconv_workspace_size(ctypes.byref(d), 3) == 16 + 2 * 3 * V * 4
     assert lib.wtconv_workspace_size(ctypes.byref(_desc(k=4)), 2) == 0
     assert lib.wtconv_workspace_size(None, 2) == 0
 
