@@ -32,6 +32,15 @@
  *     allocates, frees or keeps state between calls.  Calls are asynchronous
  *     on `stream` (a cudaStream_t; NULL = legacy default stream) and never
  *     synchronise.
+ *   - Workspace (`ws`, `ws_bytes`): device memory of at least
+ *     wtconv_workspace_size(desc, op) bytes, 16-byte aligned.  Its first 16
+ *     bytes are a header whose first int is a device status word: a kernel
+ *     whose bounded wait for an asynchronous copy ran out of iterations sets
+ *     it to 1 (its outputs are then incomplete); the library never clears it,
+ *     so a caller that checks it zeroes it first.  For the forward and
+ *     backward-data passes the workspace is optional (NULL skips the status
+ *     word); the weight-gradient passes keep their partial sums after the
+ *     header and require it.
  *   - Arithmetic is fp32 throughout; bf16 I/O is rounded to nearest even on
  *     output.  Results are deterministic run to run (fixed reduction order).
  *   - Gradients are overwritten, not accumulated.
@@ -87,16 +96,16 @@ enum {
   WTCONV_OP_BACKWARD = 3
 };
 
-/* Bytes of device workspace the operation `op` needs for `desc` (0 when it
- * needs none, or when desc is invalid).  The weight-gradient pass keeps its
- * per-CTA partial sums there before the fixed-order second stage. */
+/* Bytes of device workspace the operation `op` uses for `desc` (0 when desc
+ * is invalid): the 16-byte status header, plus, for the weight-gradient
+ * passes, the per-CTA partial sums of the fixed-order two-stage reduction. */
 size_t wtconv_workspace_size(const wtconv_desc* desc, int op);
 
 /* Forward pass: y = WTConv(x).  Source: arXiv:2608.10805, abstract (the
  * layer; reformulations (1) on-chip Haar analysis, (2) single-pass
  * synthesis indexed by output-coordinate bits, (3) scales folded into the
  * convolution weights).  b0, s0 and w0 are required; wl, sl when L > 0.
- * ws may be NULL when wtconv_workspace_size(desc, 0) == 0. */
+ * ws is optional (status word only). */
 wtconv_status wtconv_forward(const wtconv_desc* desc, const void* x,
                              const float* w0, const float* b0, const float* s0,
                              const float* wl, const float* sl, void* y,
