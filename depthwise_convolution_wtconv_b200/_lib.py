@@ -16,11 +16,13 @@ LIB_PATH = os.path.join(_PKG, "libwtconv.so")
 F32, BF16 = 0, 1
 OP_FORWARD, OP_BACKWARD_DATA, OP_BACKWARD_WEIGHT, OP_BACKWARD = 0, 1, 2, 3
 STATUS_NAMES = {0: "WTCONV_OK", 1: "WTCONV_ERR_ARG", 2: "WTCONV_ERR_SHAPE", 3: "WTCONV_ERR_ALIGN",
-                4: "WTCONV_ERR_WORKSPACE", 5: "WTCONV_ERR_CUDA", 6: "WTCONV_ERR_UNSUPPORTED"}
+                4: "WTCONV_ERR_WORKSPACE", 5: "WTCONV_ERR_CUDA", 6: "WTCONV_ERR_UNSUPPORTED",
+                7: "WTCONV_ERR_SCRATCH_LIMIT"}
+NOALLOC_SCRATCH_BYTES = 8 << 20
 
 # every symbol include/wtconv.h declares
 EXPORTS = ("wtconv_workspace_size", "wtconv_forward", "wtconv_backward_data", "wtconv_backward_weight",
-           "wtconv_backward", "wtconv_status_string")
+           "wtconv_backward", "wtconv_backward_weight_noalloc", "wtconv_status_string")
 
 
 class WTConvDesc(ctypes.Structure):
@@ -57,6 +59,8 @@ def load(path=LIB_PATH):
     lib.wtconv_backward_weight.restype = ctypes.c_int
     lib.wtconv_backward.argtypes = [dp, vp, vp, fp, fp, fp, fp, fp, vp, fp, fp, fp, fp, fp, vp, sz, vp]
     lib.wtconv_backward.restype = ctypes.c_int
+    lib.wtconv_backward_weight_noalloc.argtypes = [dp, vp, vp, fp, fp, fp, fp, fp, fp, fp, fp, fp, fp, vp]
+    lib.wtconv_backward_weight_noalloc.restype = ctypes.c_int
     lib.wtconv_status_string.argtypes = [ctypes.c_int]
     lib.wtconv_status_string.restype = ctypes.c_char_p
     _lib = lib
@@ -173,6 +177,23 @@ def backward_weight(x, dy, w0, b0, s0, wl=None, sl=None, grads=None, ws=None, st
                                       _ptr(wl), _ptr(sl), _ptr(g["dw0"]), _ptr(g["db0"]), _ptr(g["ds0"]),
                                       _ptr(g["dwl"]), _ptr(g["dsl"]), _ptr(ws), nws, _stream(stream)),
            "wtconv_backward_weight")
+    return g
+
+
+def backward_weight_noalloc(x, dy, w0, b0, s0, wl=None, sl=None, grads=None, stream=None):
+    """Parameter gradients without a workspace: the library keeps its partial
+    sums in its own fixed device array (for callers that cannot allocate
+    device memory where they call it).  Same outputs as backward_weight."""
+    lib = load()
+    _cuda(x, "x")
+    _cuda(dy, "dy", x.dtype)
+    wl, sl = _params(w0, b0, s0, wl, sl)
+    desc = _desc_from(x, w0, wl)
+    g = _grad_outputs(w0, b0, s0, wl, sl, grads)
+    _check(lib.wtconv_backward_weight_noalloc(ctypes.byref(desc), _ptr(x), _ptr(dy), _ptr(w0), _ptr(b0), _ptr(s0),
+                                              _ptr(wl), _ptr(sl), _ptr(g["dw0"]), _ptr(g["db0"]), _ptr(g["ds0"]),
+                                              _ptr(g["dwl"]), _ptr(g["dsl"]), _stream(stream)),
+           "wtconv_backward_weight_noalloc")
     return g
 
 

@@ -6,6 +6,7 @@
 #include <algorithm>
 #include <cstdint>
 #include <initializer_list>
+#include <mutex>
 
 #include "wtconv.h"
 #include "wtconv_kernels.cuh"
@@ -347,7 +348,7 @@ template <int K, typename IO>
 wtconv_status launch_bwdw_t(Plan& P, const Device& dev, const void* x, const void* dy, const float* w0,
                             const float* b0, const float* s0, const float* wl, const float* sl, float* dw0,
                             float* db0, float* ds0, float* dwl, float* dsl, float* part, int* status,
-                            cudaStream_t st) {
+                            cudaStream_t st, int max_groups) {
   auto kern = wtconv_bwdw_kernel<K, IO>;
   const size_t smem = (size_t)P.smem_floats * 4;
   int occ = 0;
@@ -360,6 +361,7 @@ wtconv_status launch_bwdw_t(Plan& P, const Device& dev, const void* x, const voi
   for (int ppc = P.PB; ppc < P.N + P.PB; ppc += P.PB) {
     const int p = std::min(ppc, P.N);
     const int groups = (P.N + p - 1) / p;
+    if (groups > max_groups) continue;
     const long ctas = (long)P.C * groups;
     const long cost = ((ctas + slots - 1) / slots) * ((p + P.PB - 1) / P.PB);
     if (best < 0 || cost <= best) {
@@ -385,34 +387,48 @@ template <int K>
 wtconv_status launch_bwdw_k(Plan& P, const Device& dev, wtconv_dtype io, const void* x, const void* dy,
                             const float* w0, const float* b0, const float* s0, const float* wl, const float* sl,
                             float* dw0, float* db0, float* ds0, float* dwl, float* dsl, float* part, int* status,
-                            cudaStream_t st) {
+                            cudaStream_t st, int max_groups) {
   if (io == WTCONV_F32)
-    return launch_bwdw_t<K, float>(P, dev, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, part, status, st);
+    return launch_bwdw_t<K, float>(P, dev, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, part, status, st,
+                                   max_groups);
   return launch_bwdw_t<K, __nv_bfloat16>(P, dev, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, part, status,
-                                         st);
+                                         st, max_groups);
 }
 
-wtconv_status run_bwdw(const wtconv_desc* d, const void* x, const void* dy, const float* w0, const float* b0,
-                       const float* s0, const float* wl, const float* sl, float* dw0, float* db0, float* ds0,
-                       float* dwl, float* dsl, void* ws, cudaStream_t st) {
+// Runs the weight-gradient kernels with the per-CTA partial sums at `part`
+// and at most `max_groups` CTAs per channel (the partials then fill
+// max_groups * C * V floats).
+wtconv_status run_bwdw_part(const wtconv_desc* d, const void* x, const void* dy, const float* w0, const float* b0,
+                            const float* s0, const float* wl, const float* sl, float* dw0, float* db0, float* ds0,
+                            float* dwl, float* dsl, float* part, int* status, int max_groups, cudaStream_t st) {
   Device dev;
   wtconv_status e = query_device(dev);
   if (e != WTCONV_OK) return e;
   Plan P;
   build_bwdw_plan(P, d, dev.max_smem);
   if ((size_t)P.smem_floats * 4 > (size_t)dev.max_smem) return WTCONV_ERR_UNSUPPORTED;
-  int* status = static_cast<int*>(ws);
-  float* part = reinterpret_cast<float*>(static_cast<char*>(ws) + WS_HEADER);
   switch (d->k) {
     case 1:
-      return launch_bwdw_k<1>(P, dev, d->io, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, part, status, st);
+      return launch_bwdw_k<1>(P, dev, d->io, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, part, status, st,
+                              max_groups);
     case 3:
-      return launch_bwdw_k<3>(P, dev, d->io, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, part, status, st);
+      return launch_bwdw_k<3>(P, dev, d->io, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, part, status, st,
+                              max_groups);
     case 5:
-      return launch_bwdw_k<5>(P, dev, d->io, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, part, status, st);
+      return launch_bwdw_k<5>(P, dev, d->io, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, part, status, st,
+                              max_groups);
     default:
-      return launch_bwdw_k<7>(P, dev, d->io, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, part, status, st);
+      return launch_bwdw_k<7>(P, dev, d->io, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, part, status, st,
+                              max_groups);
   }
+}
+
+wtconv_status run_bwdw(const wtconv_desc* d, const void* x, const void* dy, const float* w0, const float* b0,
+                       const float* s0, const float* wl, const float* sl, float* dw0, float* db0, float* ds0,
+                       float* dwl, float* dsl, void* ws, cudaStream_t st) {
+  int* status = static_cast<int*>(ws);
+  float* part = reinterpret_cast<float*>(static_cast<char*>(ws) + WS_HEADER);
+  return run_bwdw_part(d, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, part, status, d->N, st);
 }
 
 wtconv_status check_ws(void* ws, size_t ws_bytes, size_t need) {
@@ -510,6 +526,65 @@ wtconv_status wtconv_backward(const wtconv_desc* desc, const void* x, const void
   return run_bwdw(desc, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, ws, st);
 }
 
+// ------------------------------------------------------------------------
+// Weight gradients for callers that cannot allocate device memory.
+//
+// Some callers have no way to hand the library a workspace: a plain C host
+// program or plugin that has no allocator of its own at the call site, a
+// runtime whose memory is fully reserved up front and forbids cudaMalloc
+// during steady-state steps, or code whose allocator lives in a framework it
+// cannot reach.  For them the partial sums of the weight-gradient reduction
+// live in this file-scope device array instead of a caller workspace.  Every
+// GPU that loads this library holds the array (WTCONV_NOALLOC_SCRATCH_BYTES)
+// until the process exits.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[WTCONV_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+constexpr int MAX_DEVICES = 64;
+std::mutex g_scratch_mutex;
+void* g_scratch_addr[MAX_DEVICES] = {};
+
+// Device address of g_noalloc_scratch on the current device.  In host code
+// the array's name is only a host-side stand-in, so the address is looked up
+// once per device (with that device current) and cached.
+wtconv_status noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return WTCONV_ERR_CUDA;
+  if (dev < 0 || dev >= MAX_DEVICES) return WTCONV_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (!g_scratch_addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return WTCONV_ERR_CUDA;
+    g_scratch_addr[dev] = p;
+  }
+  *out = g_scratch_addr[dev];
+  return WTCONV_OK;
+}
+}  // namespace
+
+wtconv_status wtconv_backward_weight_noalloc(const wtconv_desc* desc, const void* x, const void* dy,
+                                             const float* w0, const float* b0, const float* s0, const float* wl,
+                                             const float* sl, float* dw0, float* db0, float* ds0, float* dwl,
+                                             float* dsl, void* stream) {
+  wtconv_status e = check_desc(desc);
+  if (e != WTCONV_OK) return e;
+  if (!x || !dy) return WTCONV_ERR_ARG;
+  if ((e = check_params(desc, w0, b0, s0, wl, sl, true)) != WTCONV_OK) return e;
+  if ((e = check_grad_outputs(desc, dw0, db0, ds0, dwl, dsl)) != WTCONV_OK) return e;
+  if (!aligned16(x) || !aligned16(dy)) return WTCONV_ERR_ALIGN;
+  // one group of partial sums is C * V floats; at least one must fit
+  const size_t V = (size_t)desc->k * desc->k * (1 + 4 * desc->L) + 1;
+  const size_t group_bytes = (size_t)desc->C * V * sizeof(float);
+  const size_t groups = (WTCONV_NOALLOC_SCRATCH_BYTES - WS_HEADER) / group_bytes;
+  if (groups < 1) return WTCONV_ERR_SCRATCH_LIMIT;
+  void* scratch = nullptr;
+  if ((e = noalloc_scratch(&scratch)) != WTCONV_OK) return e;
+  float* part = reinterpret_cast<float*>(static_cast<char*>(scratch) + WS_HEADER);
+  const int max_groups = (int)std::min<size_t>(groups, (size_t)desc->N);
+  return run_bwdw_part(desc, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, part, nullptr, max_groups,
+                       static_cast<cudaStream_t>(stream));
+}
+
 const char* wtconv_status_string(wtconv_status s) {
   switch (s) {
     case WTCONV_OK: return "ok";
@@ -519,6 +594,8 @@ const char* wtconv_status_string(wtconv_status s) {
     case WTCONV_ERR_WORKSPACE: return "workspace missing or too small";
     case WTCONV_ERR_CUDA: return "CUDA error at launch";
     case WTCONV_ERR_UNSUPPORTED: return "shape needs more shared memory than one SM offers";
+    case WTCONV_ERR_SCRATCH_LIMIT:
+      return "shape needs more scratch than the built-in no-allocation buffer holds";
     default: return "unknown status";
   }
 }

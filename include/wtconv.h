@@ -53,6 +53,8 @@
  *       WTCONV_ERR_WORKSPACE ws_bytes < wtconv_workspace_size(desc, op)
  *       WTCONV_ERR_UNSUPPORTED  the shape needs more on-chip memory than
  *                            one SM offers
+ *       WTCONV_ERR_SCRATCH_LIMIT  (no-allocation variant only) the partial
+ *                            sums do not fit its built-in array
  *     and WTCONV_ERR_CUDA reports a launch failure (cudaGetLastError).
  *     Nothing is launched when a check fails.  No device-side trap exists.
  *   - With L = 0, wl and sl may be NULL.
@@ -85,7 +87,8 @@ typedef enum {
   WTCONV_ERR_ALIGN = 3,
   WTCONV_ERR_WORKSPACE = 4,
   WTCONV_ERR_CUDA = 5,
-  WTCONV_ERR_UNSUPPORTED = 6
+  WTCONV_ERR_UNSUPPORTED = 6,
+  WTCONV_ERR_SCRATCH_LIMIT = 7
 } wtconv_status;
 
 /* Operation codes for wtconv_workspace_size. */
@@ -147,6 +150,38 @@ wtconv_status wtconv_backward(const wtconv_desc* desc, const void* x,
                               void* dx, float* dw0, float* db0, float* ds0,
                               float* dwl, float* dsl, void* ws, size_t ws_bytes,
                               void* stream);
+
+/* Size of the device array that wtconv_backward_weight_noalloc uses in
+ * place of a workspace (8 MiB, held by every GPU that loads the library). */
+#define WTCONV_NOALLOC_SCRATCH_BYTES (8u << 20)
+
+/* Weight gradients without a workspace, for callers that cannot allocate
+ * device memory at the call site (a plain C host program or plugin with no
+ * allocator of its own there, a runtime whose memory is reserved up front and
+ * forbids cudaMalloc during steady-state steps, or code that cannot reach
+ * the allocator of the framework it runs in).  The paper has no counterpart:
+ * this is an interface variant of wtconv_backward_weight, with the same
+ * arguments minus ws/ws_bytes and the same outputs.
+ *
+ * The per-CTA partial sums go to a file-scope device array of
+ * WTCONV_NOALLOC_SCRATCH_BYTES instead; the library then uses fewer CTAs per
+ * channel if needed so they fit.  Shapes whose partial sums for one CTA per
+ * channel, C * (k*k*(1+4L)+1) floats plus a 16-byte header, exceed that size
+ * are rejected with WTCONV_ERR_SCRATCH_LIMIT before anything touches the GPU.
+ * The first call on each device looks up the array's device address (with
+ * that device current) and caches it; make that first call before any stream
+ * capture.  The call allocates nothing (no cudaMalloc, no cudaFree, no
+ * allocating library routine).  Every call on a device shares the one array,
+ * which keeps the last call's contents (each call overwrites every partial it
+ * reads): calls that overlap on the GPU, e.g. on two streams, race and must
+ * be serialised by the caller. */
+wtconv_status wtconv_backward_weight_noalloc(const wtconv_desc* desc,
+                                             const void* x, const void* dy,
+                                             const float* w0, const float* b0,
+                                             const float* s0, const float* wl,
+                                             const float* sl, float* dw0,
+                                             float* db0, float* ds0, float* dwl,
+                                             float* dsl, void* stream);
 
 /* Static description of a status code (never NULL). */
 const char* wtconv_status_string(wtconv_status status);
