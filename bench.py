@@ -165,17 +165,17 @@ def run_ours(args, wl, world, rank, local):
     dX = torch.empty_like(X)
     gflat, grads = grads_flat_views(wl, device)
     desc = wt.make_desc(wl.N, wl.C, wl.H, wl.W, wl.k, wl.L, wl.io)
-    ws = torch.empty(max(16, wt.workspace_size(desc, 2)), dtype=torch.uint8, device=device)
+    ws = torch.empty(max(16, wt.workspace_size(desc, 3)), dtype=torch.uint8, device=device)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
     stream = torch.cuda.current_stream(device)
 
     def step(ev=None, x=X, dy=dY, y=Y, dx=dX):
         if ev is not None:
             ev[0].record(stream)
-        wt.forward(x, p["W0"], p["b0"], p["s0"], Wl, sl, y=y, stream=stream)
+        wt.forward(x, p["W0"], p["b0"], p["s0"], Wl, sl, y=y, ws=ws, stream=stream)
         if ev is not None:
             ev[1].record(stream)
-        wt.backward_data(dy, p["W0"], p["s0"], Wl, sl, dx=dx, stream=stream)
+        wt.backward_data(dy, p["W0"], p["s0"], Wl, sl, dx=dx, ws=ws, stream=stream)
         if ev is not None:
             ev[2].record(stream)
         wt.backward_weight(x, dy, p["W0"], p["b0"], p["s0"], Wl, sl, grads=grads, ws=ws, stream=stream)
@@ -280,7 +280,7 @@ def run_ours(args, wl, world, rank, local):
         "kernels_ms": kernels,
         "e2e": {"value": world * 1000.0 / e2e_ms, "unit": "steps/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
-        "gpu_launches": 4 * args.steps,
+        "gpu_launches": (6 if wl.L >= 2 else 4) * args.steps,
         "clocks": clocks,
         "wall_s_timed_region": t_wall,
     }

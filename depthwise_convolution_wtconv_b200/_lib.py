@@ -121,8 +121,6 @@ def _params(w0, b0, s0, wl, sl):
 
 
 def _workspace(desc, op, ws):
-    if op in (OP_FORWARD, OP_BACKWARD_DATA) and ws is None:
-        return None, 0  # optional: only carries the device status word
     need = workspace_size(desc, op)
     if need == 0:
         return None, 0

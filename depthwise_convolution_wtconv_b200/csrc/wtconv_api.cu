@@ -10,6 +10,7 @@
 
 #include "wtconv.h"
 #include "wtconv_kernels.cuh"
+#include "wtconv_main.cuh"
 
 namespace wt {
 namespace {
@@ -243,6 +244,174 @@ void build_bwdw_plan(Plan& P, const wtconv_desc* d, int max_smem) {
   }
 }
 
+// ------------------------------------------------ pipelined output kernel
+int main_wblk(const wtconv_desc* d) { return rup((d->L >= 1 ? 5 : 1) * rup(d->k * d->k, 4) + 4, 4); }
+
+// Slot layout for band height TH and PB planes per unit; returns the slot
+// size in floats.
+int main_slot(MainPlan& M, int TH, int PB) {
+  const int r = M.r, RB = M.R3 / 2;
+  const int hx = M.L >= 1 ? 2 * r : r;
+  int cur = 0;
+  // region written by the producer's bulk copies and read by the stagers
+  M.wraw_off = cur;
+  cur += M.wblk;
+  M.raw_off = cur;
+  M.raw_pp = rup((int)(((size_t)std::min(M.H, TH + 2 * hx) * M.W * M.io_bytes + 3) / 4), 4);
+  cur += PB * M.raw_pp;
+  M.rawt_off = cur;
+  M.rawt_pp = (M.L >= 2 && M.bulk_t) ? rup((TH / 2) * M.W1, 4) : 0;
+  cur += PB * M.rawt_pp;
+  // region written by the stagers and read by the consumers
+  M.w_off = cur;
+  cur += M.wblk;
+  int pcur = 0;  // per-plane buffers, PB copies each
+  M.xf = make_shifted(pcur, TH, M.W, r, {{M.R3, C3_CW}}, 1);
+  if (M.L >= 1) M.s1 = make_shifted(pcur, TH / 2, M.W1, r, {{RB, 4}}, 4);
+  if (M.L >= 2) M.t1 = make_plain(pcur, TH / 2, M.W1, {{RB, 4}, {1, 4}}, 1);
+  const int pstride = rup(pcur, 4);
+  for (BufDesc* bd : {&M.xf, &M.s1, &M.t1}) {
+    bd->off += cur;
+    bd->ps = pstride;
+  }
+  cur += PB * pstride;
+  return rup(cur, 4);
+}
+
+bool build_main_plan(MainPlan& M, const wtconv_desc* d, int max_smem) {
+  M = MainPlan{};
+  M.N = d->N; M.C = d->C; M.H = d->H; M.W = d->W; M.K = d->k; M.r = d->k / 2; M.L = d->L;
+  M.H1 = d->L >= 1 ? d->H / 2 : d->H;
+  M.W1 = d->L >= 1 ? d->W / 2 : d->W;
+  M.kk4 = rup(d->k * d->k, 4);
+  M.io_bytes = io_bytes(d);
+  M.vec_in = (d->W % 4) == 0;
+  M.vec_out = d->io == WTCONV_BF16 ? (d->W % 8) == 0 : (d->W % 4) == 0;
+  M.R3 = d->H >= 8 ? 4 : 2;
+  M.wblk = main_wblk(d);
+  M.bulk_t = d->L >= 2 && (M.W1 % 4) == 0;
+  const int tx = cdiv_h(d->W, C3_CW);
+  // Largest band height (H itself, else an even divisor of H) whose slots fit
+  // in half of an SM's shared memory (two CTAs per SM).  Without bands, small
+  // planes are batched so that a unit has about one tile per consumer
+  // thread; then as many slots (2..4) as fit.
+  const size_t budget = (size_t)max_smem / 2;
+  int TH = -1, PB = 1, NS = 0;
+  for (int cand = d->H; cand >= 2 && TH < 0; --cand) {
+    if (d->H % cand || (cand != d->H && (cand & 1))) continue;
+    const int tpp = cdiv_h(cand, M.R3) * tx;
+    int pb = cand == d->H ? std::max(1, std::min(d->N, MAIN_CONSUMERS / tpp)) : 1;
+    for (; pb >= 1 && TH < 0; --pb) {
+      MainPlan T = M;
+      const int slot = main_slot(T, cand, pb);
+      for (int ns = MAIN_MAXSLOTS; ns >= 2; --ns) {
+        if ((size_t)(MAIN_HEADER + ns * slot) * 4 <= budget) {
+          TH = cand;
+          PB = pb;
+          NS = ns;
+          break;
+        }
+      }
+    }
+  }
+  if (TH < 0) return false;
+  M.TH = TH;
+  M.PB = PB;
+  M.nslots = NS;
+  M.nbands = d->H / TH;
+  M.units = d->C * ((d->N + PB - 1) / PB) * M.nbands;
+  M.slot_floats = main_slot(M, TH, PB);
+  M.slot0 = MAIN_HEADER;
+  M.smem_floats = M.slot0 + NS * M.slot_floats;
+  const size_t plane_bytes = (size_t)d->H * d->W * M.io_bytes;
+  M.bulk_x = M.nbands == 1 ? (plane_bytes % 16 == 0) : (((size_t)d->W * M.io_bytes) % 16 == 0);
+  const bool band = M.nbands > 1;
+  if (d->L >= 1) {
+    M.st_row0 = band ? -M.r : 0;
+    M.st_rows = band ? TH / 2 + 2 * M.r : M.H1;
+  } else {
+    M.st_row0 = band ? -M.r : 0;
+    M.st_rows = band ? TH + 2 * M.r : M.H;
+  }
+  M.st_q = cdiv_h(d->W, 4);
+  M.stage_pp = M.st_rows * M.st_q;
+  M.tiles_pp = cdiv_h(TH, M.R3) * tx;
+  M.tiles = PB * M.tiles_pp;
+  M.f_tiles = make_fdiv(M.tiles);
+  M.f_tpp = make_fdiv(M.tiles_pp);
+  M.f_tx = make_fdiv(tx);
+  M.f_stq = make_fdiv(M.st_q);
+  M.f_spp = make_fdiv(M.stage_pp);
+  M.f_bands = make_fdiv(M.nbands);
+  M.f_C = make_fdiv(d->C);
+  return true;
+}
+
+// ------------------------------------------------------------ deep kernel
+void deep_slab_items(DeepPlan& D, int& slab) {
+  const int r = D.r;
+  int cur = 0;
+  for (int l = 2; l <= D.L; ++l) D.sd[l] = make_shifted(cur, D.H >> l, D.W >> l, r, {{DP_R, DP_CW}, {2, 2}}, 4);
+  for (int l = 2; l <= D.L; ++l) D.zd[l] = make_plain(cur, D.H >> l, D.W >> l, {{DP_R, DP_CW}}, 4);
+  slab = rup(cur, 4);
+}
+
+bool build_deep_plan(DeepPlan& D, const wtconv_desc* d, int max_smem) {
+  D = DeepPlan{};
+  D.N = d->N; D.C = d->C; D.H = d->H; D.W = d->W; D.K = d->k; D.r = d->k / 2; D.L = d->L;
+  D.H1 = d->H / 2;
+  D.W1 = d->W / 2;
+  D.kk4 = rup(d->k * d->k, 4);
+  D.io_bytes = io_bytes(d);
+  D.vec_in = (d->W % 4) == 0;
+  int slab = 0;
+  deep_slab_items(D, slab);
+  D.w_off = 0;
+  const int base = rup((D.L - 1) * 4 * D.kk4, 4);
+  const int t1_items = D.H1 * cdiv_h(D.W1, 4);
+  int PB = std::max(1, std::min(d->N, DEEP_NT / std::max(1, t1_items)));
+  while (PB > 1 && (size_t)(base + PB * slab) * 4 > (size_t)max_smem / 2) --PB;
+  if ((size_t)(base + PB * slab) * 4 > (size_t)max_smem) return false;
+  D.PB = PB;
+  D.nbatch = (d->N + PB - 1) / PB;
+  for (int l = 0; l <= MAXL; ++l) {
+    D.sd[l].off += base;
+    D.sd[l].ps = slab;
+    D.zd[l].off += base;
+    D.zd[l].ps = slab;
+  }
+  D.smem_floats = base + PB * slab;
+  const int bw = D.W >> 2;
+  D.f_stage_per = make_fdiv((D.H >> 2) * bw);
+  D.f_stage_x = make_fdiv(bw);
+  int first = 0;
+  for (int l = 0; l <= MAXL + 1; ++l) D.deep_first[l] = 0;
+  for (int l = 2; l <= D.L; ++l) {
+    const int tx = cdiv_h(D.W >> l, DP_CW), tiles = cdiv_h(D.H >> l, DP_R) * tx;
+    D.f_l_tiles[l] = make_fdiv(tiles);
+    D.f_l_tx[l] = make_fdiv(tx);
+    D.deep_first[l] = first;
+    first += 4 * tiles;
+  }
+  D.deep_items = first;
+  D.deep_first[D.L + 1] = first;
+  D.f_deep_per = make_fdiv(first);
+  const int tq = cdiv_h(D.W1, 4);
+  D.f_t1_x = make_fdiv(tq);
+  D.f_t1_per = make_fdiv(D.H1 * tq);
+  return true;
+}
+
+size_t t1_bytes(const wtconv_desc* d) {
+  return d->L >= 2 ? (((size_t)d->N * d->C * (d->H / 2) * (d->W / 2) * sizeof(float) + 15) / 16) * 16 : 0;
+}
+
+// Forward / backward-data workspace: 16-byte header (status word), t1 of
+// every plane (levels >= 2), then the folded weights of every channel.
+size_t fwd_ws_bytes(const wtconv_desc* d) {
+  return 16 + t1_bytes(d) + (size_t)d->C * main_wblk(d) * sizeof(float);
+}
+
 wtconv_status check_desc(const wtconv_desc* d) {
   if (!d) return WTCONV_ERR_ARG;
   if (d->k < 1 || d->k > WTCONV_MAX_K || (d->k % 2) == 0) return WTCONV_ERR_ARG;
@@ -291,47 +460,72 @@ wtconv_status prepare(F kern, size_t smem, int& occ, int nthreads = NT) {
   return WTCONV_OK;
 }
 
-template <int K, int R3, typename IO>
-wtconv_status launch_fwd_t(const Plan& P, const Device& dev, const void* x, const float* w0, const float* b0,
-                           const float* s0, const float* wl, const float* sl, void* y, int flip, int* status,
-                           cudaStream_t st) {
-  auto kern = wtconv_fwd_kernel<K, R3, IO>;
-  const size_t smem = (size_t)P.smem_floats * 4;
+template <int K, typename IO>
+wtconv_status launch_forward_t(const wtconv_desc* d, const Device& dev, const void* x, const float* w0,
+                               const float* b0, const float* s0, const float* wl, const float* sl, void* y, int flip,
+                               int* status, float* t1, cudaStream_t st) {
+  float* wfold = reinterpret_cast<float*>(reinterpret_cast<char*>(t1) + t1_bytes(d));
+  {
+    const int kk4 = rup(d->k * d->k, 4), wblk = main_wblk(d);
+    const int n = d->C * wblk;
+    wtconv_fold_kernel<K><<<std::min((n + 255) / 256, dev.sms * 4), 256, 0, st>>>(d->C, d->L, kk4, wblk, w0, b0, s0,
+                                                                                   wl, sl, flip, wfold);
+    if (cudaGetLastError() != cudaSuccess) return WTCONV_ERR_CUDA;
+  }
+  if (d->L >= 2) {
+    DeepPlan D;
+    if (!build_deep_plan(D, d, dev.max_smem)) return WTCONV_ERR_UNSUPPORTED;
+    auto kd = wtconv_deep_kernel<K, IO>;
+    const size_t smem = (size_t)D.smem_floats * 4;
+    int occ = 0;
+    wtconv_status e = prepare(kd, smem, occ, DEEP_NT);
+    if (e != WTCONV_OK) return e;
+    const int units = D.C * D.nbatch;
+    kd<<<std::min(units, dev.sms * occ), DEEP_NT, smem, st>>>(D, static_cast<const IO*>(x), wl, sl, t1, flip);
+    if (cudaGetLastError() != cudaSuccess) return WTCONV_ERR_CUDA;
+  }
+  MainPlan M;
+  if (!build_main_plan(M, d, dev.max_smem)) return WTCONV_ERR_UNSUPPORTED;
+  const size_t smem = (size_t)M.smem_floats * 4;
   int occ = 0;
-  wtconv_status e = prepare(kern, smem, occ, P.nthreads);
-  if (e != WTCONV_OK) return e;
-  const int units = P.C * P.nbatch;
-  const int grid = std::min(units, dev.sms * occ);
-  kern<<<grid, P.nthreads, smem, st>>>(P, static_cast<const IO*>(x), w0, b0, s0, wl, sl, static_cast<IO*>(y), flip,
-                                       status);
+  if (M.R3 == 4) {
+    auto km = wtconv_main_kernel<K, 4, IO>;
+    wtconv_status e = prepare(km, smem, occ, MAIN_NT);
+    if (e != WTCONV_OK) return e;
+    km<<<std::min(M.units, dev.sms * occ), MAIN_NT, smem, st>>>(M, static_cast<const IO*>(x), t1, wfold,
+                                                                static_cast<IO*>(y), status);
+  } else {
+    auto km = wtconv_main_kernel<K, 2, IO>;
+    wtconv_status e = prepare(km, smem, occ, MAIN_NT);
+    if (e != WTCONV_OK) return e;
+    km<<<std::min(M.units, dev.sms * occ), MAIN_NT, smem, st>>>(M, static_cast<const IO*>(x), t1, wfold,
+                                                                static_cast<IO*>(y), status);
+  }
   return cudaGetLastError() == cudaSuccess ? WTCONV_OK : WTCONV_ERR_CUDA;
 }
 
 template <int K>
-wtconv_status launch_fwd_k(const Plan& P, const Device& dev, wtconv_dtype io, const void* x, const float* w0,
-                           const float* b0, const float* s0, const float* wl, const float* sl, void* y, int flip,
-                           int* status, cudaStream_t st) {
-  if (io == WTCONV_F32) {
-    if (P.R3 == 4) return launch_fwd_t<K, 4, float>(P, dev, x, w0, b0, s0, wl, sl, y, flip, status, st);
-    return launch_fwd_t<K, 2, float>(P, dev, x, w0, b0, s0, wl, sl, y, flip, status, st);
-  }
-  if (P.R3 == 4) return launch_fwd_t<K, 4, __nv_bfloat16>(P, dev, x, w0, b0, s0, wl, sl, y, flip, status, st);
-  return launch_fwd_t<K, 2, __nv_bfloat16>(P, dev, x, w0, b0, s0, wl, sl, y, flip, status, st);
+wtconv_status launch_forward_k(const wtconv_desc* d, const Device& dev, const void* x, const float* w0,
+                               const float* b0, const float* s0, const float* wl, const float* sl, void* y, int flip,
+                               int* status, float* t1, cudaStream_t st) {
+  if (d->io == WTCONV_F32) return launch_forward_t<K, float>(d, dev, x, w0, b0, s0, wl, sl, y, flip, status, t1, st);
+  return launch_forward_t<K, __nv_bfloat16>(d, dev, x, w0, b0, s0, wl, sl, y, flip, status, t1, st);
 }
 
+// Forward (flip = 0) or backward-data (flip = 1).  ws: 16-byte header (status
+// word) followed by t1 when L >= 2 (ws may be NULL when L < 2).
 wtconv_status run_forward(const wtconv_desc* d, const void* x, const float* w0, const float* b0, const float* s0,
-                          const float* wl, const float* sl, void* y, int flip, int* status, cudaStream_t st) {
+                          const float* wl, const float* sl, void* y, int flip, void* ws, cudaStream_t st) {
   Device dev;
   wtconv_status e = query_device(dev);
   if (e != WTCONV_OK) return e;
-  Plan P;
-  build_forward_plan(P, d, dev.max_smem);
-  if ((size_t)P.smem_floats * 4 > (size_t)dev.max_smem) return WTCONV_ERR_UNSUPPORTED;
+  int* status = static_cast<int*>(ws);
+  float* t1 = reinterpret_cast<float*>(static_cast<char*>(ws) + 16);
   switch (d->k) {
-    case 1: return launch_fwd_k<1>(P, dev, d->io, x, w0, b0, s0, wl, sl, y, flip, status, st);
-    case 3: return launch_fwd_k<3>(P, dev, d->io, x, w0, b0, s0, wl, sl, y, flip, status, st);
-    case 5: return launch_fwd_k<5>(P, dev, d->io, x, w0, b0, s0, wl, sl, y, flip, status, st);
-    default: return launch_fwd_k<7>(P, dev, d->io, x, w0, b0, s0, wl, sl, y, flip, status, st);
+    case 1: return launch_forward_k<1>(d, dev, x, w0, b0, s0, wl, sl, y, flip, status, t1, st);
+    case 3: return launch_forward_k<3>(d, dev, x, w0, b0, s0, wl, sl, y, flip, status, t1, st);
+    case 5: return launch_forward_k<5>(d, dev, x, w0, b0, s0, wl, sl, y, flip, status, t1, st);
+    default: return launch_forward_k<7>(d, dev, x, w0, b0, s0, wl, sl, y, flip, status, t1, st);
   }
 }
 
@@ -459,10 +653,11 @@ size_t wtconv_workspace_size(const wtconv_desc* desc, int op) {
   switch (op) {
     case WTCONV_OP_FORWARD:
     case WTCONV_OP_BACKWARD_DATA:
-      return WS_HEADER;
+      return fwd_ws_bytes(desc);
     case WTCONV_OP_BACKWARD_WEIGHT:
-    case WTCONV_OP_BACKWARD:
       return bwdw_ws_bytes(desc);
+    case WTCONV_OP_BACKWARD:
+      return std::max(bwdw_ws_bytes(desc), fwd_ws_bytes(desc));
     default:
       return 0;
   }
@@ -476,9 +671,8 @@ wtconv_status wtconv_forward(const wtconv_desc* desc, const void* x, const float
   if (!x || !y) return WTCONV_ERR_ARG;
   if ((e = check_params(desc, w0, b0, s0, wl, sl, true)) != WTCONV_OK) return e;
   if (!aligned16(x) || !aligned16(y)) return WTCONV_ERR_ALIGN;
-  if (ws && !aligned16(ws)) return WTCONV_ERR_ALIGN;
-  int* status = (ws && ws_bytes >= WS_HEADER) ? static_cast<int*>(ws) : nullptr;
-  return run_forward(desc, x, w0, b0, s0, wl, sl, y, 0, status, static_cast<cudaStream_t>(stream));
+  if ((e = check_ws(ws, ws_bytes, fwd_ws_bytes(desc))) != WTCONV_OK) return e;
+  return run_forward(desc, x, w0, b0, s0, wl, sl, y, 0, ws, static_cast<cudaStream_t>(stream));
 }
 
 wtconv_status wtconv_backward_data(const wtconv_desc* desc, const void* dy, const float* w0, const float* s0,
@@ -489,9 +683,8 @@ wtconv_status wtconv_backward_data(const wtconv_desc* desc, const void* dy, cons
   if (!dy || !dx) return WTCONV_ERR_ARG;
   if ((e = check_params(desc, w0, nullptr, s0, wl, sl, false)) != WTCONV_OK) return e;
   if (!aligned16(dy) || !aligned16(dx)) return WTCONV_ERR_ALIGN;
-  if (ws && !aligned16(ws)) return WTCONV_ERR_ALIGN;
-  int* status = (ws && ws_bytes >= WS_HEADER) ? static_cast<int*>(ws) : nullptr;
-  return run_forward(desc, dy, w0, nullptr, s0, wl, sl, dx, 1, status, static_cast<cudaStream_t>(stream));
+  if ((e = check_ws(ws, ws_bytes, fwd_ws_bytes(desc))) != WTCONV_OK) return e;
+  return run_forward(desc, dy, w0, nullptr, s0, wl, sl, dx, 1, ws, static_cast<cudaStream_t>(stream));
 }
 
 wtconv_status wtconv_backward_weight(const wtconv_desc* desc, const void* x, const void* dy, const float* w0,
@@ -519,9 +712,9 @@ wtconv_status wtconv_backward(const wtconv_desc* desc, const void* x, const void
   if ((e = check_params(desc, w0, b0, s0, wl, sl, true)) != WTCONV_OK) return e;
   if ((e = check_grad_outputs(desc, dw0, db0, ds0, dwl, dsl)) != WTCONV_OK) return e;
   if (!aligned16(x) || !aligned16(dy) || !aligned16(dx)) return WTCONV_ERR_ALIGN;
-  if ((e = check_ws(ws, ws_bytes, bwdw_ws_bytes(desc))) != WTCONV_OK) return e;
+  if ((e = check_ws(ws, ws_bytes, wtconv_workspace_size(desc, WTCONV_OP_BACKWARD))) != WTCONV_OK) return e;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  e = run_forward(desc, dy, w0, nullptr, s0, wl, sl, dx, 1, static_cast<int*>(ws), st);
+  e = run_forward(desc, dy, w0, nullptr, s0, wl, sl, dx, 1, ws, st);
   if (e != WTCONV_OK) return e;
   return run_bwdw(desc, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, ws, st);
 }

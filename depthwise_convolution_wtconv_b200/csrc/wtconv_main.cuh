@@ -1,0 +1,591 @@
+// Warp-specialised output kernel and deep-level kernel (sm_100a).
+//
+// Output kernel (forward and backward-data): one producer warp issues TMA
+// 1-D bulk copies (cp.async.bulk) of each unit's input rows and t1 rows into
+// a two-slot ring; two stager warps fold the channel's weights and turn the
+// raw rows into the zero-padded fp32 rows and the level-1 Haar subbands
+// (reformulation (1) of arXiv:2608.10805, abstract); six consumer warps run
+// register tiles back to back across units: the four level-1 band convs with
+// folded weights (reformulation (3)), t1 added to the LL band, the synthesis
+// signs, then the base conv, and store y.  Slots are handed over with
+// mbarriers (full / raw free / staged / empty) and a per-slot ready counter;
+// there is no CTA-wide barrier after set-up, so consumer lanes only idle at
+// the very end of the grid.
+//
+// Why a counter for "ready": a parity wait (mbarrier.try_wait.parity) reports
+// the phase before the current one as complete.  A consumer thread that has
+// no tile in a unit skips that unit's wait and can come to a slot's next use
+// while the slot's barrier is still one phase behind; a parity wait would
+// then pass at once.  Producer and stagers wait on every phase in order, so
+// their parity waits are safe; consumers wait on the monotonic counter.
+//
+// Deep kernel: levels 2..L of a batch of planes on chip (pyramid, every level
+// conv, then the closed-form synthesis of all levels >= 2 at level-1
+// resolution indexed by coordinate bits -- reformulation (2)), written as t1.
+#pragma once
+
+#include "wtconv_kernels.cuh"
+
+namespace wt {
+
+constexpr int MAIN_CONSUMERS = 128;  // warps 3-6
+constexpr int MAIN_STAGERS = 64;     // warps 1-2
+constexpr int MAIN_NT = 32 + MAIN_STAGERS + MAIN_CONSUMERS;
+constexpr int MAIN_MAXSLOTS = 4;
+constexpr int MAIN_HEADER = 48;      // floats: 16 mbarriers, abort flag, ready counters
+constexpr int DEEP_NT = 256;
+
+// ------------------------------------------------------------ mbarriers
+__device__ __forceinline__ unsigned smem_u32(const void* p) { return (unsigned)__cvta_generic_to_shared(p); }
+__device__ __forceinline__ void mb_init(uint64_t* b, unsigned count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(b)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mb_arrive(uint64_t* b) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(b)) : "memory");
+}
+__device__ __forceinline__ bool mb_try(uint64_t* b, unsigned parity) {
+  unsigned done;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(done)
+      : "r"(smem_u32(b)), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+// Waits for the phase with the given parity.  Gives up (returns false) when
+// another thread has raised the abort flag, or after an iteration limit, in
+// which case it raises the flag itself.
+__device__ __forceinline__ bool mb_wait(uint64_t* b, unsigned parity, volatile int* abort_flag) {
+  for (int i = 0; i < (1 << 22); ++i) {
+    if (mb_try(b, parity)) return true;
+    if (*abort_flag) return false;
+  }
+  *abort_flag = 1;
+  return false;
+}
+// Bounded wait that ignores the abort flag: used before exit so that bulk
+// copies already issued land before the CTA's shared memory is released.
+__device__ __forceinline__ void mb_drain(uint64_t* b, unsigned parity) {
+  for (int i = 0; i < (1 << 22); ++i)
+    if (mb_try(b, parity)) return;
+}
+__device__ __forceinline__ void st_release(int* p, int v) {
+  asm volatile("st.release.cta.shared::cta.u32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
+}
+__device__ __forceinline__ int ld_acquire(const int* p) {
+  int v;
+  asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)) : "memory");
+  return v;
+}
+// Waits until *seq >= want (bounded; abort-aware like mb_wait).
+__device__ __forceinline__ bool seq_wait(const int* seq, int want, volatile int* abort_flag) {
+  for (int i = 0; i < (1 << 24); ++i) {
+    if (ld_acquire(seq) >= want) return true;
+    if (*abort_flag) return false;
+  }
+  *abort_flag = 1;
+  return false;
+}
+
+// ------------------------------------------------------------ unit geometry
+// A unit is one band of one plane (nbands > 1) or a batch of npb planes of
+// one channel (nbands == 1, consecutive batch entries).
+struct UnitGeo {
+  int c, nb0, npb, y0, y_lo, y_hi;  // channel, first batch entry, planes, first output row, staged x rows
+};
+__device__ __forceinline__ UnitGeo unit_geo(const MainPlan& P, int u) {
+  UnitGeo g;
+  const int pg = P.f_bands.div(u);
+  const int b = u - pg * P.nbands;
+  const int bt = P.f_C.div(pg);
+  g.c = pg - bt * P.C;
+  g.nb0 = bt * P.PB;
+  g.npb = min(P.PB, P.N - g.nb0);
+  g.y0 = b * P.TH;
+  const int hx = P.L >= 1 ? 2 * P.r : P.r;
+  g.y_lo = max(0, g.y0 - hx);
+  g.y_hi = min(P.H, g.y0 + P.TH + hx);
+  return g;
+}
+__device__ __forceinline__ size_t plane_index(const MainPlan& P, const UnitGeo& g, int j) {
+  return (size_t)(g.nb0 + j) * P.C + g.c;
+}
+
+// Folded weights of every channel (one block of wblk floats per channel):
+//   [0, kk4): s0 * W0   [kk4]: s0 * b0 (0 for the adjoint)   [kk4+4 + s*kk4]:
+//   s_1[s] * W_1[s] / 2 (the level-1 synthesis factor); flipped for the adjoint.
+template <int K>
+__global__ void wtconv_fold_kernel(int C, int L, int kk4, int wblk, const float* __restrict__ w0,
+                                   const float* __restrict__ b0, const float* __restrict__ s0,
+                                   const float* __restrict__ wl, const float* __restrict__ sl, int flip,
+                                   float* __restrict__ out) {
+  constexpr int KK = K * K;
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < C * wblk; i += gridDim.x * blockDim.x) {
+    const int c = i / wblk, e = i - c * wblk;
+    float v = 0.f;
+    if (e < KK) {
+      v = s0[c] * w0[(size_t)c * KK + (flip ? KK - 1 - e : e)];
+    } else if (e == kk4) {
+      v = flip ? 0.f : s0[c] * b0[c];
+    } else if (L >= 1 && e >= kk4 + 4 && e < kk4 + 4 + 4 * kk4) {
+      const int s = (e - kk4 - 4) / kk4, t = (e - kk4 - 4) - s * kk4;
+      if (t < KK) {
+        const size_t base = (size_t)c * 4 + s;
+        v = (sl[base] * wl[base * KK + (flip ? KK - 1 - t : t)]) * 0.5f;
+      }
+    }
+    out[i] = v;
+  }
+}
+
+// Stager work for one plane of a unit: padded fp32 rows xf (band rows
+// [-r, TH+r)) and level-1 subbands s1 (half rows [-r, TH/2+r)), zero outside
+// the plane.  SMEM: rows come from the raw copy (row y at src + (y - y_lo) * W).
+template <int K, typename IO, bool SMEM>
+__device__ __forceinline__ void main_stage_item(const MainPlan& P, float* xf, float* s1, const IO* __restrict__ src,
+                                                const UnitGeo& g, int ri, int x0) {
+  constexpr int r = K / 2;
+  const bool vec = P.vec_in != 0;
+  const int ldx = P.xf.ld;
+  auto row_ptr = [&](int y) -> const IO* {
+    return SMEM ? src + (size_t)(y - g.y_lo) * P.W : src + (size_t)y * P.W;
+  };
+  if (P.L >= 1) {
+    const int ld1 = P.s1.ld, bs1 = P.s1.ld * P.s1.rows;
+    const int irel = P.st_row0 + ri;  // half row relative to the band
+    const int i = (g.y0 >> 1) + irel;  // absolute half row
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
+    if (i >= 0 && i < P.H1) {
+      a = src4<SMEM>(row_ptr(2 * i) + x0, x0, P.W, vec);
+      b = src4<SMEM>(row_ptr(2 * i + 1) + x0, x0, P.W, vec);
+    }
+    const int yrel = 2 * irel;
+    float* d0 = xf + (yrel + r) * ldx + x0 + r;
+    float* q1 = s1 + (irel + r) * ld1 + (x0 >> 1) + r;
+    float l0, h0, g0, k0, l1, h1, g1, k1;
+    haar4(a.x, a.y, b.x, b.y, l0, h0, g0, k0);
+    haar4(a.z, a.w, b.z, b.w, l1, h1, g1, k1);
+    const bool r0 = yrel >= -r && yrel < P.TH + r, r1 = yrel + 1 >= -r && yrel + 1 < P.TH + r;
+    if (x0 + 3 < P.W) {
+      if (r0) sts4<r>(d0, a);
+      if (r1) sts4<r>(d0 + ldx, b);
+      sts2<r>(q1, l0, l1);
+      sts2<r>(q1 + bs1, h0, h1);
+      sts2<r>(q1 + 2 * bs1, g0, g1);
+      sts2<r>(q1 + 3 * bs1, k0, k1);
+    } else {  // W % 4 == 2: one 2-wide block left in the row
+      if (r0) {
+        d0[0] = a.x;
+        d0[1] = a.y;
+      }
+      if (r1) {
+        d0[ldx] = b.x;
+        d0[ldx + 1] = b.y;
+      }
+      q1[0] = l0;
+      q1[bs1] = h0;
+      q1[2 * bs1] = g0;
+      q1[3 * bs1] = k0;
+    }
+  } else {
+    const int yrel = P.st_row0 + ri;
+    const int y = g.y0 + yrel;
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (y >= 0 && y < P.H) a = src4<SMEM>(row_ptr(y) + x0, x0, P.W, vec);
+    float* d0 = xf + (yrel + r) * ldx + x0 + r;
+    if (x0 + 3 < P.W) {
+      sts4<r>(d0, a);
+    } else {
+      const float av[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if (x0 + e < P.W) d0[e] = av[e];
+    }
+  }
+}
+
+// One output tile of plane j of a unit: (R3/2) x 4 band convs for the four
+// level-1 bands, t1 on LL, synthesis signs, base conv, store.
+template <int K, int R3, typename IO>
+__device__ __forceinline__ void main_tile(const MainPlan& P, const float* slot, const UnitGeo& g, int j, int tile,
+                                          IO* __restrict__ y) {
+  constexpr int RB = R3 / 2;
+  const int ti = P.f_tx.div(tile);
+  const int tj = tile - ti * P.f_tx.d;
+  const int yy0 = ti * R3, xx0 = tj * C3_CW;
+  const float* sw = slot + P.w_off;
+  const float bias = sw[P.kk4];
+  float acc[R3][C3_CW];
+#pragma unroll
+  for (int a = 0; a < R3; ++a)
+#pragma unroll
+    for (int b = 0; b < C3_CW; ++b) acc[a][b] = bias;
+  if (P.L >= 1) {
+    const int bs1 = P.s1.ld * P.s1.rows;
+    const float* s1 = slot + P.s1.off + j * P.s1.ps + (yy0 >> 1) * P.s1.ld + (xx0 >> 1);
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
+      float z[RB][4];
+#pragma unroll
+      for (int a = 0; a < RB; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) z[a][b] = 0.f;
+      conv_tile<K, RB, 4>(s1 + s * bs1, P.s1.ld, sw + P.kk4 + 4 + s * P.kk4, z);
+      if (s == 0 && P.L >= 2) {
+        const float* t1 = slot + P.t1.off + j * P.t1.ps + (yy0 >> 1) * P.t1.ld + (xx0 >> 1);
+#pragma unroll
+        for (int a = 0; a < RB; ++a) {
+          const float4 tv = reinterpret_cast<const float4*>(t1 + a * P.t1.ld)[0];
+          z[a][0] += tv.x;
+          z[a][1] += tv.y;
+          z[a][2] += tv.z;
+          z[a][3] += tv.w;
+        }
+      }
+      // sigma_s(py, px): LL +,+,+,+  LH +,+,-,-  HL +,-,+,-  HH +,-,-,+
+      const float s01 = (s == 2 || s == 3) ? -1.f : 1.f;
+      const float s10 = (s == 1 || s == 3) ? -1.f : 1.f;
+      const float s11 = (s == 1 || s == 2) ? -1.f : 1.f;
+#pragma unroll
+      for (int a = 0; a < RB; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+          const float v = z[a][b];
+          acc[2 * a][2 * b] += v;
+          acc[2 * a][2 * b + 1] = fmaf(s01, v, acc[2 * a][2 * b + 1]);
+          acc[2 * a + 1][2 * b] = fmaf(s10, v, acc[2 * a + 1][2 * b]);
+          acc[2 * a + 1][2 * b + 1] = fmaf(s11, v, acc[2 * a + 1][2 * b + 1]);
+        }
+    }
+  }
+  conv_tile<K, R3, C3_CW>(slot + P.xf.off + j * P.xf.ps + yy0 * P.xf.ld + xx0, P.xf.ld, sw, acc);
+  const int n = P.W - xx0 < C3_CW ? P.W - xx0 : C3_CW;
+  IO* yp = y + plane_index(P, g, j) * P.H * P.W;
+#pragma unroll
+  for (int a = 0; a < R3; ++a) {
+    const int yr = g.y0 + yy0 + a;
+    if (yy0 + a < P.TH && yr < P.H) store8(yp + (size_t)yr * P.W + xx0, acc[a], n, P.vec_out != 0);
+  }
+}
+
+template <int K, int R3, typename IO>
+__global__ void __launch_bounds__(MAIN_NT, 2)
+    wtconv_main_kernel(const MainPlan P, const IO* __restrict__ x, const float* __restrict__ t1g,
+                       const float* __restrict__ wfold, IO* __restrict__ y, int* __restrict__ status) {
+  extern __shared__ float4 smem4[];
+  float* sm = reinterpret_cast<float*>(smem4);
+  uint64_t* full = reinterpret_cast<uint64_t*>(sm);
+  uint64_t* rawfree = full + MAIN_MAXSLOTS;
+  uint64_t* staged = full + 2 * MAIN_MAXSLOTS;  // all stagers done with a use of the slot
+  uint64_t* empty = full + 3 * MAIN_MAXSLOTS;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + 32);
+  int* ready_seq = reinterpret_cast<int*>(sm + 36);  // slot s holds uses < ready_seq[s]
+  const int tid = threadIdx.x;
+  for (int i = tid + MAIN_HEADER / 4; i < (P.smem_floats >> 2); i += MAIN_NT)
+    smem4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (tid == 0) {
+    for (int i = 0; i < MAIN_HEADER / 4; ++i) smem4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s = 0; s < P.nslots; ++s) {
+      mb_init(full + s, 1);
+      mb_init(rawfree + s, MAIN_STAGERS);
+      mb_init(staged + s, MAIN_STAGERS);
+      mb_init(empty + s, P.tiles);
+    }
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  const int myunits = (int)blockIdx.x < P.units ? (P.units - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+  const int warp = tid >> 5;
+  const int NS = P.nslots;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------- producer
+    if (tid != 0) return;
+    int k = 0;
+    for (; k < myunits; ++k) {
+      const int u = blockIdx.x + k * gridDim.x, s = k % NS, use = k / NS;
+      if (use >= 1 && !mb_wait(rawfree + s, (use - 1) & 1, abort_flag)) break;
+      const UnitGeo g = unit_geo(P, u);
+      float* slot = sm + P.slot0 + s * P.slot_floats;
+      const unsigned bx = P.bulk_x ? (unsigned)((g.y_hi - g.y_lo) * P.W * P.io_bytes) : 0u;
+      const unsigned bt = (P.L >= 2 && P.bulk_t) ? (unsigned)((P.TH >> 1) * P.W1 * 4) : 0u;
+      const unsigned bw = (unsigned)(P.wblk * 4);
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(full + s)),
+                   "r"(bw + (bx + bt) * g.npb)
+                   : "memory");
+      asm volatile(
+          "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+              smem_u32(slot + P.wraw_off)),
+          "l"(wfold + (size_t)g.c * P.wblk), "r"(bw), "r"(smem_u32(full + s))
+          : "memory");
+      for (int j = 0; j < g.npb; ++j) {
+        const size_t pi = plane_index(P, g, j);
+        if (bx) {
+          const IO* src = x + pi * P.H * P.W + (size_t)g.y_lo * P.W;
+          asm volatile(
+              "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                  smem_u32(slot + P.raw_off + j * P.raw_pp)),
+              "l"(src), "r"(bx), "r"(smem_u32(full + s))
+              : "memory");
+        }
+        if (bt) {
+          const float* src = t1g + pi * P.H1 * P.W1 + (size_t)(g.y0 >> 1) * P.W1;
+          asm volatile(
+              "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                  smem_u32(slot + P.rawt_off + j * P.rawt_pp)),
+              "l"(src), "r"(bt), "r"(smem_u32(full + s))
+              : "memory");
+        }
+      }
+    }
+    // the copies already issued must land before this CTA can exit
+    for (int j = (k > NS ? k - NS : 0); j < k; ++j) mb_drain(full + (j % NS), (j / NS) & 1);
+    if (*abort_flag && status) atomicExch(status, 1);
+    return;
+  }
+
+  if (warp <= 2) {
+    // ---------------------------------------------------------- stagers
+    const int t = tid - 32;
+    for (int k = 0; k < myunits; ++k) {
+      const int u = blockIdx.x + k * gridDim.x, s = k % NS, use = k / NS;
+      if (!mb_wait(full + s, use & 1, abort_flag)) break;
+      if (use >= 1 && !mb_wait(empty + s, (use - 1) & 1, abort_flag)) break;
+      const UnitGeo g = unit_geo(P, u);
+      float* slot = sm + P.slot0 + s * P.slot_floats;
+      const int n = g.npb * P.stage_pp;
+      for (int it = t; it < n; it += MAIN_STAGERS) {
+        const int j = P.f_spp.div(it);
+        const int rem = it - j * P.stage_pp;
+        const int ri = P.f_stq.div(rem);
+        const int x0 = (rem - ri * P.st_q) << 2;
+        float* xf = slot + P.xf.off + j * P.xf.ps;
+        float* s1 = slot + P.s1.off + j * P.s1.ps;
+        if (P.bulk_x)
+          main_stage_item<K, IO, true>(P, xf, s1, reinterpret_cast<const IO*>(slot + P.raw_off + j * P.raw_pp), g,
+                                       ri, x0);
+        else
+          main_stage_item<K, IO, false>(P, xf, s1, x + plane_index(P, g, j) * P.H * P.W, g, ri, x0);
+      }
+      // folded weights and t1 rows move to the consumer side of the slot
+      for (int i = t; i < (P.wblk >> 2); i += MAIN_STAGERS)
+        reinterpret_cast<float4*>(slot + P.w_off)[i] = reinterpret_cast<const float4*>(slot + P.wraw_off)[i];
+      if (P.L >= 2) {
+        const int rows = P.TH >> 1, q4 = (P.W1 + 3) >> 2;
+        for (int it = t; it < g.npb * rows * q4; it += MAIN_STAGERS) {
+          const int j = it / (rows * q4), rem = it - j * rows * q4;
+          const int rr = rem / q4, x0 = (rem - rr * q4) << 2;
+          float4 v;
+          if (P.bulk_t) {
+            v = *reinterpret_cast<const float4*>(slot + P.rawt_off + j * P.rawt_pp + rr * P.W1 + x0);
+          } else {
+            const float* q = t1g + plane_index(P, g, j) * P.H1 * P.W1 + (size_t)((g.y0 >> 1) + rr) * P.W1 + x0;
+            v = load4(q, x0, P.W1, (P.W1 & 3) == 0);
+          }
+          *reinterpret_cast<float4*>(slot + P.t1.off + j * P.t1.ps + rr * P.t1.ld + x0) = v;
+        }
+      }
+      mb_arrive(rawfree + s);
+      mb_arrive(staged + s);
+      // stager 0 publishes the slot once every stager is done (in-order wait)
+      if (t == 0) {
+        if (!mb_wait(staged + s, use & 1, abort_flag)) break;
+        st_release(ready_seq + s, use + 1);
+      }
+    }
+    return;
+  }
+
+  // ------------------------------------------------------------ consumers
+  const int t = tid - 96;
+  const int total = myunits * P.tiles;
+  int cur = -1;
+  UnitGeo g{};
+  for (int gi = t; gi < total; gi += MAIN_CONSUMERS) {
+    const int k = P.f_tiles.div(gi);
+    const int tile = gi - k * P.tiles;
+    const int s = k % NS;
+    if (k != cur) {
+      if (!seq_wait(ready_seq + s, k / NS + 1, abort_flag)) break;
+      cur = k;
+      g = unit_geo(P, blockIdx.x + k * gridDim.x);
+    }
+    const int j = P.f_tpp.div(tile);
+    if (j < g.npb) main_tile<K, R3, IO>(P, sm + P.slot0 + s * P.slot_floats, g, j, tile - j * P.tiles_pp, y);
+    mb_arrive(empty + s);
+  }
+}
+
+// ------------------------------------------------------------ deep kernel
+// Levels 2..L of the planes of a batch: level-2 subbands from 4x4 blocks of
+// x, the rest of the pyramid, every level conv (folded weights
+// 2^-l s_l W_l), then t1 by the closed form, stored to global memory.
+template <int K, typename IO>
+__global__ void __launch_bounds__(DEEP_NT) wtconv_deep_kernel(const DeepPlan P, const IO* __restrict__ x,
+                                                              const float* __restrict__ wl,
+                                                              const float* __restrict__ sl, float* __restrict__ t1g,
+                                                              int flip) {
+  constexpr int r = K / 2;
+  constexpr int KK = K * K;
+  extern __shared__ float4 smem4[];
+  float* sm = reinterpret_cast<float*>(smem4);
+  for (int i = threadIdx.x; i < (P.smem_floats >> 2); i += DEEP_NT) smem4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  __syncthreads();
+  const int kk4 = P.kk4;
+  float* sw = sm + P.w_off;  // wlf[l][s] at ((l - 2) * 4 + s) * kk4
+  const size_t plane = (size_t)P.H * P.W;
+  const int units = P.C * P.nbatch;
+  for (int u = blockIdx.x; u < units; u += gridDim.x) {
+    const int bt = u / P.C;
+    const int c = u - bt * P.C;
+    const int nb0 = bt * P.PB;
+    const int npb = (P.N - nb0) < P.PB ? (P.N - nb0) : P.PB;
+    for (int i = threadIdx.x; i < (P.L - 1) * 4 * kk4; i += DEEP_NT) {
+      const int blk = i / kk4, e = i - blk * kk4;
+      float v = 0.f;
+      if (e < KK) {
+        const int l = blk / 4 + 2, s = blk & 3;
+        const int tt = flip ? (KK - 1 - e) : e;
+        const size_t base = ((size_t)(l - 1) * P.C + c) * 4 + s;
+        v = (sl[base] * wl[base * KK + tt]) * pow2neg(l);
+      }
+      sw[i] = v;
+    }
+    // level-2 subbands straight from 4x4 blocks of x (two blocks in flight)
+    {
+      const int bw = P.W >> 2, per = (P.H >> 2) * bw, n = npb * per;
+      const BufDesc& d = P.sd[2];
+      const int bs = d.ld * d.rows;
+      for (int it0 = threadIdx.x; it0 < n; it0 += 2 * DEEP_NT) {
+        float4 v[2][4];
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          const int it = it0 + q * DEEP_NT;
+          if (it < n) {
+            const int pb = P.f_stage_per.div(it);
+            const int rem = it - pb * per;
+            const int by = P.f_stage_x.div(rem);
+            const int x0 = (rem - by * bw) << 2;
+            const IO* src = x + ((size_t)(nb0 + pb) * P.C + c) * plane + (size_t)(by << 2) * P.W + x0;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) v[q][i] = load4(src + (size_t)i * P.W, x0, P.W, true);
+          }
+        }
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          const int it = it0 + q * DEEP_NT;
+          if (it < n) {
+            const int pb = P.f_stage_per.div(it);
+            const int rem = it - pb * per;
+            const int by = P.f_stage_x.div(rem);
+            const int bxi = rem - by * bw;
+            float ll[2][2];
+#pragma unroll
+            for (int a = 0; a < 2; ++a) {
+              float l0, h0, g0, k0, l1, h1, g1, k1;
+              haar4(v[q][2 * a].x, v[q][2 * a].y, v[q][2 * a + 1].x, v[q][2 * a + 1].y, l0, h0, g0, k0);
+              haar4(v[q][2 * a].z, v[q][2 * a].w, v[q][2 * a + 1].z, v[q][2 * a + 1].w, l1, h1, g1, k1);
+              ll[a][0] = l0;
+              ll[a][1] = l1;
+            }
+            float L2, H2, G2, K2;
+            haar4(ll[0][0], ll[0][1], ll[1][0], ll[1][1], L2, H2, G2, K2);
+            float* s2 = sm + d.off + pb * d.ps + (by + r) * d.ld + bxi + r;
+            s2[0] = L2;
+            s2[bs] = H2;
+            s2[2 * bs] = G2;
+            s2[3 * bs] = K2;
+          }
+        }
+      }
+    }
+    __syncthreads();
+    for (int l = 3; l <= P.L; ++l) {
+      const BufDesc& sb = P.sd[l - 1];
+      const BufDesc& d = P.sd[l];
+      pyramid_level(npb, P.H >> l, P.W >> l, sm + sb.off + r * sb.ld + r, sb.ld, sb.ps, sm + d.off + r * d.ld + r,
+                    d.ld, d.ld * d.rows, d.ps);
+      __syncthreads();
+    }
+    const int per = P.deep_items;
+    for (int it = threadIdx.x; it < npb * per; it += DEEP_NT) {
+      const int pb = P.f_deep_per.div(it);
+      int rem = it - pb * per;
+      int l = 2;
+      while (rem >= P.deep_first[l + 1]) ++l;
+      rem -= P.deep_first[l];
+      const int tpb = P.f_l_tiles[l].d;
+      const int s = P.f_l_tiles[l].div(rem);
+      rem -= s * tpb;
+      const int ti = P.f_l_tx[l].div(rem);
+      const int tj = rem - ti * P.f_l_tx[l].d;
+      const BufDesc& d = P.sd[l];
+      const BufDesc& z = P.zd[l];
+      float acc[DP_R][DP_CW];
+#pragma unroll
+      for (int a = 0; a < DP_R; ++a)
+#pragma unroll
+        for (int b = 0; b < DP_CW; ++b) acc[a][b] = 0.f;
+      conv_tile<K, DP_R, DP_CW>(sm + d.off + pb * d.ps + s * d.ld * d.rows + ti * DP_R * d.ld + tj * DP_CW, d.ld,
+                                sw + ((l - 2) * 4 + s) * kk4, acc);
+      float* o = sm + z.off + pb * z.ps + s * z.ld * z.rows + ti * DP_R * z.ld + tj * DP_CW;
+#pragma unroll
+      for (int a = 0; a < DP_R; ++a)
+        reinterpret_cast<float4*>(o + a * z.ld)[0] = make_float4(acc[a][0], acc[a][1], acc[a][2], acc[a][3]);
+    }
+    __syncthreads();
+    {
+      // t1(i, j) = sum_{l>=2} sum_s sigma_s(bit_{l-2}(i), bit_{l-2}(j)) Zd_l^s(i >> (l-1), j >> (l-1))
+      const int tq = P.f_t1_x.d, per1 = P.f_t1_per.d;
+      const BufDesc& z2 = P.zd[2];
+      const int bz2 = z2.ld * z2.rows;
+      for (int it = threadIdx.x; it < npb * per1; it += DEEP_NT) {
+        const int pb = P.f_t1_per.div(it);
+        const int rem = it - pb * per1;
+        const int i = P.f_t1_x.div(rem);
+        const int j0 = (rem - i * tq) << 2;
+        const float* q = sm + z2.off + pb * z2.ps + (i >> 1) * z2.ld + (j0 >> 1);
+        const float2 zl = *reinterpret_cast<const float2*>(q);
+        const float2 zh = *reinterpret_cast<const float2*>(q + bz2);
+        const float2 zg = *reinterpret_cast<const float2*>(q + 2 * bz2);
+        const float2 zk = *reinterpret_cast<const float2*>(q + 3 * bz2);
+        const float sy = (i & 1) ? -1.f : 1.f;
+        const float a0 = fmaf(sy, zh.x, zl.x), c0 = fmaf(sy, zk.x, zg.x);
+        const float a1 = fmaf(sy, zh.y, zl.y), c1 = fmaf(sy, zk.y, zg.y);
+        float o[4] = {a0 + c0, a0 - c0, a1 + c1, a1 - c1};
+        for (int l = 3; l <= P.L; ++l) {
+          const BufDesc& z = P.zd[l];
+          const int bz = z.ld * z.rows;
+          const float* pz = sm + z.off + pb * z.ps + (i >> (l - 1)) * z.ld + (j0 >> (l - 1));
+          const float syl = ((i >> (l - 2)) & 1) ? -1.f : 1.f;
+          const float A = fmaf(syl, pz[bz], pz[0]), B = fmaf(syl, pz[3 * bz], pz[2 * bz]);
+          if (l == 3) {  // bit1 of j: 0 for j0, j0+1 and 1 for j0+2, j0+3
+            o[0] += A + B;
+            o[1] += A + B;
+            o[2] += A - B;
+            o[3] += A - B;
+          } else {
+            const float sxl = ((j0 >> (l - 2)) & 1) ? -1.f : 1.f;
+            const float v = fmaf(sxl, B, A);
+            o[0] += v;
+            o[1] += v;
+            o[2] += v;
+            o[3] += v;
+          }
+        }
+        float* dst = t1g + ((size_t)(nb0 + pb) * P.C + c) * P.H1 * P.W1 + (size_t)i * P.W1 + j0;
+        if ((P.W1 & 3) == 0) {
+          *reinterpret_cast<float4*>(dst) = make_float4(o[0], o[1], o[2], o[3]);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            if (j0 + e < P.W1) dst[e] = o[e];
+        }
+      }
+    }
+    __syncthreads();
+  }
+}
+
+}  // namespace wt

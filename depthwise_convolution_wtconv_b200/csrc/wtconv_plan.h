@@ -99,3 +99,45 @@ struct Plan {
 };
 
 }  // namespace wt
+
+namespace wt {
+
+// Plan of the warp-specialised output kernel (forward and backward-data).
+// A unit is one band of TH output rows of one (n, c) plane (TH = H when the
+// whole plane fits in a slot).  The CTA owns a ring of two slots; each slot
+// holds the raw rows of one unit (TMA bulk copy), its t1 rows, the folded
+// base and level-1 weights of its channel, the padded fp32 rows xf and the
+// padded level-1 subbands s1.  Offsets are floats relative to a slot start.
+struct MainPlan {
+  int N, C, H, W, K, r, L, H1, W1, kk4, io_bytes;
+  int TH, nbands, PB;        // band rows, bands per plane, planes per unit (PB > 1 only without bands)
+  int units;                 // C * ceil(N/PB) * nbands
+  int nslots;                // ring slots (2..4)
+  int R3, tiles, tiles_pp;   // output tile rows, tiles per unit, per plane
+  int bulk_x, bulk_t;        // TMA bulk copies usable for x rows / t1 rows
+  int vec_in, vec_out;
+  int st_row0, st_rows, st_q, stage_pp;  // staged rows per plane (band), items per plane
+  int slot0, slot_floats;    // first slot offset, slot stride
+  int wblk;                  // floats of one channel's folded weights
+  int wraw_off, raw_off, rawt_off, raw_pp, rawt_pp;  // producer-written raw copies (per-plane strides)
+  int w_off;                 // stager-written folded weights read by the consumers
+  BufDesc xf, s1, t1;        // per-plane copies at ps stride
+  FDiv f_tiles, f_tpp, f_tx, f_stq, f_spp, f_bands, f_C;
+  int smem_floats;
+};
+
+// Plan of the deep-level kernel: levels 2..L of PB planes of one channel,
+// written as t1 (the synthesis of levels >= 2 at level-1 resolution,
+// already scaled by the level-1 synthesis factor) to global memory.
+struct DeepPlan {
+  int N, C, H, W, K, r, L, H1, W1, kk4, io_bytes, vec_in;
+  int PB, nbatch;
+  int w_off;                 // folded weights of levels 2..L
+  BufDesc sd[MAXL + 1], zd[MAXL + 1];
+  FDiv f_stage_per, f_stage_x, f_deep_per, f_t1_per, f_t1_x;
+  FDiv f_l_tiles[MAXL + 1], f_l_tx[MAXL + 1];
+  int deep_items, deep_first[MAXL + 2];
+  int smem_floats;
+};
+
+}  // namespace wt

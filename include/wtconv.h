@@ -37,10 +37,11 @@
  *     bytes are a header whose first int is a device status word: a kernel
  *     whose bounded wait for an asynchronous copy ran out of iterations sets
  *     it to 1 (its outputs are then incomplete); the library never clears it,
- *     so a caller that checks it zeroes it first.  For the forward and
- *     backward-data passes the workspace is optional (NULL skips the status
- *     word); the weight-gradient passes keep their partial sums after the
- *     header and require it.
+ *     so a caller that checks it zeroes it first.  After the header, the
+ *     forward and backward-data passes keep the folded weights of every
+ *     channel and, for L >= 2, the synthesis of levels >= 2 at level-1
+ *     resolution (fp32, N*C*(H/2)*(W/2)); the weight-gradient passes keep
+ *     their per-CTA partial sums.  The workspace is required.
  *   - Arithmetic is fp32 throughout; bf16 I/O is rounded to nearest even on
  *     output.  Results are deterministic run to run (fixed reduction order).
  *   - Gradients are overwritten, not accumulated.
@@ -100,15 +101,17 @@ enum {
 };
 
 /* Bytes of device workspace the operation `op` uses for `desc` (0 when desc
- * is invalid): the 16-byte status header, plus, for the weight-gradient
- * passes, the per-CTA partial sums of the fixed-order two-stage reduction. */
+ * is invalid): the 16-byte status header, then the folded weights and the
+ * level >= 2 synthesis (forward, backward-data) or the per-CTA partial sums
+ * of the fixed-order two-stage reduction (weight gradients); op 3 (both
+ * backward passes) is the larger of the two. */
 size_t wtconv_workspace_size(const wtconv_desc* desc, int op);
 
 /* Forward pass: y = WTConv(x).  Source: arXiv:2608.10805, abstract (the
  * layer; reformulations (1) on-chip Haar analysis, (2) single-pass
  * synthesis indexed by output-coordinate bits, (3) scales folded into the
  * convolution weights).  b0, s0 and w0 are required; wl, sl when L > 0.
- * ws is optional (status word only). */
+ * Needs wtconv_workspace_size(desc, 0) bytes of ws. */
 wtconv_status wtconv_forward(const wtconv_desc* desc, const void* x,
                              const float* w0, const float* b0, const float* s0,
                              const float* wl, const float* sl, void* y,
@@ -118,7 +121,8 @@ wtconv_status wtconv_forward(const wtconv_desc* desc, const void* x,
  * The adjoint of the +-1/2 Haar analysis is the synthesis and vice versa,
  * and the adjoint of each depthwise conv is the correlation with its
  * spatially flipped kernel, so this is the forward pass run on dy with
- * flipped kernels and no bias (arXiv:2608.10805, abstract: training). */
+ * flipped kernels and no bias (arXiv:2608.10805, abstract: training).
+ * Needs wtconv_workspace_size(desc, 1) bytes of ws. */
 wtconv_status wtconv_backward_data(const wtconv_desc* desc, const void* dy,
                                    const float* w0, const float* s0,
                                    const float* wl, const float* sl, void* dx,

@@ -50,16 +50,20 @@ def _desc(N=2, C=3, H=16, W=16, k=5, L=2, io=0):
 def test_workspace_sizes(lib):
     d = _desc()
     V = 25 * (1 + 4 * 2) + 1
-    assert lib.wtconv_workspace_size(ctypes.byref(d), 0) == 16
-    assert lib.wtconv_workspace_size(ctypes.byref(d), 1) == 16
+    t1 = 2 * 3 * 8 * 8 * 4  # level-1 resolution synthesis of levels >= 2
+    folded = 3 * (5 * 28 + 4) * 4  # per channel: base + 4 level-1 kernels (k*k padded to 28) + bias
+    assert lib.wtconv_workspace_size(ctypes.byref(d), 0) == 16 + t1 + folded
+    assert lib.wtconv_workspace_size(ctypes.byref(d), 1) == 16 + t1 + folded
     assert lib.wtconv_workspace_size(ctypes.byref(d), 2) == 16 + 2 * 3 * V * 4
-    assert lib.wtconv_workspace_size(ctypes.byref(d), 3) == 16 + 2 * 3 * V * 4
+    assert lib.wtconv_workspace_size(ctypes.byref(d), 3) == 16 + max(2 * 3 * V * 4, t1 + folded)
+    assert lib.wtconv_workspace_size(ctypes.byref(_desc(L=1)), 0) == 16 + folded
+    assert lib.wtconv_workspace_size(ctypes.byref(_desc(L=0)), 0) == 16 + 3 * (28 + 4) * 4
     assert lib.wtconv_workspace_size(ctypes.byref(_desc(k=4)), 2) == 0
     assert lib.wtconv_workspace_size(None, 2) == 0
 
 
-def _fwd(lib, d, x=FAKE, y=FAKE, w0=FAKE, b0=FAKE, s0=FAKE, wl=FAKE, sl=FAKE):
-    return lib.wtconv_forward(ctypes.byref(d) if d is not None else None, x, w0, b0, s0, wl, sl, y, None, 0, None)
+def _fwd(lib, d, x=FAKE, y=FAKE, w0=FAKE, b0=FAKE, s0=FAKE, wl=FAKE, sl=FAKE, ws=FAKE, nws=1 << 30):
+    return lib.wtconv_forward(ctypes.byref(d) if d is not None else None, x, w0, b0, s0, wl, sl, y, ws, nws, None)
 
 
 @pytest.mark.parametrize("kw,status", [
@@ -80,6 +84,9 @@ def test_forward_rejects_null_and_misaligned(lib):
     assert _fwd(lib, _desc(), x=FAKE_MIS) == ALIGN
     assert _fwd(lib, _desc(), y=FAKE + 8) == ALIGN
     assert _fwd(lib, _desc(), w0=FAKE + 2) == ALIGN
+    assert _fwd(lib, _desc(), ws=None) == WS
+    assert _fwd(lib, _desc(), nws=16) == WS
+    assert _fwd(lib, _desc(), ws=FAKE + 4) == ALIGN
 
 
 def test_level0_allows_null_level_params(lib):
@@ -91,9 +98,10 @@ def test_level0_allows_null_level_params(lib):
 def test_backward_data_checks(lib):
     d = _desc()
     f = lib.wtconv_backward_data
-    assert f(ctypes.byref(d), None, FAKE, FAKE, FAKE, FAKE, FAKE, None, 0, None) == ARG
-    assert f(ctypes.byref(d), FAKE_MIS, FAKE, FAKE, FAKE, FAKE, FAKE, None, 0, None) == ALIGN
-    assert f(ctypes.byref(_desc(W=10, L=2)), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, 0, None) == SHAPE
+    assert f(ctypes.byref(d), None, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 30, None) == ARG
+    assert f(ctypes.byref(d), FAKE_MIS, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 30, None) == ALIGN
+    assert f(ctypes.byref(_desc(W=10, L=2)), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 30, None) == SHAPE
+    assert f(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, 0, None) == WS
 
 
 def test_backward_weight_checks_workspace(lib):

@@ -89,6 +89,11 @@ EDGE = [
     Workload("multi_tile_L4", 2, 3, 64, 64, 5, 4, "f32"),
     Workload("L4_bf16", 3, 2, 48, 32, 5, 4, "bf16"),
     Workload("batchy_small", 37, 3, 14, 14, 5, 1, "f32"),
+    # more work units than resident CTAs: every slot of the ring is reused
+    Workload("reuse_L1_k5", 1, 1024, 8, 8, 5, 1, "f32"),
+    Workload("reuse_L3_k3", 2, 600, 16, 16, 3, 3, "f32"),
+    Workload("reuse_bf16_L2", 3, 500, 12, 12, 5, 2, "bf16"),
+    Workload("reuse_L0_k5", 2, 900, 14, 14, 5, 0, "f32"),
 ]
 
 
