@@ -337,6 +337,18 @@ bool build_main_plan(MainPlan& M, const wtconv_desc* d, int max_smem) {
   M.stage_pp = M.st_rows * M.st_q;
   M.tiles_pp = cdiv_h(TH, M.R3) * tx;
   M.tiles = PB * M.tiles_pp;
+  // consumer warp chunks: a unit of >= 32 tiles splits into ch_n balanced
+  // chunks; smaller units go ch_units whole units (at most nslots) a chunk
+  if (M.tiles >= 32) {
+    M.ch_units = 1;
+    M.ch_n = cdiv_h(M.tiles, 32);
+  } else {
+    M.ch_units = std::min(32 / M.tiles, NS);
+    M.ch_n = 1;
+  }
+  M.ch_base = M.ch_units * M.tiles / M.ch_n;
+  M.ch_rem = M.ch_units * M.tiles % M.ch_n;
+  M.f_chn = make_fdiv(M.ch_n);
   M.f_tiles = make_fdiv(M.tiles);
   M.f_tpp = make_fdiv(M.tiles_pp);
   M.f_tx = make_fdiv(tx);

@@ -2,10 +2,10 @@
 //
 // Output kernel (forward and backward-data): one producer warp issues TMA
 // 1-D bulk copies (cp.async.bulk) of each unit's input rows and t1 rows into
-// a two-slot ring; two stager warps fold the channel's weights and turn the
-// raw rows into the zero-padded fp32 rows and the level-1 Haar subbands
-// (reformulation (1) of arXiv:2608.10805, abstract); six consumer warps run
-// register tiles back to back across units: the four level-1 band convs with
+// a ring of two to four slots; three stager warps copy the channel's folded
+// weights and turn the raw rows into the zero-padded fp32 rows and the
+// level-1 Haar subbands (reformulation (1) of arXiv:2608.10805, abstract);
+// four consumer warps run register tiles back to back across units: the four level-1 band convs with
 // folded weights (reformulation (3)), t1 added to the LL band, the synthesis
 // signs, then the base conv, and store y.  Slots are handed over with
 // mbarriers (full / raw free / staged / empty) and a per-slot ready counter;
@@ -28,12 +28,12 @@
 
 namespace wt {
 
-constexpr int MAIN_CONSUMERS = 128;  // warps 3-6
-constexpr int MAIN_STAGERS = 64;     // warps 1-2
+constexpr int MAIN_CONSUMERS = 128;  // warps 4-7
+constexpr int MAIN_STAGERS = 96;     // warps 1-3
 constexpr int MAIN_NT = 32 + MAIN_STAGERS + MAIN_CONSUMERS;
 constexpr int MAIN_MAXSLOTS = 4;
 constexpr int MAIN_HEADER = 48;      // floats: 16 mbarriers, abort flag, ready counters
-constexpr int DEEP_NT = 256;
+constexpr int DEEP_NT = 128;
 
 // ------------------------------------------------------------ mbarriers
 __device__ __forceinline__ unsigned smem_u32(const void* p) { return (unsigned)__cvta_generic_to_shared(p); }
@@ -77,11 +77,15 @@ __device__ __forceinline__ int ld_acquire(const int* p) {
   asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)) : "memory");
   return v;
 }
-// Waits until *seq >= want (bounded; abort-aware like mb_wait).
+// Waits until *seq >= want (bounded; abort-aware like mb_wait), backing off
+// between polls so that a waiting warp leaves its issue slots to others.
 __device__ __forceinline__ bool seq_wait(const int* seq, int want, volatile int* abort_flag) {
-  for (int i = 0; i < (1 << 24); ++i) {
+  unsigned ns = 32;
+  for (int i = 0; i < (1 << 22); ++i) {
     if (ld_acquire(seq) >= want) return true;
     if (*abort_flag) return false;
+    __nanosleep(ns);
+    if (ns < 512) ns <<= 1;
   }
   *abort_flag = 1;
   return false;
@@ -345,7 +349,7 @@ __global__ void __launch_bounds__(MAIN_NT, 2)
     return;
   }
 
-  if (warp <= 2) {
+  if (warp <= MAIN_STAGERS / 32) {
     // ---------------------------------------------------------- stagers
     const int t = tid - 32;
     for (int k = 0; k < myunits; ++k) {
@@ -398,22 +402,39 @@ __global__ void __launch_bounds__(MAIN_NT, 2)
   }
 
   // ------------------------------------------------------------ consumers
-  const int t = tid - 96;
-  const int total = myunits * P.tiles;
-  int cur = -1;
-  UnitGeo g{};
-  for (int gi = t; gi < total; gi += MAIN_CONSUMERS) {
-    const int k = P.f_tiles.div(gi);
-    const int tile = gi - k * P.tiles;
-    const int s = k % NS;
-    if (k != cur) {
-      if (!seq_wait(ready_seq + s, k / NS + 1, abort_flag)) break;
-      cur = k;
-      g = unit_geo(P, blockIdx.x + k * gridDim.x);
+  // Warp-sized chunks that never straddle two units: a unit of >= 32 tiles
+  // is split into ch_n chunks of near-equal size; smaller units are grouped,
+  // ch_units whole units (at most nslots) per chunk.  Lane 0 waits for the
+  // newest unit of its chunk (units are published in order), the warp syncs,
+  // and every lane then works without spinning.  A chunk holds back only the
+  // slots of its own units, so the stagers refill a slot as soon as that
+  // unit's tiles are done.
+  const int cw = warp - 1 - MAIN_STAGERS / 32, lane = tid & 31;
+  const int total = cdiv(myunits, P.ch_units) * P.ch_n;
+  for (int g = cw; g < total; g += MAIN_CONSUMERS / 32) {
+    const int grp = P.f_chn.div(g);
+    const int jc = g - grp * P.ch_n;
+    const int k0 = grp * P.ch_units;
+    const int kmax = min(k0 + P.ch_units, myunits) - 1;
+    int ok = 1;
+    if (lane == 0) ok = seq_wait(ready_seq + kmax % NS, kmax / NS + 1, abort_flag);
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    if (!ok) break;
+    const int size = P.ch_base + (jc < P.ch_rem);
+    const int gi = jc * P.ch_base + min(jc, P.ch_rem) + lane;
+    if (lane < size) {
+      const int kk = P.f_tiles.div(gi);
+      const int k = k0 + kk;
+      if (k <= kmax) {
+        const int tile = gi - kk * P.tiles;
+        const int s = k % NS;
+        (void)ld_acquire(ready_seq + s);  // this lane's own acquire of the published slot
+        const UnitGeo u = unit_geo(P, blockIdx.x + k * gridDim.x);
+        const int j = P.f_tpp.div(tile);
+        if (j < u.npb) main_tile<K, R3, IO>(P, sm + P.slot0 + s * P.slot_floats, u, j, tile - j * P.tiles_pp, y);
+        mb_arrive(empty + s);
+      }
     }
-    const int j = P.f_tpp.div(tile);
-    if (j < g.npb) main_tile<K, R3, IO>(P, sm + P.slot0 + s * P.slot_floats, g, j, tile - j * P.tiles_pp, y);
-    mb_arrive(empty + s);
   }
 }
 

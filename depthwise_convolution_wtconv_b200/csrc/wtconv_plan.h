@@ -122,7 +122,9 @@ struct MainPlan {
   int wraw_off, raw_off, rawt_off, raw_pp, rawt_pp;  // producer-written raw copies (per-plane strides)
   int w_off;                 // stager-written folded weights read by the consumers
   BufDesc xf, s1, t1;        // per-plane copies at ps stride
-  FDiv f_tiles, f_tpp, f_tx, f_stq, f_spp, f_bands, f_C;
+  int ch_units, ch_n;        // consumer-warp chunks: units per chunk, chunks per unit group
+  int ch_base, ch_rem;       // chunk jc of a group holds ch_base + (jc < ch_rem) tiles
+  FDiv f_tiles, f_tpp, f_tx, f_stq, f_spp, f_bands, f_C, f_chn;
   int smem_floats;
 };
 
