@@ -58,6 +58,22 @@ def algorithmic_counts(wl):
     )
 
 
+def launches_per_step(wl):
+    """Kernels of this library launched per step: forward and backward-data
+    each run the weight-folding kernel, the deep-level kernel (L >= 2) and
+    the output kernel; backward-weight runs its partial-sum kernel and the
+    fixed-order finalize kernel."""
+    per_pass = 2 + (1 if wl.L >= 2 else 0)
+    return 2 * per_pass + 2
+
+
+PASS_KERNELS = {
+    "fwd": "wtconv_fold_kernel + wtconv_deep_kernel (L >= 2) + wtconv_main_kernel",
+    "bwd_data": "wtconv_fold_kernel + wtconv_deep_kernel (L >= 2) + wtconv_main_kernel (flipped)",
+    "bwd_weight": "wtconv_bwdw_kernel + wtconv_bwdw_finalize",
+}
+
+
 def load_peaks():
     try:
         with open(PEAKS_PATH) as f:
@@ -271,7 +287,7 @@ def run_ours(args, wl, world, rank, local):
         "config": {"workload": wl.name, **{k: v for k, v in wl.as_dict().items() if k != "name"},
                    "global_batch": wl.N * world, "parallelism": f"dp{world}",
                    "l2": "flushed before every timed step (256 MiB write)"},
-        "roofline": {"bound": "alu", "kernel": dom, "achieved": achieved_tflops,
+        "roofline": {"bound": "alu", "kernel": f"{dom} pass: {PASS_KERNELS[dom]}", "achieved": achieved_tflops,
                      "peak": fp32_peak_tflops, "unit": "TFLOP/s", "frac": achieved_tflops / fp32_peak_tflops,
                      "traffic": traffic,
                      "peak_source": f"{sms} SMs x {FP32_LANES_PER_SM} FP32 lanes x 2 x {sm_max:.0f} MHz"},
@@ -280,7 +296,7 @@ def run_ours(args, wl, world, rank, local):
         "kernels_ms": kernels,
         "e2e": {"value": world * 1000.0 / e2e_ms, "unit": "steps/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
-        "gpu_launches": (6 if wl.L >= 2 else 4) * args.steps,
+        "gpu_launches": launches_per_step(wl) * args.steps,
         "clocks": clocks,
         "wall_s_timed_region": t_wall,
     }
@@ -289,15 +305,26 @@ def run_ours(args, wl, world, rank, local):
     return line
 
 
+def sources_sha256():
+    """Hash of the CUDA sources, to tell whether committed counters still apply."""
+    import glob
+    import hashlib
+    paths = sorted(glob.glob(os.path.join(ROOT, "depthwise_convolution_wtconv_b200", "csrc", "*")))
+    return hashlib.sha256(b"".join(open(p, "rb").read() for p in paths)).hexdigest()
+
+
 def load_traffic(kernel, workload):
-    """DRAM bytes per launch from the committed ncu summary, if present."""
+    """DRAM bytes per launch from the committed ncu summary, or None when it
+    is missing or the kernels changed since the counters were taken."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             d = json.load(f)
-        return d.get(workload, {}).get(kernel)
     except (OSError, ValueError):
         return None
+    if d.get("sources_sha256") != sources_sha256():
+        return None
+    return d.get(workload, {}).get(kernel)
 
 
 def oracle_step(p):
@@ -314,9 +341,11 @@ def cpu_baseline(wl, sample_n):
     n = max(1, min(sample_n, wl.N))
     sub = dataclasses.replace(wl, N=n)
     p = as_float64(make_inputs(sub, 0))
-    t = time.perf_counter()
-    oracle_step(p)
-    dt = time.perf_counter() - t
+    from threadpoolctl import threadpool_limits
+    with threadpool_limits(limits=1):
+        t = time.perf_counter()
+        oracle_step(p)
+        dt = time.perf_counter() - t
     return {"value": (n / wl.N) / dt, "unit": "steps/s", "cores": 1, "kind": "oracle",
             "sample": f"N={n} of {wl.N} (same C, H, W, k, L), one fwd+bwd in numpy float64, "
                       f"single-threaded; host has {os.cpu_count()} cores; scaled by {n}/{wl.N}",
@@ -342,18 +371,21 @@ def run_reference(args, wl, world, rank):
     from depthwise_convolution_wtconv_b200.inputs import as_float64
     cal, cal_planes = _plane_sample(wl, min(8, wl.N * wl.C))
     pc = as_float64(make_inputs(cal, 0))
-    t = time.perf_counter()
-    oracle_step(pc)
-    tau = (time.perf_counter() - t) / cal_planes
+    from threadpoolctl import threadpool_limits
+    with threadpool_limits(limits=1):
+        t = time.perf_counter()
+        oracle_step(pc)
+        tau = (time.perf_counter() - t) / cal_planes
     planes = int(120.0 / max(1e-9, (args.steps + args.warmup) * tau))
     sub, planes = _plane_sample(wl, planes)
     p = as_float64(make_inputs(sub, 0))
-    for _ in range(args.warmup):
-        oracle_step(p)
-    t = time.perf_counter()
-    for _ in range(args.steps):
-        oracle_step(p)
-    dt = (time.perf_counter() - t) / args.steps
+    with threadpool_limits(limits=1):
+        for _ in range(args.warmup):
+            oracle_step(p)
+        t = time.perf_counter()
+        for _ in range(args.steps):
+            oracle_step(p)
+        dt = (time.perf_counter() - t) / args.steps
     frac = planes / (wl.N * wl.C)
     value = frac / dt
     sample = (f"{planes} of {wl.N * wl.C} (n, c) planes per step ({sub.N}x{sub.C}x{wl.H}x{wl.W}), numpy float64, "
