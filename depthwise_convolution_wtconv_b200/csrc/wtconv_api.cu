@@ -11,6 +11,7 @@
 #include "wtconv.h"
 #include "wtconv_kernels.cuh"
 #include "wtconv_main.cuh"
+#include "wtconv_bwband.cuh"
 
 namespace wt {
 namespace {
@@ -545,9 +546,130 @@ wtconv_status run_forward(const wtconv_desc* d, const void* x, const float* w0, 
 // then (weight gradients) the per-CTA partial sums.
 constexpr size_t WS_HEADER = 16;
 
+// Plan constants of sm_100a (B200): opt-in shared memory per CTA and SM
+// count.  The weight-gradient path and its workspace depend on the shape
+// only, through these, so wtconv_workspace_size needs no device query.
+constexpr int PLAN_SMEM = 232448;
+constexpr int PLAN_SMS = 148;
+
+// True when one plane's whole weight-gradient working set fits one SM.
+bool bwdw_whole_plane(const wtconv_desc* d) {
+  Plan P;
+  build_bwdw_plan(P, d, PLAN_SMEM);
+  return (size_t)P.smem_floats * 4 <= (size_t)PLAN_SMEM;
+}
+
+// ---- row-band weight-gradient path
+
+void band_layout(BandPlan& B, int TB) {
+  const int r = B.r;
+  const bool base = B.lvl <= 1, bands = B.lvl >= 1;
+  B.TB = TB;
+  B.nb = B.Hl / TB;
+  B.FR = B.lvl == 0 ? TB : 2 * TB;
+  const int nvb = (BW_CW + 2 * r + 3) / 4;
+  B.a_ld = rup(std::max(B.W + 2 * r, rup(B.W, BW_CW) - BW_CW + 4 * nvb), 4);
+  B.a_rows = B.FR + 2 * B.ha;
+  if (base) B.a_rows = std::max(B.a_rows, rup(B.FR, BW_R) + B.ha + r);
+  B.b_ld = rup(B.W, base ? BW_CW : 4);
+  B.b_rows = base ? rup(B.FR, BW_R) : B.FR;
+  if (bands) {
+    const int nv1 = (B1_CW + 2 * r + 3) / 4;
+    B.s_ld = rup(std::max(B.Wl + 2 * r, rup(B.Wl, B1_CW) - B1_CW + 4 * nv1), 4);
+    B.s_rows = rup(TB, B1_R) + 2 * r;
+    B.d_ld = rup(B.Wl, B1_CW);
+    B.d_rows = rup(TB, B1_R);
+  } else {
+    B.s_ld = B.s_rows = B.d_ld = B.d_rows = 0;
+  }
+  int cur = 0;
+  B.a_off = cur;
+  cur += rup(B.a_ld * B.a_rows, 4);
+  B.b_off = cur;
+  cur += rup(B.b_ld * B.b_rows, 4);
+  B.s_off = cur;
+  cur += rup(4 * B.s_ld * B.s_rows, 4);
+  B.d_off = cur;
+  cur += rup(4 * B.d_ld * B.d_rows, 4);
+  B.red_off = cur;
+  cur += rup((NT / 32) * B.kk4 + NT / 32, 4);
+  B.smem_floats = cur;
+  B.units = B.N * B.nb;
+  B.f_nb = make_fdiv(B.nb);
+  const int bx = cdiv_h(B.W, BW_CW);
+  B.f_bx = make_fdiv(bx);
+  B.f_bper = make_fdiv(base ? (rup(B.FR, BW_R) / BW_R) * bx : 1);
+  const int sx = bands ? cdiv_h(B.Wl, B1_CW) : 1;
+  B.f_sx = make_fdiv(sx);
+  B.f_sper = make_fdiv(bands ? cdiv_h(TB, B1_R) * sx : 1);
+}
+
+// Plan of the launch for level lvl (0 only when L = 0): the largest band
+// height that divides the level grid and leaves room for two CTAs per SM
+// (else one).  False when not even one row of the level grid fits.
+bool build_band_plan(BandPlan& B, const wtconv_desc* d, int lvl) {
+  B = BandPlan{};
+  B.N = d->N;
+  B.C = d->C;
+  B.K = d->k;
+  B.r = d->k / 2;
+  B.kk4 = rup(d->k * d->k, 4);
+  B.V = d->k * d->k * (1 + 4 * d->L) + 1;
+  B.lvl = lvl;
+  B.H = lvl == 0 ? d->H : d->H >> (lvl - 1);
+  B.W = lvl == 0 ? d->W : d->W >> (lvl - 1);
+  B.Hl = lvl == 0 ? B.H : B.H / 2;
+  B.Wl = lvl == 0 ? B.W : B.W / 2;
+  B.ha = lvl == 0 ? B.r : 2 * B.r;
+  B.vec = (B.W % 4) == 0;
+  B.write_ll = lvl >= 1 && lvl < d->L;
+  B.seg = lvl >= 1 ? d->k * d->k * (1 + 4 * (lvl - 1)) : 0;
+  for (const int budget : {PLAN_SMEM / 2, PLAN_SMEM}) {
+    for (int TB = B.Hl; TB >= 1; --TB) {
+      if (B.Hl % TB) continue;
+      band_layout(B, TB);
+      if ((size_t)B.smem_floats * 4 <= (size_t)budget) return true;
+    }
+  }
+  return false;
+}
+
+int band_first_level(const wtconv_desc* d) { return d->L == 0 ? 0 : 1; }
+
+// CTAs per channel of every band launch (the same for all, so that the
+// partials keep the whole-plane layout): enough CTAs for four per SM, at
+// most one per unit of the launch with the fewest units.  0 if a level
+// does not fit.
+int band_groups(const wtconv_desc* d) {
+  int umin = 1 << 30;
+  for (int lvl = band_first_level(d); lvl <= d->L; ++lvl) {
+    BandPlan B;
+    if (!build_band_plan(B, d, lvl)) return 0;
+    umin = std::min(umin, B.units);
+  }
+  const int target = (4 * PLAN_SMS + d->C - 1) / d->C;
+  return std::max(1, std::min(umin, target));
+}
+
+// Floats of the raw LL planes of x and dy that level l (1 <= l < L) hands
+// to level l + 1.
+size_t band_ll_floats(const wtconv_desc* d) {
+  size_t f = 0;
+  for (int l = 1; l < d->L; ++l) f += 2 * (size_t)d->N * d->C * (size_t)(d->H >> l) * (d->W >> l);
+  return f;
+}
+
+size_t band_part_bytes(const wtconv_desc* d, int groups) {
+  const size_t V = (size_t)d->k * d->k * (1 + 4 * d->L) + 1;
+  return (((size_t)groups * d->C * V * sizeof(float)) + 15) / 16 * 16;
+}
+
 size_t bwdw_ws_bytes(const wtconv_desc* d) {
   const size_t V = (size_t)d->k * d->k * (1 + 4 * d->L) + 1;
-  return WS_HEADER + (size_t)d->N * d->C * V * sizeof(float);
+  if (bwdw_whole_plane(d)) return WS_HEADER + (size_t)d->N * d->C * V * sizeof(float);
+  const int G = band_groups(d);
+  if (G == 0) return WS_HEADER;  // unsupported; the call reports it
+  return WS_HEADER + band_part_bytes(d, G) + band_ll_floats(d) * sizeof(float);
 }
 
 template <int K, typename IO>
@@ -610,6 +732,7 @@ wtconv_status run_bwdw_part(const wtconv_desc* d, const void* x, const void* dy,
   Device dev;
   wtconv_status e = query_device(dev);
   if (e != WTCONV_OK) return e;
+  if (dev.max_smem < PLAN_SMEM) return WTCONV_ERR_UNSUPPORTED;
   Plan P;
   build_bwdw_plan(P, d, dev.max_smem);
   if ((size_t)P.smem_floats * 4 > (size_t)dev.max_smem) return WTCONV_ERR_UNSUPPORTED;
@@ -629,12 +752,94 @@ wtconv_status run_bwdw_part(const wtconv_desc* d, const void* x, const void* dy,
   }
 }
 
+template <int K, typename IN>
+wtconv_status launch_band_level(const BandPlan& B, const void* a, const void* b, float* llx, float* lld, float* part,
+                                cudaStream_t st) {
+  auto kern = wtconv_bwband_kernel<K, IN>;
+  const size_t smem = (size_t)B.smem_floats * 4;
+  int occ = 0;
+  wtconv_status e = prepare(kern, smem, occ);
+  if (e != WTCONV_OK) return e;
+  kern<<<B.C * B.ngroups, NT, smem, st>>>(B, static_cast<const IN*>(a), static_cast<const IN*>(b), llx, lld, part);
+  return cudaGetLastError() == cudaSuccess ? WTCONV_OK : WTCONV_ERR_CUDA;
+}
+
+// Row-band path: one launch per level (the first on x and dy, the others on
+// the raw LL planes the level above wrote to `ll`), then the fixed-order
+// finalize over `groups` partial vectors per channel.
+template <int K>
+wtconv_status run_band_k(const wtconv_desc* d, const void* x, const void* dy, const float* w0, const float* b0,
+                         const float* s0, const float* wl, const float* sl, float* dw0, float* db0, float* ds0,
+                         float* dwl, float* dsl, float* part, float* ll, int groups, cudaStream_t st) {
+  const float* prevx = nullptr;
+  const float* prevd = nullptr;
+  size_t off = 0;
+  for (int lvl = band_first_level(d); lvl <= d->L; ++lvl) {
+    BandPlan B;
+    if (!build_band_plan(B, d, lvl)) return WTCONV_ERR_UNSUPPORTED;
+    B.ngroups = groups;
+    float* llx = nullptr;
+    float* lld = nullptr;
+    if (B.write_ll) {
+      const size_t n = (size_t)d->N * d->C * B.Hl * B.Wl;
+      llx = ll + off;
+      lld = ll + off + n;
+      off += 2 * n;
+    }
+    wtconv_status e;
+    if (lvl <= 1)
+      e = d->io == WTCONV_F32 ? launch_band_level<K, float>(B, x, dy, llx, lld, part, st)
+                              : launch_band_level<K, __nv_bfloat16>(B, x, dy, llx, lld, part, st);
+    else
+      e = launch_band_level<K, float>(B, prevx, prevd, llx, lld, part, st);
+    if (e != WTCONV_OK) return e;
+    prevx = llx;
+    prevd = lld;
+  }
+  Plan P;
+  fill_common(P, d);
+  P.ngroups = groups;
+  const size_t fsmem = (size_t)P.V * sizeof(float);
+  auto fin = wtconv_bwdw_finalize<K>;
+  if (fsmem > 48 * 1024 &&
+      cudaFuncSetAttribute(fin, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fsmem) != cudaSuccess)
+    return WTCONV_ERR_CUDA;
+  fin<<<P.C, 128, fsmem, st>>>(P, part, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl);
+  return cudaGetLastError() == cudaSuccess ? WTCONV_OK : WTCONV_ERR_CUDA;
+}
+
+wtconv_status run_band(const wtconv_desc* d, const void* x, const void* dy, const float* w0, const float* b0,
+                       const float* s0, const float* wl, const float* sl, float* dw0, float* db0, float* ds0,
+                       float* dwl, float* dsl, float* part, float* ll, int groups, cudaStream_t st) {
+  Device dev;
+  wtconv_status e = query_device(dev);
+  if (e != WTCONV_OK) return e;
+  if (dev.max_smem < PLAN_SMEM) return WTCONV_ERR_UNSUPPORTED;
+  switch (d->k) {
+    case 1:
+      return run_band_k<1>(d, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, part, ll, groups, st);
+    case 3:
+      return run_band_k<3>(d, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, part, ll, groups, st);
+    case 5:
+      return run_band_k<5>(d, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, part, ll, groups, st);
+    default:
+      return run_band_k<7>(d, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, part, ll, groups, st);
+  }
+}
+
+// Weight gradients with the workspace `ws` laid out as wtconv_workspace_size
+// sizes it (header, partial sums, and the LL planes of the row-band path).
 wtconv_status run_bwdw(const wtconv_desc* d, const void* x, const void* dy, const float* w0, const float* b0,
                        const float* s0, const float* wl, const float* sl, float* dw0, float* db0, float* ds0,
                        float* dwl, float* dsl, void* ws, cudaStream_t st) {
   int* status = static_cast<int*>(ws);
   float* part = reinterpret_cast<float*>(static_cast<char*>(ws) + WS_HEADER);
-  return run_bwdw_part(d, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, part, status, d->N, st);
+  if (bwdw_whole_plane(d))
+    return run_bwdw_part(d, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, part, status, d->N, st);
+  const int G = band_groups(d);
+  if (G == 0) return WTCONV_ERR_UNSUPPORTED;
+  float* ll = reinterpret_cast<float*>(static_cast<char*>(ws) + WS_HEADER + band_part_bytes(d, G));
+  return run_band(d, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, part, ll, G, st);
 }
 
 wtconv_status check_ws(void* ws, size_t ws_bytes, size_t need) {
@@ -777,17 +982,27 @@ wtconv_status wtconv_backward_weight_noalloc(const wtconv_desc* desc, const void
   if ((e = check_params(desc, w0, b0, s0, wl, sl, true)) != WTCONV_OK) return e;
   if ((e = check_grad_outputs(desc, dw0, db0, ds0, dwl, dsl)) != WTCONV_OK) return e;
   if (!aligned16(x) || !aligned16(dy)) return WTCONV_ERR_ALIGN;
-  // one group of partial sums is C * V floats; at least one must fit
+  // one group of partial sums is C * V floats; at least one must fit, with
+  // the LL planes of the row-band path when the planes need it
   const size_t V = (size_t)desc->k * desc->k * (1 + 4 * desc->L) + 1;
   const size_t group_bytes = (size_t)desc->C * V * sizeof(float);
-  const size_t groups = (WTCONV_NOALLOC_SCRATCH_BYTES - WS_HEADER) / group_bytes;
-  if (groups < 1) return WTCONV_ERR_SCRATCH_LIMIT;
+  const bool whole = bwdw_whole_plane(desc);
+  const size_t ll_bytes = whole ? 0 : band_ll_floats(desc) * sizeof(float);
+  const size_t avail = WTCONV_NOALLOC_SCRATCH_BYTES - WS_HEADER;
+  if (ll_bytes + 16 + group_bytes > avail) return WTCONV_ERR_SCRATCH_LIMIT;
+  const size_t groups = (avail - ll_bytes - 16) / group_bytes;
   void* scratch = nullptr;
   if ((e = noalloc_scratch(&scratch)) != WTCONV_OK) return e;
   float* part = reinterpret_cast<float*>(static_cast<char*>(scratch) + WS_HEADER);
-  const int max_groups = (int)std::min<size_t>(groups, (size_t)desc->N);
-  return run_bwdw_part(desc, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, part, nullptr, max_groups,
-                       static_cast<cudaStream_t>(stream));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (whole) {
+    const int max_groups = (int)std::min<size_t>(groups, (size_t)desc->N);
+    return run_bwdw_part(desc, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, part, nullptr, max_groups, st);
+  }
+  const int G = std::min<int>(band_groups(desc), (int)std::min<size_t>(groups, 1u << 20));
+  if (G == 0) return WTCONV_ERR_UNSUPPORTED;
+  float* ll = reinterpret_cast<float*>(static_cast<char*>(scratch) + WS_HEADER + band_part_bytes(desc, G));
+  return run_band(desc, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, part, ll, G, st);
 }
 
 const char* wtconv_status_string(wtconv_status s) {

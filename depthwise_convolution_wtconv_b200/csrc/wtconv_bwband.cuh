@@ -1,0 +1,186 @@
+// Row-band weight-gradient kernel for planes too large to keep whole in one
+// SM's shared memory (sm_100a).
+//
+// The weight gradients are sums over the image of local products, so they
+// split over row bands of a plane.  The pass runs one launch per level:
+//
+//   level 1 (or level 0 when L = 0): reads bands of x and dy; forms the base
+//     correlation G_0 = sum dy(i,j) x(i+u-r, j+v-r) and sum(dy) from the
+//     staged rows, and, for L >= 1, the Haar subbands of both on chip
+//     (reformulation (1) of arXiv:2608.10805, abstract) and their four band
+//     correlations G_1[s] = sum dZ_1^s(i,j) sub_1^s(i+u-r, j+v-r);
+//   level l >= 2: the same band correlations one level down, on the raw LL
+//     of the level above.
+//
+// Only the raw LL bands (a quarter of the level's input) go back to HBM for
+// the next launch; the detail subbands never leave the chip.  A band of TB
+// rows of the level grid needs 2*TB input rows of dy and 2*TB + 4r rows of
+// x (the correlation halo of r rows at the level grid).
+//
+// Each CTA owns channel c = blockIdx.x % C and the units (image n, band b)
+// u = g, g + G, g + 2G, ... of that channel (g = blockIdx.x / C); its
+// register sums are reduced by a fixed warp-shuffle tree and a fixed
+// warp order, and written to this launch's segment of the CTA's partial
+// vector part[g][c][V] (the layout of the whole-plane kernel).  Every
+// launch uses the same G, so the fixed-order finalize applies unchanged.
+#pragma once
+
+#include "wtconv_kernels.cuh"
+
+namespace wt {
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// Stages `rows` rows of a plane (row y0 first; rows outside [0, h) are
+// written as zeros) into shared memory at dst + i*ld + col0, converting to
+// fp32.  Returns this thread's sum of the staged in-image values when SUM.
+template <typename IN, bool SUM>
+__device__ __forceinline__ float stage_band_rows(const IN* __restrict__ src, int h, int w, int y0, int rows,
+                                                 float* __restrict__ dst, int ld, int col0, bool vec) {
+  float sum = 0.f;
+  const int q4 = (w + 3) >> 2;
+  for (int it = threadIdx.x; it < rows * q4; it += NT) {
+    const int i = it / q4, q = it - i * q4;
+    const int y = y0 + i, x = 4 * q;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (y >= 0 && y < h) v = load4(src + (size_t)y * w + x, x, w, vec);
+    float* o = dst + i * ld + col0 + x;
+    o[0] = v.x;
+    if (x + 1 < w) o[1] = v.y;
+    if (x + 2 < w) o[2] = v.z;
+    if (x + 3 < w) o[3] = v.w;
+    if (SUM) sum += (v.x + v.y) + (v.z + v.w);
+  }
+  return sum;
+}
+
+template <int K, typename IN>
+__global__ void __launch_bounds__(NT, 2) wtconv_bwband_kernel(const BandPlan P, const IN* __restrict__ A,
+                                                              const IN* __restrict__ B, float* __restrict__ llx,
+                                                              float* __restrict__ lld, float* __restrict__ part) {
+  constexpr int KK = K * K;
+  constexpr int r = K / 2;
+  extern __shared__ float4 smem4[];
+  float* sm = reinterpret_cast<float*>(smem4);
+  for (int i = threadIdx.x; i < (P.smem_floats >> 2); i += NT) smem4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  __syncthreads();
+  const int c = blockIdx.x % P.C, g = blockIdx.x / P.C;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nbase = P.lvl == 0 ? NT : (P.lvl == 1 ? 128 : 0);  // threads on the base taps
+  const int tpb = (NT - nbase) >> 2;                           // threads per subband
+  const size_t plane = (size_t)P.H * P.W;
+  float* sa = sm + P.a_off;
+  float* sb = sm + P.b_off;
+  float* ss = sm + P.s_off;
+  float* sd = sm + P.d_off;
+  const int s_band = P.s_ld * P.s_rows, d_band = P.d_ld * P.d_rows;
+  float G[KK];
+  zero_taps<K>(G);
+  float sumdy = 0.f;
+
+  for (int u = g; u < P.units; u += P.ngroups) {
+    const int n = P.f_nb.div(u), b = u - n * P.nb;
+    const int i0 = b * P.TB;                     // first row of the level grid
+    const int y0 = P.lvl == 0 ? i0 : 2 * i0;     // first input row of the band
+    const IN* a = A + ((size_t)n * P.C + c) * plane;
+    const IN* bb = B + ((size_t)n * P.C + c) * plane;
+    stage_band_rows<IN, false>(a, P.H, P.W, y0 - P.ha, P.FR + 2 * P.ha, sa, P.a_ld, r, P.vec);
+    const float sdy = stage_band_rows<IN, true>(bb, P.H, P.W, y0, P.FR, sb, P.b_ld, 0, P.vec);
+    if (P.lvl <= 1) sumdy += sdy;
+    __syncthreads();
+    if (P.lvl >= 1) {
+      // subbands of x over TB + 2r level rows (the halo rows outside the
+      // image come out zero from the zero rows staged above) and of dy over
+      // the TB band rows; raw LL of the band rows to the next level
+      const int wl = P.Wl;
+      const int nsub = (P.TB + 2 * r) * wl;
+      for (int it = threadIdx.x; it < nsub + P.TB * wl; it += NT) {
+        const bool isx = it < nsub;
+        const int k = isx ? it : it - nsub;
+        const int q = k / wl, jj = k - q * wl;
+        const float* src = isx ? sa + 2 * q * P.a_ld + r + 2 * jj : sb + 2 * q * P.b_ld + 2 * jj;
+        const int ld = isx ? P.a_ld : P.b_ld;
+        float ll, lh, hl, hh;
+        haar4(src[0], src[1], src[ld], src[ld + 1], ll, lh, hl, hh);
+        if (isx) {
+          float* o = ss + q * P.s_ld + r + jj;
+          o[0] = ll;
+          o[s_band] = lh;
+          o[2 * s_band] = hl;
+          o[3 * s_band] = hh;
+          const int qi = q - r;
+          if (P.write_ll && qi >= 0 && qi < P.TB)
+            llx[((size_t)n * P.C + c) * P.Hl * wl + (size_t)(i0 + qi) * wl + jj] = ll;
+        } else {
+          float* o = sd + q * P.d_ld + jj;
+          o[0] = ll;
+          o[d_band] = lh;
+          o[2 * d_band] = hl;
+          o[3 * d_band] = hh;
+          if (P.write_ll) lld[((size_t)n * P.C + c) * P.Hl * wl + (size_t)(i0 + q) * wl + jj] = ll;
+        }
+      }
+      __syncthreads();
+    }
+    if ((int)threadIdx.x < nbase) {
+      const int tx = P.f_bx.d, per = P.f_bper.d;
+      for (int it = threadIdx.x; it < per; it += nbase) {
+        const int ti = P.f_bx.div(it), tj = it - ti * tx;
+        const int yy = ti * BW_R, x0 = tj * BW_CW;
+        corr_tile<K, BW_R, BW_CW>(sa + (P.ha - r + yy) * P.a_ld + x0, P.a_ld, sb + yy * P.b_ld + x0, P.b_ld, G);
+      }
+    } else {
+      const int t = threadIdx.x - nbase;
+      const int s = t / tpb, lt = t - s * tpb;
+      const int tx = P.f_sx.d, per = P.f_sper.d;
+      for (int it = lt; it < per; it += tpb) {
+        const int ti = P.f_sx.div(it), tj = it - ti * tx;
+        const int q0 = ti * B1_R, j0 = tj * B1_CW;
+        corr_tile<K, B1_R, B1_CW>(ss + s * s_band + q0 * P.s_ld + j0, P.s_ld, sd + s * d_band + q0 * P.d_ld + j0,
+                                  P.d_ld, G);
+      }
+    }
+    __syncthreads();
+  }
+
+  // fixed-order reduction: shuffle tree within each warp, then warps in order
+  float* red = sm + P.red_off;
+#pragma unroll
+  for (int t = 0; t < KK; ++t) {
+    const float v = warp_sum(G[t]);
+    if (lane == 0) red[warp * P.kk4 + t] = v;
+  }
+  {
+    const float v = warp_sum(sumdy);
+    if (lane == 0) red[(NT / 32) * P.kk4 + warp] = v;
+  }
+  __syncthreads();
+  float* out = part + ((size_t)g * P.C + c) * P.V;
+  const int nbw = nbase >> 5, wpb = tpb >> 5;
+  if (P.lvl <= 1) {
+    for (int t = threadIdx.x; t < KK; t += NT) {
+      float acc = 0.f;
+      for (int w = 0; w < nbw; ++w) acc += red[w * P.kk4 + t];
+      out[t] = acc;
+    }
+    if (threadIdx.x == 0) {
+      float acc = 0.f;
+      for (int w = 0; w < NT / 32; ++w) acc += red[(NT / 32) * P.kk4 + w];
+      out[P.V - 1] = acc;
+    }
+  }
+  if (P.lvl >= 1) {
+    for (int e = threadIdx.x; e < 4 * KK; e += NT) {
+      const int s = e / KK, t = e - s * KK;
+      float acc = 0.f;
+      for (int w = 0; w < wpb; ++w) acc += red[(nbw + s * wpb + w) * P.kk4 + t];
+      out[P.seg + e] = acc;
+    }
+  }
+}
+
+}  // namespace wt

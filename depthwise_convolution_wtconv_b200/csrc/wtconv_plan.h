@@ -142,4 +142,28 @@ struct DeepPlan {
   int smem_floats;
 };
 
+// Plan of one launch of the row-band weight-gradient kernel.  The launch
+// correlates on the "level grid" (Hl x Wl): the image itself for lvl 0, the
+// level-lvl subbands for lvl >= 1, whose input planes A (x or a raw LL) and
+// B (dy or its raw LL) are H x W = 2Hl x 2Wl.  A band is TB rows of the
+// level grid.  Shared buffers (offsets and lds in floats, multiples of 4):
+//   a: FR + 2*ha input rows of A from row y0 - ha, column j at j + r
+//   b: FR input rows of B from row y0, column j at j
+//   s: 4 subbands of A over TB + 2r level rows from i0 - r, column j at j + r
+//   d: 4 subbands of B over the TB band rows, column j at j
+struct BandPlan {
+  int N, C, H, W, K, r, kk4, V;
+  int lvl, Hl, Wl;
+  int TB, nb, FR, ha;
+  int units, ngroups;
+  int a_off, a_ld, a_rows;
+  int b_off, b_ld, b_rows;
+  int s_off, s_ld, s_rows;
+  int d_off, d_ld, d_rows;
+  int red_off;               // (NT/32) * kk4 + NT/32 floats of the final reduction
+  int smem_floats;
+  int vec, write_ll, seg;
+  FDiv f_nb, f_bx, f_bper, f_sx, f_sper;
+};
+
 }  // namespace wt

@@ -62,6 +62,21 @@ def test_workspace_sizes(lib):
     assert lib.wtconv_workspace_size(None, 2) == 0
 
 
+def test_workspace_of_the_row_band_weight_gradient_path(lib):
+    """256x256 planes with 5 levels do not fit one SM: the weight-gradient
+    workspace then holds fewer partial-sum groups than N plus the raw LL
+    planes of x and dy that each level hands to the next."""
+    N, C, H, W, k, L = 16, 64, 256, 256, 5, 5
+    d = _lib.WTConvDesc(N, C, H, W, k, L, 1)
+    V = k * k * (1 + 4 * L) + 1
+    ll = sum(2 * N * C * (H >> l) * (W >> l) for l in range(1, L)) * 4
+    ws = lib.wtconv_workspace_size(ctypes.byref(d), 2)
+    part = ws - 16 - ll  # C * V * 4 = 134656 bytes, a multiple of 16: no rounding
+    assert part % (C * V * 4) == 0
+    assert 1 <= part // (C * V * 4) < N
+    assert lib.wtconv_workspace_size(ctypes.byref(d), 3) == max(ws, lib.wtconv_workspace_size(ctypes.byref(d), 0))
+
+
 def _fwd(lib, d, x=FAKE, y=FAKE, w0=FAKE, b0=FAKE, s0=FAKE, wl=FAKE, sl=FAKE, ws=FAKE, nws=1 << 30):
     return lib.wtconv_forward(ctypes.byref(d) if d is not None else None, x, w0, b0, s0, wl, sl, y, ws, nws, None)
 

@@ -94,6 +94,11 @@ EDGE = [
     Workload("reuse_L3_k3", 2, 600, 16, 16, 3, 3, "f32"),
     Workload("reuse_bf16_L2", 3, 500, 12, 12, 5, 2, "bf16"),
     Workload("reuse_L0_k5", 2, 900, 14, 14, 5, 0, "f32"),
+    # planes too large for one SM's shared memory: row-band weight gradients
+    Workload("band_L0_k3", 2, 3, 224, 224, 3, 0, "f32"),
+    Workload("band_L1_bf16", 1, 2, 192, 160, 5, 1, "bf16"),
+    Workload("band_L3_k7", 2, 2, 256, 128, 7, 3, "f32"),
+    Workload("band_ragged_L2", 1, 2, 200, 180, 3, 2, "f32"),
 ]
 
 

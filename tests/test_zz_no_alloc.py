@@ -46,6 +46,8 @@ CASES = [
     # must use fewer CTAs per channel than it would with a workspace
     Workload("many_channels", 8, 2048, 16, 16, 5, 2, "f32"),
     Workload("bf16_L0", 6, 64, 28, 28, 3, 0, "bf16"),
+    # planes too large for one SM: the row-band path, LL planes in the array too
+    Workload("band_path_L2", 1, 2, 192, 192, 5, 2, "f32"),
 ]
 
 
