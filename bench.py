@@ -150,6 +150,24 @@ def max_over_ranks(value, world, device):
     return float(t.item())
 
 
+def rank_inputs(wl, rank):
+    """Inputs of one data-parallel rank: the parameters are the same on every
+    rank (seed 0), the activations X and dY are this rank's own batch
+    (seed = rank; rank 0 sees exactly the seed-0 workload)."""
+    inp = make_inputs(wl, seed=0)
+    if rank:
+        mine = make_inputs(wl, seed=rank)
+        inp["X"], inp["dY"] = mine["X"], mine["dY"]
+    return inp
+
+
+def allreduce_grads(flat, world):
+    """Sums the parameter gradients over the ranks (the layer is a sum over
+    the batch, so the sum of per-rank gradients is the global-batch one)."""
+    if world > 1:
+        dist.all_reduce(flat)
+
+
 def grads_flat_views(wl, device):
     """One flat fp32 buffer with views for every parameter gradient (so the
     data-parallel all-reduce is a single collective)."""
@@ -171,7 +189,7 @@ def run_ours(args, wl, world, rank, local):
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
     dt = torch.float32 if wl.io == "f32" else torch.bfloat16
-    inp = make_inputs(wl, seed=rank)
+    inp = rank_inputs(wl, rank)
     X = inp["X"].to(dt).to(device)
     dY = inp["dY"].to(dt).to(device)
     p = {k: inp[k].to(device) for k in ("W0", "b0", "s0")}
@@ -197,8 +215,7 @@ def run_ours(args, wl, world, rank, local):
         wt.backward_weight(x, dy, p["W0"], p["b0"], p["s0"], Wl, sl, grads=grads, ws=ws, stream=stream)
         if ev is not None:
             ev[3].record(stream)
-        if world > 1:
-            dist.all_reduce(gflat)
+        allreduce_grads(gflat, world)
         if ev is not None:
             ev[4].record(stream)
 
