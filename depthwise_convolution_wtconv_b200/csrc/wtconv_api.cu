@@ -246,32 +246,46 @@ void build_bwdw_plan(Plan& P, const wtconv_desc* d, int max_smem) {
 }
 
 // ------------------------------------------------ pipelined output kernel
+constexpr int SM_SMEM = 233472;  // shared memory per SM on sm_100a (228 KB)
+
+// Floats of one channel's folded weights: base and (L >= 1) four level-1
+// kernels (kk4 floats each) and the bias.
 int main_wblk(const wtconv_desc* d) { return rup((d->L >= 1 ? 5 : 1) * rup(d->k * d->k, 4) + 4, 4); }
+
+// Output tile rows for band height TH: 8, unless 4 wastes fewer padded rows.
+int main_r3(int TH) { return rup(TH, 8) == rup(TH, 4) ? 8 : 4; }
 
 // Slot layout for band height TH and PB planes per unit; returns the slot
 // size in floats.
 int main_slot(MainPlan& M, int TH, int PB) {
-  const int r = M.r, RB = M.R3 / 2;
+  const int r = M.r, R3 = main_r3(TH), TH1 = TH / 2;
   const int hx = M.L >= 1 ? 2 * r : r;
   int cur = 0;
-  // region written by the producer's bulk copies and read by the stagers
+  // raw region: written by the bulk copies of the next unit
   M.wraw_off = cur;
   cur += M.wblk;
   M.raw_off = cur;
   M.raw_pp = rup((int)(((size_t)std::min(M.H, TH + 2 * hx) * M.W * M.io_bytes + 3) / 4), 4);
   cur += PB * M.raw_pp;
   M.rawt_off = cur;
-  M.rawt_pp = (M.L >= 2 && M.bulk_t) ? rup((TH / 2) * M.W1, 4) : 0;
+  M.rawt_pp = (M.L >= 2 && M.bulk_t) ? rup(TH1 * M.W1, 4) : 0;
   cur += PB * M.rawt_pp;
-  // region written by the stagers and read by the consumers
+  // the current unit's staged data, read by the register tiles
   M.w_off = cur;
   cur += M.wblk;
   int pcur = 0;  // per-plane buffers, PB copies each
-  M.xf = make_shifted(pcur, TH, M.W, r, {{M.R3, C3_CW}}, 1);
-  if (M.L >= 1) M.s1 = make_shifted(pcur, TH / 2, M.W1, r, {{RB, 4}}, 4);
-  if (M.L >= 2) M.t1 = make_plain(pcur, TH / 2, M.W1, {{RB, 4}, {1, 4}}, 1);
+  M.xf = make_shifted(pcur, TH, M.W, r, {{R3, 4}}, 1);
+  M.s1 = BufDesc{0, 0, 0, 0};
+  M.t1 = BufDesc{0, 0, 0, 0};
+  M.zb = BufDesc{0, 0, 0, 0};
+  if (M.L >= 1) {
+    M.s1 = make_shifted(pcur, TH1, M.W1, r, {{4, 4}}, 4);
+    const int zrows = std::max(rup(TH1, 4), rup(TH, R3) / 2);
+    M.zb = make_plain(pcur, zrows, M.W1, {{4, 4}}, 4);
+  }
+  if (M.L >= 2) M.t1 = make_plain(pcur, TH1, M.W1, {{4, 4}}, 1);
   const int pstride = rup(pcur, 4);
-  for (BufDesc* bd : {&M.xf, &M.s1, &M.t1}) {
+  for (BufDesc* bd : {&M.xf, &M.s1, &M.t1, &M.zb}) {
     bd->off += cur;
     bd->ps = pstride;
   }
@@ -287,30 +301,29 @@ bool build_main_plan(MainPlan& M, const wtconv_desc* d, int max_smem) {
   M.kk4 = rup(d->k * d->k, 4);
   M.io_bytes = io_bytes(d);
   M.vec_in = (d->W % 4) == 0;
-  M.vec_out = d->io == WTCONV_BF16 ? (d->W % 8) == 0 : (d->W % 4) == 0;
-  M.R3 = d->H >= 8 ? 4 : 2;
+  M.vec_out = (d->W % 4) == 0;
   M.wblk = main_wblk(d);
   M.bulk_t = d->L >= 2 && (M.W1 % 4) == 0;
-  const int tx = cdiv_h(d->W, C3_CW);
-  // Largest band height (H itself, else an even divisor of H) whose slots fit
-  // in half of an SM's shared memory (two CTAs per SM).  Without bands, small
-  // planes are batched so that a unit has about one tile per consumer
-  // thread; then as many slots (2..4) as fit.
-  const size_t budget = (size_t)max_smem / 2;
-  int TH = -1, PB = 1, NS = 0;
-  for (int cand = d->H; cand >= 2 && TH < 0; --cand) {
-    if (d->H % cand || (cand != d->H && (cand & 1))) continue;
-    const int tpp = cdiv_h(cand, M.R3) * tx;
-    int pb = cand == d->H ? std::max(1, std::min(d->N, MAIN_CONSUMERS / tpp)) : 1;
-    for (; pb >= 1 && TH < 0; --pb) {
-      MainPlan T = M;
-      const int slot = main_slot(T, cand, pb);
-      for (int ns = MAIN_MAXSLOTS; ns >= 2; --ns) {
-        if ((size_t)(MAIN_HEADER + ns * slot) * 4 <= budget) {
+  const int tx = cdiv_h(d->W, 4);
+  // Whole planes when at least three CTAs fit per SM (no halo rows staged
+  // twice); else the most CTAs per SM (four, then three, two, one) with the
+  // largest band height (an even divisor of H) whose slot fits that share of
+  // the SM's shared memory.  Without bands, small planes are batched so that
+  // a unit has about one tile per thread.
+  int TH = -1, PB = 1;
+  for (int pass = 0; pass < 2 && TH < 0; ++pass)
+  for (int occ = 4; occ >= (pass == 0 ? 3 : 1) && TH < 0; --occ) {
+    const size_t budget = std::min((size_t)max_smem, (size_t)SM_SMEM / occ - 1024);
+    for (int cand = d->H; cand >= (pass == 0 ? d->H : 2) && TH < 0; --cand) {
+      if (d->H % cand || (cand != d->H && (cand & 1))) continue;
+      const int tpp = cdiv_h(cand, main_r3(cand)) * tx;
+      int pb = cand == d->H ? std::max(1, std::min(d->N, MAIN_NT / tpp)) : 1;
+      for (; pb >= 1 && TH < 0; --pb) {
+        MainPlan T = M;
+        const int slot = main_slot(T, cand, pb);
+        if ((size_t)(MAIN_HEADER + slot) * 4 <= budget) {
           TH = cand;
           PB = pb;
-          NS = ns;
-          break;
         }
       }
     }
@@ -318,12 +331,12 @@ bool build_main_plan(MainPlan& M, const wtconv_desc* d, int max_smem) {
   if (TH < 0) return false;
   M.TH = TH;
   M.PB = PB;
-  M.nslots = NS;
+  M.R3 = main_r3(TH);
   M.nbands = d->H / TH;
   M.units = d->C * ((d->N + PB - 1) / PB) * M.nbands;
   M.slot_floats = main_slot(M, TH, PB);
   M.slot0 = MAIN_HEADER;
-  M.smem_floats = M.slot0 + NS * M.slot_floats;
+  M.smem_floats = M.slot0 + M.slot_floats;
   const size_t plane_bytes = (size_t)d->H * d->W * M.io_bytes;
   M.bulk_x = M.nbands == 1 ? (plane_bytes % 16 == 0) : (((size_t)d->W * M.io_bytes) % 16 == 0);
   const bool band = M.nbands > 1;
@@ -338,18 +351,11 @@ bool build_main_plan(MainPlan& M, const wtconv_desc* d, int max_smem) {
   M.stage_pp = M.st_rows * M.st_q;
   M.tiles_pp = cdiv_h(TH, M.R3) * tx;
   M.tiles = PB * M.tiles_pp;
-  // consumer warp chunks: a unit of >= 32 tiles splits into ch_n balanced
-  // chunks; smaller units go ch_units whole units (at most nslots) a chunk
-  if (M.tiles >= 32) {
-    M.ch_units = 1;
-    M.ch_n = cdiv_h(M.tiles, 32);
-  } else {
-    M.ch_units = std::min(32 / M.tiles, NS);
-    M.ch_n = 1;
-  }
-  M.ch_base = M.ch_units * M.tiles / M.ch_n;
-  M.ch_rem = M.ch_units * M.tiles % M.ch_n;
-  M.f_chn = make_fdiv(M.ch_n);
+  const int atx = cdiv_h(M.W1, 4), aty = cdiv_h(TH / 2, 4);
+  M.a_pp = d->L >= 1 ? 4 * aty * atx : 0;
+  M.f_app = make_fdiv(std::max(1, M.a_pp));
+  M.f_abt = make_fdiv(aty * atx);
+  M.f_atx = make_fdiv(atx);
   M.f_tiles = make_fdiv(M.tiles);
   M.f_tpp = make_fdiv(M.tiles_pp);
   M.f_tx = make_fdiv(tx);
@@ -501,14 +507,14 @@ wtconv_status launch_forward_t(const wtconv_desc* d, const Device& dev, const vo
   if (!build_main_plan(M, d, dev.max_smem)) return WTCONV_ERR_UNSUPPORTED;
   const size_t smem = (size_t)M.smem_floats * 4;
   int occ = 0;
-  if (M.R3 == 4) {
-    auto km = wtconv_main_kernel<K, 4, IO>;
+  if (M.R3 == 8) {
+    auto km = wtconv_main_kernel<K, 8, IO>;
     wtconv_status e = prepare(km, smem, occ, MAIN_NT);
     if (e != WTCONV_OK) return e;
     km<<<std::min(M.units, dev.sms * occ), MAIN_NT, smem, st>>>(M, static_cast<const IO*>(x), t1, wfold,
                                                                 static_cast<IO*>(y), status);
   } else {
-    auto km = wtconv_main_kernel<K, 2, IO>;
+    auto km = wtconv_main_kernel<K, 4, IO>;
     wtconv_status e = prepare(km, smem, occ, MAIN_NT);
     if (e != WTCONV_OK) return e;
     km<<<std::min(M.units, dev.sms * occ), MAIN_NT, smem, st>>>(M, static_cast<const IO*>(x), t1, wfold,

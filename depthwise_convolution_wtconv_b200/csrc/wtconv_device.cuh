@@ -86,6 +86,31 @@ __device__ __forceinline__ void store8(__nv_bfloat16* __restrict__ p, const floa
     if (e < n) p[e] = __float2bfloat16_rn(v[e]);
 }
 
+// Stores n (<= 4) consecutive values of one output row.  `vec` says the row
+// start p is aligned for the 4-element vector form (16 bytes for fp32, 8 for
+// bf16).
+__device__ __forceinline__ void store4(float* __restrict__ p, const float (&v)[4], int n, bool vec) {
+  if (vec && n == 4) {
+    *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+    return;
+  }
+#pragma unroll
+  for (int e = 0; e < 4; ++e)
+    if (e < n) p[e] = v[e];
+}
+__device__ __forceinline__ void store4(__nv_bfloat16* __restrict__ p, const float (&v)[4], int n, bool vec) {
+  if (vec && n == 4) {
+    uint2 t;
+    t.x = pack_bf16x2(v[0], v[1]);
+    t.y = pack_bf16x2(v[2], v[3]);
+    *reinterpret_cast<uint2*>(p) = t;
+    return;
+  }
+#pragma unroll
+  for (int e = 0; e < 4; ++e)
+    if (e < n) p[e] = __float2bfloat16_rn(v[e]);
+}
+
 // ------------------------------------------------------ register-tiled conv
 // acc[R][CW] += sum_{u,v<K} w[u*K+v] * in[(orow+u)*ld + (j+v)]
 // `in` points at the input element (y0-r, x0-r) of the tile and must be

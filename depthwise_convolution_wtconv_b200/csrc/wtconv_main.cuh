@@ -1,23 +1,20 @@
-// Warp-specialised output kernel and deep-level kernel (sm_100a).
+// Output kernel and deep-level kernel (sm_100a).
 //
-// Output kernel (forward and backward-data): one producer warp issues TMA
-// 1-D bulk copies (cp.async.bulk) of each unit's input rows and t1 rows into
-// a ring of two to four slots; three stager warps copy the channel's folded
-// weights and turn the raw rows into the zero-padded fp32 rows and the
-// level-1 Haar subbands (reformulation (1) of arXiv:2608.10805, abstract);
-// four consumer warps run register tiles back to back across units: the four level-1 band convs with
-// folded weights (reformulation (3)), t1 added to the LL band, the synthesis
-// signs, then the base conv, and store y.  Slots are handed over with
-// mbarriers (full / raw free / staged / empty) and a per-slot ready counter;
-// there is no CTA-wide barrier after set-up, so consumer lanes only idle at
-// the very end of the grid.
-//
-// Why a counter for "ready": a parity wait (mbarrier.try_wait.parity) reports
-// the phase before the current one as complete.  A consumer thread that has
-// no tile in a unit skips that unit's wait and can come to a slot's next use
-// while the slot's barrier is still one phase behind; a parity wait would
-// then pass at once.  Producer and stagers wait on every phase in order, so
-// their parity waits are safe; consumers wait on the monotonic counter.
+// Output kernel (forward and backward-data): a CTA of four warps works
+// through its units (a band of one plane, or a batch of small planes of one
+// channel) in phases.  Thread 0 keeps the next unit's input rows, t1 rows
+// and folded weights in flight with TMA 1-D bulk copies (cp.async.bulk,
+// completing on one mbarrier) while the CTA computes the current unit; the
+// CTA turns the raw rows into zero-padded fp32 rows and the level-1 Haar
+// subbands (reformulation (1) of arXiv:2608.10805, abstract), then runs
+// register tiles in two phases: (A) each thread convolves one level-1 band
+// over a 4x4 tile with folded weights (reformulation (3)), adds t1 to the LL
+// band and writes the band's Z plane to shared memory; (B) each thread takes
+// an R3 x 4 output tile, adds the synthesis of the four Z planes, runs the
+// base conv and stores y.  Tiles four floats wide let the lanes of a warp
+// read consecutive 16-byte words of a row, nearly free of bank conflicts.
+// Small CTAs (about 64 KB of shared memory on 56x56 planes) let three run
+// per SM, so one CTA's staging and barriers overlap the others' arithmetic.
 //
 // Deep kernel: levels 2..L of a batch of planes on chip (pyramid, every level
 // conv, then the closed-form synthesis of all levels >= 2 at level-1
@@ -28,11 +25,8 @@
 
 namespace wt {
 
-constexpr int MAIN_CONSUMERS = 128;  // warps 4-7
-constexpr int MAIN_STAGERS = 96;     // warps 1-3
-constexpr int MAIN_NT = 32 + MAIN_STAGERS + MAIN_CONSUMERS;
-constexpr int MAIN_MAXSLOTS = 4;
-constexpr int MAIN_HEADER = 48;      // floats: 16 mbarriers, abort flag, ready counters
+constexpr int MAIN_NT = 128;
+constexpr int MAIN_HEADER = 4;       // floats: mbarrier (8 bytes), abort flag
 constexpr int DEEP_NT = 128;
 
 // ------------------------------------------------------------ mbarriers
@@ -69,28 +63,6 @@ __device__ __forceinline__ void mb_drain(uint64_t* b, unsigned parity) {
   for (int i = 0; i < (1 << 22); ++i)
     if (mb_try(b, parity)) return;
 }
-__device__ __forceinline__ void st_release(int* p, int v) {
-  asm volatile("st.release.cta.shared::cta.u32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
-}
-__device__ __forceinline__ int ld_acquire(const int* p) {
-  int v;
-  asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)) : "memory");
-  return v;
-}
-// Waits until *seq >= want (bounded; abort-aware like mb_wait), backing off
-// between polls so that a waiting warp leaves its issue slots to others.
-__device__ __forceinline__ bool seq_wait(const int* seq, int want, volatile int* abort_flag) {
-  unsigned ns = 32;
-  for (int i = 0; i < (1 << 22); ++i) {
-    if (ld_acquire(seq) >= want) return true;
-    if (*abort_flag) return false;
-    __nanosleep(ns);
-    if (ns < 512) ns <<= 1;
-  }
-  *abort_flag = 1;
-  return false;
-}
-
 // ------------------------------------------------------------ unit geometry
 // A unit is one band of one plane (nbands > 1) or a batch of npb planes of
 // one channel (nbands == 1, consecutive batch entries).
@@ -208,233 +180,202 @@ __device__ __forceinline__ void main_stage_item(const MainPlan& P, float* xf, fl
   }
 }
 
-// One output tile of plane j of a unit: (R3/2) x 4 band convs for the four
-// level-1 bands, t1 on LL, synthesis signs, base conv, store.
+// Phase A, one tile: band s of plane j, a 4x4 tile of the level-1 grid:
+// the band conv with folded weights (reformulation (3) of arXiv:2608.10805,
+// abstract), t1 added to the LL band, stored to the band's Z plane.
+template <int K>
+__device__ __forceinline__ void main_band_tile(const MainPlan& P, float* slot, int it) {
+  const int j = P.f_app.div(it);
+  int rem = it - j * P.a_pp;
+  const int s = P.f_abt.div(rem);
+  rem -= s * P.f_abt.d;
+  const int ti = P.f_atx.div(rem);
+  const int i0 = ti * 4, j0 = (rem - ti * P.f_atx.d) * 4;
+  float z[4][4];
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int b = 0; b < 4; ++b) z[a][b] = 0.f;
+  const float* s1 = slot + P.s1.off + j * P.s1.ps + s * P.s1.ld * P.s1.rows + i0 * P.s1.ld + j0;
+  conv_tile<K, 4, 4>(s1, P.s1.ld, slot + P.w_off + P.kk4 + 4 + s * P.kk4, z);
+  if (s == 0 && P.L >= 2) {
+    const float* t1 = slot + P.t1.off + j * P.t1.ps + i0 * P.t1.ld + j0;
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+      const float4 tv = *reinterpret_cast<const float4*>(t1 + a * P.t1.ld);
+      z[a][0] += tv.x;
+      z[a][1] += tv.y;
+      z[a][2] += tv.z;
+      z[a][3] += tv.w;
+    }
+  }
+  float* zp = slot + P.zb.off + j * P.zb.ps + s * P.zb.ld * P.zb.rows + i0 * P.zb.ld + j0;
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+    *reinterpret_cast<float4*>(zp + a * P.zb.ld) = make_float4(z[a][0], z[a][1], z[a][2], z[a][3]);
+}
+
+// Phase B, one tile: R3 x 4 outputs of plane j: bias, the level-1 synthesis
+// of the four Z planes (signs sigma_s(py, px); the 1/2 is in the weights),
+// the base conv, and the store.
 template <int K, int R3, typename IO>
-__device__ __forceinline__ void main_tile(const MainPlan& P, const float* slot, const UnitGeo& g, int j, int tile,
-                                          IO* __restrict__ y) {
-  constexpr int RB = R3 / 2;
+__device__ __forceinline__ void main_out_tile(const MainPlan& P, const float* slot, const UnitGeo& g, int j, int tile,
+                                              IO* __restrict__ y) {
   const int ti = P.f_tx.div(tile);
-  const int tj = tile - ti * P.f_tx.d;
-  const int yy0 = ti * R3, xx0 = tj * C3_CW;
+  const int yy0 = ti * R3, xx0 = (tile - ti * P.f_tx.d) * 4;
   const float* sw = slot + P.w_off;
   const float bias = sw[P.kk4];
-  float acc[R3][C3_CW];
+  float acc[R3][4];
 #pragma unroll
   for (int a = 0; a < R3; ++a)
 #pragma unroll
-    for (int b = 0; b < C3_CW; ++b) acc[a][b] = bias;
+    for (int b = 0; b < 4; ++b) acc[a][b] = bias;
   if (P.L >= 1) {
-    const int bs1 = P.s1.ld * P.s1.rows;
-    const float* s1 = slot + P.s1.off + j * P.s1.ps + (yy0 >> 1) * P.s1.ld + (xx0 >> 1);
+    const int bz = P.zb.ld * P.zb.rows;
+    const float* zb = slot + P.zb.off + j * P.zb.ps + (yy0 >> 1) * P.zb.ld + (xx0 >> 1);
 #pragma unroll
-    for (int s = 0; s < 4; ++s) {
-      float z[RB][4];
+    for (int a = 0; a < R3 / 2; ++a) {
+      float2 zs[4];
 #pragma unroll
-      for (int a = 0; a < RB; ++a)
-#pragma unroll
-        for (int b = 0; b < 4; ++b) z[a][b] = 0.f;
-      conv_tile<K, RB, 4>(s1 + s * bs1, P.s1.ld, sw + P.kk4 + 4 + s * P.kk4, z);
-      if (s == 0 && P.L >= 2) {
-        const float* t1 = slot + P.t1.off + j * P.t1.ps + (yy0 >> 1) * P.t1.ld + (xx0 >> 1);
-#pragma unroll
-        for (int a = 0; a < RB; ++a) {
-          const float4 tv = reinterpret_cast<const float4*>(t1 + a * P.t1.ld)[0];
-          z[a][0] += tv.x;
-          z[a][1] += tv.y;
-          z[a][2] += tv.z;
-          z[a][3] += tv.w;
-        }
-      }
-      // sigma_s(py, px): LL +,+,+,+  LH +,+,-,-  HL +,-,+,-  HH +,-,-,+
-      const float s01 = (s == 2 || s == 3) ? -1.f : 1.f;
-      const float s10 = (s == 1 || s == 3) ? -1.f : 1.f;
-      const float s11 = (s == 1 || s == 2) ? -1.f : 1.f;
-#pragma unroll
-      for (int a = 0; a < RB; ++a)
-#pragma unroll
-        for (int b = 0; b < 4; ++b) {
-          const float v = z[a][b];
-          acc[2 * a][2 * b] += v;
-          acc[2 * a][2 * b + 1] = fmaf(s01, v, acc[2 * a][2 * b + 1]);
-          acc[2 * a + 1][2 * b] = fmaf(s10, v, acc[2 * a + 1][2 * b]);
-          acc[2 * a + 1][2 * b + 1] = fmaf(s11, v, acc[2 * a + 1][2 * b + 1]);
-        }
+      for (int s = 0; s < 4; ++s) zs[s] = *reinterpret_cast<const float2*>(zb + s * bz + a * P.zb.ld);
+      float o00, o01, o10, o11;
+      synth4(zs[0].x, zs[1].x, zs[2].x, zs[3].x, o00, o01, o10, o11);
+      acc[2 * a][0] += o00;
+      acc[2 * a][1] += o01;
+      acc[2 * a + 1][0] += o10;
+      acc[2 * a + 1][1] += o11;
+      synth4(zs[0].y, zs[1].y, zs[2].y, zs[3].y, o00, o01, o10, o11);
+      acc[2 * a][2] += o00;
+      acc[2 * a][3] += o01;
+      acc[2 * a + 1][2] += o10;
+      acc[2 * a + 1][3] += o11;
     }
   }
-  conv_tile<K, R3, C3_CW>(slot + P.xf.off + j * P.xf.ps + yy0 * P.xf.ld + xx0, P.xf.ld, sw, acc);
-  const int n = P.W - xx0 < C3_CW ? P.W - xx0 : C3_CW;
+  conv_tile<K, R3, 4>(slot + P.xf.off + j * P.xf.ps + yy0 * P.xf.ld + xx0, P.xf.ld, sw, acc);
+  const int n = P.W - xx0 < 4 ? P.W - xx0 : 4;
   IO* yp = y + plane_index(P, g, j) * P.H * P.W;
 #pragma unroll
   for (int a = 0; a < R3; ++a) {
     const int yr = g.y0 + yy0 + a;
-    if (yy0 + a < P.TH && yr < P.H) store8(yp + (size_t)yr * P.W + xx0, acc[a], n, P.vec_out != 0);
+    if (yy0 + a < P.TH && yr < P.H) store4(yp + (size_t)yr * P.W + xx0, acc[a], n, P.vec_out != 0);
+  }
+}
+
+// One unit's bulk copies into the raw region of the slot: the channel's
+// folded weights, the unit's input rows (bulk_x) and t1 rows (bulk_t), all
+// completing on one mbarrier phase.
+template <typename IO>
+__device__ __forceinline__ void main_issue(const MainPlan& P, float* slot, uint64_t* full, const UnitGeo& g,
+                                           const IO* __restrict__ x, const float* __restrict__ t1g,
+                                           const float* __restrict__ wfold) {
+  const unsigned bx = P.bulk_x ? (unsigned)((g.y_hi - g.y_lo) * P.W * P.io_bytes) : 0u;
+  const unsigned bt = (P.L >= 2 && P.bulk_t) ? (unsigned)((P.TH >> 1) * P.W1 * 4) : 0u;
+  const unsigned bw = (unsigned)(P.wblk * 4);
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(full)),
+               "r"(bw + (bx + bt) * g.npb)
+               : "memory");
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(slot + P.wraw_off)),
+      "l"(wfold + (size_t)g.c * P.wblk), "r"(bw), "r"(smem_u32(full))
+      : "memory");
+  for (int j = 0; j < g.npb; ++j) {
+    const size_t pi = plane_index(P, g, j);
+    if (bx) {
+      const IO* src = x + pi * P.H * P.W + (size_t)g.y_lo * P.W;
+      asm volatile(
+          "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+              smem_u32(slot + P.raw_off + j * P.raw_pp)),
+          "l"(src), "r"(bx), "r"(smem_u32(full))
+          : "memory");
+    }
+    if (bt) {
+      const float* src = t1g + pi * P.H1 * P.W1 + (size_t)(g.y0 >> 1) * P.W1;
+      asm volatile(
+          "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+              smem_u32(slot + P.rawt_off + j * P.rawt_pp)),
+          "l"(src), "r"(bt), "r"(smem_u32(full))
+          : "memory");
+    }
   }
 }
 
 template <int K, int R3, typename IO>
-__global__ void __launch_bounds__(MAIN_NT, 2)
+__global__ void __launch_bounds__(MAIN_NT, 4)
     wtconv_main_kernel(const MainPlan P, const IO* __restrict__ x, const float* __restrict__ t1g,
                        const float* __restrict__ wfold, IO* __restrict__ y, int* __restrict__ status) {
   extern __shared__ float4 smem4[];
   float* sm = reinterpret_cast<float*>(smem4);
   uint64_t* full = reinterpret_cast<uint64_t*>(sm);
-  uint64_t* rawfree = full + MAIN_MAXSLOTS;
-  uint64_t* staged = full + 2 * MAIN_MAXSLOTS;  // all stagers done with a use of the slot
-  uint64_t* empty = full + 3 * MAIN_MAXSLOTS;
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + 32);
-  int* ready_seq = reinterpret_cast<int*>(sm + 36);  // slot s holds uses < ready_seq[s]
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + 2);
   const int tid = threadIdx.x;
-  for (int i = tid + MAIN_HEADER / 4; i < (P.smem_floats >> 2); i += MAIN_NT)
-    smem4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int i = tid; i < (P.smem_floats >> 2); i += MAIN_NT) smem4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  __syncthreads();
   if (tid == 0) {
-    for (int i = 0; i < MAIN_HEADER / 4; ++i) smem4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int s = 0; s < P.nslots; ++s) {
-      mb_init(full + s, 1);
-      mb_init(rawfree + s, MAIN_STAGERS);
-      mb_init(staged + s, MAIN_STAGERS);
-      mb_init(empty + s, P.tiles);
-    }
+    mb_init(full, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
   const int myunits = (int)blockIdx.x < P.units ? (P.units - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
-  const int warp = tid >> 5;
-  const int NS = P.nslots;
-
-  if (warp == 0) {
-    // ---------------------------------------------------------- producer
-    if (tid != 0) return;
-    int k = 0;
-    for (; k < myunits; ++k) {
-      const int u = blockIdx.x + k * gridDim.x, s = k % NS, use = k / NS;
-      if (use >= 1 && !mb_wait(rawfree + s, (use - 1) & 1, abort_flag)) break;
-      const UnitGeo g = unit_geo(P, u);
-      float* slot = sm + P.slot0 + s * P.slot_floats;
-      const unsigned bx = P.bulk_x ? (unsigned)((g.y_hi - g.y_lo) * P.W * P.io_bytes) : 0u;
-      const unsigned bt = (P.L >= 2 && P.bulk_t) ? (unsigned)((P.TH >> 1) * P.W1 * 4) : 0u;
-      const unsigned bw = (unsigned)(P.wblk * 4);
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(full + s)),
-                   "r"(bw + (bx + bt) * g.npb)
-                   : "memory");
-      asm volatile(
-          "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-              smem_u32(slot + P.wraw_off)),
-          "l"(wfold + (size_t)g.c * P.wblk), "r"(bw), "r"(smem_u32(full + s))
-          : "memory");
-      for (int j = 0; j < g.npb; ++j) {
-        const size_t pi = plane_index(P, g, j);
-        if (bx) {
-          const IO* src = x + pi * P.H * P.W + (size_t)g.y_lo * P.W;
-          asm volatile(
-              "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                  smem_u32(slot + P.raw_off + j * P.raw_pp)),
-              "l"(src), "r"(bx), "r"(smem_u32(full + s))
-              : "memory");
+  float* slot = sm + P.slot0;
+  if (tid == 0 && myunits > 0) main_issue<IO>(P, slot, full, unit_geo(P, blockIdx.x), x, t1g, wfold);
+  int k = 0;
+  for (; k < myunits; ++k) {
+    const UnitGeo g = unit_geo(P, blockIdx.x + k * gridDim.x);
+    // every thread waits on every phase in order, so a parity wait is exact
+    mb_wait(full, k & 1, abort_flag);
+    const int n = g.npb * P.stage_pp;
+    for (int it = tid; it < n; it += MAIN_NT) {
+      const int j = P.f_spp.div(it);
+      const int rem = it - j * P.stage_pp;
+      const int ri = P.f_stq.div(rem);
+      const int x0 = (rem - ri * P.st_q) << 2;
+      float* xf = slot + P.xf.off + j * P.xf.ps;
+      float* s1 = slot + P.s1.off + j * P.s1.ps;
+      if (P.bulk_x)
+        main_stage_item<K, IO, true>(P, xf, s1, reinterpret_cast<const IO*>(slot + P.raw_off + j * P.raw_pp), g, ri,
+                                     x0);
+      else
+        main_stage_item<K, IO, false>(P, xf, s1, x + plane_index(P, g, j) * P.H * P.W, g, ri, x0);
+    }
+    // folded weights and t1 rows leave the raw region, which the next
+    // unit's copies overwrite while this unit computes
+    for (int i = tid; i < (P.wblk >> 2); i += MAIN_NT)
+      reinterpret_cast<float4*>(slot + P.w_off)[i] = reinterpret_cast<const float4*>(slot + P.wraw_off)[i];
+    if (P.L >= 2) {
+      const int rows = P.TH >> 1, q4 = (P.W1 + 3) >> 2;
+      for (int it = tid; it < g.npb * rows * q4; it += MAIN_NT) {
+        const int j = it / (rows * q4), rem = it - j * rows * q4;
+        const int rr = rem / q4, x0 = (rem - rr * q4) << 2;
+        float4 v;
+        if (P.bulk_t) {
+          v = *reinterpret_cast<const float4*>(slot + P.rawt_off + j * P.rawt_pp + rr * P.W1 + x0);
+        } else {
+          const float* q = t1g + plane_index(P, g, j) * P.H1 * P.W1 + (size_t)((g.y0 >> 1) + rr) * P.W1 + x0;
+          v = load4(q, x0, P.W1, (P.W1 & 3) == 0);
         }
-        if (bt) {
-          const float* src = t1g + pi * P.H1 * P.W1 + (size_t)(g.y0 >> 1) * P.W1;
-          asm volatile(
-              "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                  smem_u32(slot + P.rawt_off + j * P.rawt_pp)),
-              "l"(src), "r"(bt), "r"(smem_u32(full + s))
-              : "memory");
-        }
+        *reinterpret_cast<float4*>(slot + P.t1.off + j * P.t1.ps + rr * P.t1.ld + x0) = v;
       }
     }
-    // the copies already issued must land before this CTA can exit
-    for (int j = (k > NS ? k - NS : 0); j < k; ++j) mb_drain(full + (j % NS), (j / NS) & 1);
-    if (*abort_flag && status) atomicExch(status, 1);
-    return;
+    __syncthreads();
+    if (*abort_flag) break;  // uniform: read after the barrier
+    if (tid == 0 && k + 1 < myunits)
+      main_issue<IO>(P, slot, full, unit_geo(P, blockIdx.x + (k + 1) * gridDim.x), x, t1g, wfold);
+    if (P.L >= 1) {
+      const int na = g.npb * P.a_pp;
+      for (int it = tid; it < na; it += MAIN_NT) main_band_tile<K>(P, slot, it);
+      __syncthreads();
+    }
+    for (int it = tid; it < P.tiles; it += MAIN_NT) {
+      const int j = P.f_tpp.div(it);
+      if (j < g.npb) main_out_tile<K, R3, IO>(P, slot, g, j, it - j * P.tiles_pp, y);
+    }
+    __syncthreads();
   }
-
-  if (warp <= MAIN_STAGERS / 32) {
-    // ---------------------------------------------------------- stagers
-    const int t = tid - 32;
-    for (int k = 0; k < myunits; ++k) {
-      const int u = blockIdx.x + k * gridDim.x, s = k % NS, use = k / NS;
-      if (!mb_wait(full + s, use & 1, abort_flag)) break;
-      if (use >= 1 && !mb_wait(empty + s, (use - 1) & 1, abort_flag)) break;
-      const UnitGeo g = unit_geo(P, u);
-      float* slot = sm + P.slot0 + s * P.slot_floats;
-      const int n = g.npb * P.stage_pp;
-      for (int it = t; it < n; it += MAIN_STAGERS) {
-        const int j = P.f_spp.div(it);
-        const int rem = it - j * P.stage_pp;
-        const int ri = P.f_stq.div(rem);
-        const int x0 = (rem - ri * P.st_q) << 2;
-        float* xf = slot + P.xf.off + j * P.xf.ps;
-        float* s1 = slot + P.s1.off + j * P.s1.ps;
-        if (P.bulk_x)
-          main_stage_item<K, IO, true>(P, xf, s1, reinterpret_cast<const IO*>(slot + P.raw_off + j * P.raw_pp), g,
-                                       ri, x0);
-        else
-          main_stage_item<K, IO, false>(P, xf, s1, x + plane_index(P, g, j) * P.H * P.W, g, ri, x0);
-      }
-      // folded weights and t1 rows move to the consumer side of the slot
-      for (int i = t; i < (P.wblk >> 2); i += MAIN_STAGERS)
-        reinterpret_cast<float4*>(slot + P.w_off)[i] = reinterpret_cast<const float4*>(slot + P.wraw_off)[i];
-      if (P.L >= 2) {
-        const int rows = P.TH >> 1, q4 = (P.W1 + 3) >> 2;
-        for (int it = t; it < g.npb * rows * q4; it += MAIN_STAGERS) {
-          const int j = it / (rows * q4), rem = it - j * rows * q4;
-          const int rr = rem / q4, x0 = (rem - rr * q4) << 2;
-          float4 v;
-          if (P.bulk_t) {
-            v = *reinterpret_cast<const float4*>(slot + P.rawt_off + j * P.rawt_pp + rr * P.W1 + x0);
-          } else {
-            const float* q = t1g + plane_index(P, g, j) * P.H1 * P.W1 + (size_t)((g.y0 >> 1) + rr) * P.W1 + x0;
-            v = load4(q, x0, P.W1, (P.W1 & 3) == 0);
-          }
-          *reinterpret_cast<float4*>(slot + P.t1.off + j * P.t1.ps + rr * P.t1.ld + x0) = v;
-        }
-      }
-      mb_arrive(rawfree + s);
-      mb_arrive(staged + s);
-      // stager 0 publishes the slot once every stager is done (in-order wait)
-      if (t == 0) {
-        if (!mb_wait(staged + s, use & 1, abort_flag)) break;
-        st_release(ready_seq + s, use + 1);
-      }
-    }
-    return;
-  }
-
-  // ------------------------------------------------------------ consumers
-  // Warp-sized chunks that never straddle two units: a unit of >= 32 tiles
-  // is split into ch_n chunks of near-equal size; smaller units are grouped,
-  // ch_units whole units (at most nslots) per chunk.  Lane 0 waits for the
-  // newest unit of its chunk (units are published in order), the warp syncs,
-  // and every lane then works without spinning.  A chunk holds back only the
-  // slots of its own units, so the stagers refill a slot as soon as that
-  // unit's tiles are done.
-  const int cw = warp - 1 - MAIN_STAGERS / 32, lane = tid & 31;
-  const int total = cdiv(myunits, P.ch_units) * P.ch_n;
-  for (int g = cw; g < total; g += MAIN_CONSUMERS / 32) {
-    const int grp = P.f_chn.div(g);
-    const int jc = g - grp * P.ch_n;
-    const int k0 = grp * P.ch_units;
-    const int kmax = min(k0 + P.ch_units, myunits) - 1;
-    int ok = 1;
-    if (lane == 0) ok = seq_wait(ready_seq + kmax % NS, kmax / NS + 1, abort_flag);
-    ok = __shfl_sync(0xffffffffu, ok, 0);
-    if (!ok) break;
-    const int size = P.ch_base + (jc < P.ch_rem);
-    const int gi = jc * P.ch_base + min(jc, P.ch_rem) + lane;
-    if (lane < size) {
-      const int kk = P.f_tiles.div(gi);
-      const int k = k0 + kk;
-      if (k <= kmax) {
-        const int tile = gi - kk * P.tiles;
-        const int s = k % NS;
-        (void)ld_acquire(ready_seq + s);  // this lane's own acquire of the published slot
-        const UnitGeo u = unit_geo(P, blockIdx.x + k * gridDim.x);
-        const int j = P.f_tpp.div(tile);
-        if (j < u.npb) main_tile<K, R3, IO>(P, sm + P.slot0 + s * P.slot_floats, u, j, tile - j * P.tiles_pp, y);
-        mb_arrive(empty + s);
-      }
-    }
+  if (*abort_flag && tid == 0) {
+    mb_drain(full, k & 1);  // the copies of unit k were issued; let them land before exit
+    if (status) atomicExch(status, 1);
   }
 }
 

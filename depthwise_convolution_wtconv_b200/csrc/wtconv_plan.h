@@ -102,29 +102,28 @@ struct Plan {
 
 namespace wt {
 
-// Plan of the warp-specialised output kernel (forward and backward-data).
-// A unit is one band of TH output rows of one (n, c) plane (TH = H when the
-// whole plane fits in a slot).  The CTA owns a ring of two slots; each slot
-// holds the raw rows of one unit (TMA bulk copy), its t1 rows, the folded
-// base and level-1 weights of its channel, the padded fp32 rows xf and the
-// padded level-1 subbands s1.  Offsets are floats relative to a slot start.
+// Plan of the output kernel (forward and backward-data).  A unit is one band
+// of TH output rows of one (n, c) plane (TH = H when the whole plane fits),
+// or PB whole planes of one channel.  The CTA's one slot holds a raw region
+// (the next unit's bulk copies: folded weights, input rows, t1 rows) and the
+// current unit's folded weights, padded fp32 rows xf, padded level-1
+// subbands s1 and t1 rows.  Offsets are floats relative to the slot start.
 struct MainPlan {
   int N, C, H, W, K, r, L, H1, W1, kk4, io_bytes;
   int TH, nbands, PB;        // band rows, bands per plane, planes per unit (PB > 1 only without bands)
   int units;                 // C * ceil(N/PB) * nbands
-  int nslots;                // ring slots (2..4)
-  int R3, tiles, tiles_pp;   // output tile rows, tiles per unit, per plane
+  int R3, tiles, tiles_pp;   // output tile rows (8 or 4; tiles are 4 wide), tiles per unit, per plane
   int bulk_x, bulk_t;        // TMA bulk copies usable for x rows / t1 rows
   int vec_in, vec_out;
   int st_row0, st_rows, st_q, stage_pp;  // staged rows per plane (band), items per plane
-  int slot0, slot_floats;    // first slot offset, slot stride
+  int slot0, slot_floats;    // slot offset (after the header) and size
   int wblk;                  // floats of one channel's folded weights
-  int wraw_off, raw_off, rawt_off, raw_pp, rawt_pp;  // producer-written raw copies (per-plane strides)
-  int w_off;                 // stager-written folded weights read by the consumers
-  BufDesc xf, s1, t1;        // per-plane copies at ps stride
-  int ch_units, ch_n;        // consumer-warp chunks: units per chunk, chunks per unit group
-  int ch_base, ch_rem;       // chunk jc of a group holds ch_base + (jc < ch_rem) tiles
-  FDiv f_tiles, f_tpp, f_tx, f_stq, f_spp, f_bands, f_C, f_chn;
+  int wraw_off, raw_off, rawt_off, raw_pp, rawt_pp;  // raw region of the bulk copies (per-plane strides)
+  int w_off;                 // the current unit's folded weights
+  BufDesc xf, s1, t1, zb;    // per-plane copies at ps stride (zb: the four level-1 Z planes)
+  int a_pp;                  // phase-A tiles per plane: 4 bands x ceil(TH/8) x ceil(W1/4)
+  FDiv f_tiles, f_tpp, f_tx, f_stq, f_spp, f_bands, f_C;
+  FDiv f_app, f_abt, f_atx;  // phase-A decomposition: per plane, per band, per tile row
   int smem_floats;
 };
 
