@@ -248,9 +248,9 @@ void build_bwdw_plan(Plan& P, const wtconv_desc* d, int max_smem) {
 // ------------------------------------------------ pipelined output kernel
 constexpr int SM_SMEM = 233472;  // shared memory per SM on sm_100a (228 KB)
 
-// Floats of one channel's folded weights: base and (L >= 1) four level-1
-// kernels (kk4 floats each) and the bias.
-int main_wblk(const wtconv_desc* d) { return rup((d->L >= 1 ? 5 : 1) * rup(d->k * d->k, 4) + 4, 4); }
+// Floats of one channel's folded weights: the base kernel, the bias and
+// four kernels per level (kk4 floats each).
+int main_wblk(const wtconv_desc* d) { return rup((1 + 4 * d->L) * rup(d->k * d->k, 4) + 4, 4); }
 
 // Output tile rows for band height TH: 8, unless 4 wastes fewer padded rows.
 int main_r3(int TH) { return rup(TH, 8) == rup(TH, 4) ? 8 : 4; }
@@ -260,6 +260,8 @@ int main_r3(int TH) { return rup(TH, 8) == rup(TH, 4) ? 8 : 4; }
 int main_slot(MainPlan& M, int TH, int PB) {
   const int r = M.r, R3 = main_r3(TH), TH1 = TH / 2;
   const int hx = M.L >= 1 ? 2 * r : r;
+  M.fused = TH == M.H && M.L >= 2;
+  if (M.fused) M.bulk_t = 0;
   int cur = 0;
   // raw region: written by the bulk copies of the next unit
   M.wraw_off = cur;
@@ -283,12 +285,22 @@ int main_slot(MainPlan& M, int TH, int PB) {
     const int zrows = std::max(rup(TH1, 4), rup(TH, R3) / 2);
     M.zb = make_plain(pcur, zrows, M.W1, {{4, 4}}, 4);
   }
-  if (M.L >= 2) M.t1 = make_plain(pcur, TH1, M.W1, {{4, 4}}, 1);
+  if (M.L >= 2 && !M.fused) M.t1 = make_plain(pcur, TH1, M.W1, {{4, 4}}, 1);
+  for (int l = 0; l <= MAXL; ++l) M.sd[l] = M.zd[l] = BufDesc{0, 0, 0, 0};
+  if (M.fused) {
+    for (int l = 2; l <= M.L; ++l) M.sd[l] = make_shifted(pcur, M.H >> l, M.W >> l, r, {{4, 4}}, 4);
+    for (int l = 2; l <= M.L; ++l) M.zd[l] = make_plain(pcur, M.H >> l, M.W >> l, {{4, 4}}, 4);
+  }
   const int pstride = rup(pcur, 4);
   for (BufDesc* bd : {&M.xf, &M.s1, &M.t1, &M.zb}) {
     bd->off += cur;
     bd->ps = pstride;
   }
+  for (int l = 2; l <= M.L && M.fused; ++l)
+    for (BufDesc* bd : {&M.sd[l], &M.zd[l]}) {
+      bd->off += cur;
+      bd->ps = pstride;
+    }
   cur += PB * pstride;
   return rup(cur, 4);
 }
@@ -356,6 +368,19 @@ bool build_main_plan(MainPlan& M, const wtconv_desc* d, int max_smem) {
   M.f_app = make_fdiv(std::max(1, M.a_pp));
   M.f_abt = make_fdiv(aty * atx);
   M.f_atx = make_fdiv(atx);
+  int first = 0;
+  for (int l = 0; l <= MAXL + 1; ++l) M.dfirst[l] = 0;
+  for (int l = 2; l <= d->L && M.fused; ++l) {
+    const int dtx = cdiv_h(d->W >> l, 4), tiles = cdiv_h(d->H >> l, 4) * dtx;
+    M.f_dtiles[l] = make_fdiv(tiles);
+    M.f_dtx[l] = make_fdiv(dtx);
+    M.dfirst[l] = first;
+    first += 4 * tiles;
+  }
+  if (M.fused) M.dfirst[d->L + 1] = first;
+  M.f_dper = make_fdiv(std::max(1, first));
+  M.f_bpp = make_fdiv(std::max(1, (d->H / 4) * (d->W / 4)));
+  M.f_bx4 = make_fdiv(std::max(1, d->W / 4));
   M.f_tiles = make_fdiv(M.tiles);
   M.f_tpp = make_fdiv(M.tiles_pp);
   M.f_tx = make_fdiv(tx);
@@ -491,7 +516,9 @@ wtconv_status launch_forward_t(const wtconv_desc* d, const Device& dev, const vo
                                                                                    wl, sl, flip, wfold);
     if (cudaGetLastError() != cudaSuccess) return WTCONV_ERR_CUDA;
   }
-  if (d->L >= 2) {
+  MainPlan M;
+  if (!build_main_plan(M, d, dev.max_smem)) return WTCONV_ERR_UNSUPPORTED;
+  if (d->L >= 2 && !M.fused) {
     DeepPlan D;
     if (!build_deep_plan(D, d, dev.max_smem)) return WTCONV_ERR_UNSUPPORTED;
     auto kd = wtconv_deep_kernel<K, IO>;
@@ -503,8 +530,6 @@ wtconv_status launch_forward_t(const wtconv_desc* d, const Device& dev, const vo
     kd<<<std::min(units, dev.sms * occ), DEEP_NT, smem, st>>>(D, static_cast<const IO*>(x), wl, sl, t1, flip);
     if (cudaGetLastError() != cudaSuccess) return WTCONV_ERR_CUDA;
   }
-  MainPlan M;
-  if (!build_main_plan(M, d, dev.max_smem)) return WTCONV_ERR_UNSUPPORTED;
   const size_t smem = (size_t)M.smem_floats * 4;
   int occ = 0;
   if (M.R3 == 8) {

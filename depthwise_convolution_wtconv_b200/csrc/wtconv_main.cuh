@@ -88,8 +88,10 @@ __device__ __forceinline__ size_t plane_index(const MainPlan& P, const UnitGeo& 
 }
 
 // Folded weights of every channel (one block of wblk floats per channel):
-//   [0, kk4): s0 * W0   [kk4]: s0 * b0 (0 for the adjoint)   [kk4+4 + s*kk4]:
-//   s_1[s] * W_1[s] / 2 (the level-1 synthesis factor); flipped for the adjoint.
+//   [0, kk4): s0 * W0   [kk4]: s0 * b0 (0 for the adjoint)
+//   [kk4+4 + ((l-1)*4 + s)*kk4, ...): 2^-l * s_l[s] * W_l[s], l = 1..L
+// (2^-l: the synthesis factors of the l inverse transforms between level l
+// and the image); every kernel flipped for the adjoint.
 template <int K>
 __global__ void wtconv_fold_kernel(int C, int L, int kk4, int wblk, const float* __restrict__ w0,
                                    const float* __restrict__ b0, const float* __restrict__ s0,
@@ -103,11 +105,12 @@ __global__ void wtconv_fold_kernel(int C, int L, int kk4, int wblk, const float*
       v = s0[c] * w0[(size_t)c * KK + (flip ? KK - 1 - e : e)];
     } else if (e == kk4) {
       v = flip ? 0.f : s0[c] * b0[c];
-    } else if (L >= 1 && e >= kk4 + 4 && e < kk4 + 4 + 4 * kk4) {
-      const int s = (e - kk4 - 4) / kk4, t = (e - kk4 - 4) - s * kk4;
+    } else if (e >= kk4 + 4 && e < kk4 + 4 + 4 * L * kk4) {
+      const int blk = (e - kk4 - 4) / kk4, t = (e - kk4 - 4) - blk * kk4;
       if (t < KK) {
-        const size_t base = (size_t)c * 4 + s;
-        v = (sl[base] * wl[base * KK + (flip ? KK - 1 - t : t)]) * 0.5f;
+        const int l = (blk >> 2) + 1, s = blk & 3;
+        const size_t base = ((size_t)(l - 1) * C + c) * 4 + s;
+        v = (sl[base] * wl[base * KK + (flip ? KK - 1 - t : t)]) * __int_as_float((127 - l) << 23);
       }
     }
     out[i] = v;
@@ -180,6 +183,122 @@ __device__ __forceinline__ void main_stage_item(const MainPlan& P, float* xf, fl
   }
 }
 
+// Staging for whole planes with L >= 2, one 4x4 block of plane j per item:
+// the padded fp32 rows xf, the level-1 subbands s1 (2x2 per band) and the
+// level-2 subbands sd[2] (one per band), the butterflies in registers.
+template <int K, typename IO, bool SMEM>
+__device__ __forceinline__ void main_stage_block(const MainPlan& P, float* slot, int j, const IO* __restrict__ src,
+                                                 int by, int bx) {
+  constexpr int r = K / 2;
+  const int x0 = bx << 2, y0 = by << 2;
+  float4 v[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) v[i] = src4<SMEM>(src + (size_t)(y0 + i) * P.W + x0, x0, P.W, true);
+  float* xf = slot + P.xf.off + j * P.xf.ps + (y0 + r) * P.xf.ld + x0 + r;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) sts4<r>(xf + i * P.xf.ld, v[i]);
+  const int ld1 = P.s1.ld, bs1 = P.s1.ld * P.s1.rows;
+  float* s1 = slot + P.s1.off + j * P.s1.ps + (2 * by + r) * ld1 + 2 * bx + r;
+  float ll[2][2];
+#pragma unroll
+  for (int a = 0; a < 2; ++a) {
+    float l0, h0, g0, k0, l1, h1, g1, k1;
+    haar4(v[2 * a].x, v[2 * a].y, v[2 * a + 1].x, v[2 * a + 1].y, l0, h0, g0, k0);
+    haar4(v[2 * a].z, v[2 * a].w, v[2 * a + 1].z, v[2 * a + 1].w, l1, h1, g1, k1);
+    sts2<r>(s1 + a * ld1, l0, l1);
+    sts2<r>(s1 + bs1 + a * ld1, h0, h1);
+    sts2<r>(s1 + 2 * bs1 + a * ld1, g0, g1);
+    sts2<r>(s1 + 3 * bs1 + a * ld1, k0, k1);
+    ll[a][0] = l0;
+    ll[a][1] = l1;
+  }
+  const BufDesc& d = P.sd[2];
+  const int bs = d.ld * d.rows;
+  float* s2 = slot + d.off + j * d.ps + (by + r) * d.ld + bx + r;
+  float L2, H2, G2, K2;
+  haar4(ll[0][0], ll[0][1], ll[1][0], ll[1][1], L2, H2, G2, K2);
+  s2[0] = L2;
+  s2[bs] = H2;
+  s2[2 * bs] = G2;
+  s2[3 * bs] = K2;
+}
+
+// One 4x4 tile of a deep level's band conv (levels 2..L of whole planes):
+// Zd_l^s = conv(sd_l^s, 2^-l s_l W_l^s), stored plain.
+template <int K>
+__device__ __forceinline__ void main_deep_tile(const MainPlan& P, float* slot, int it) {
+  const int j = P.f_dper.div(it);
+  int rem = it - j * P.f_dper.d;
+  int l = 2;
+  while (l < P.L && rem >= P.dfirst[l + 1]) ++l;
+  rem -= P.dfirst[l];
+  const int s = P.f_dtiles[l].div(rem);
+  rem -= s * P.f_dtiles[l].d;
+  const int ti = P.f_dtx[l].div(rem);
+  const int i0 = ti * 4, j0 = (rem - ti * P.f_dtx[l].d) * 4;
+  const BufDesc& d = P.sd[l];
+  const BufDesc& z = P.zd[l];
+  float acc[4][4];
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
+  conv_tile<K, 4, 4>(slot + d.off + j * d.ps + s * d.ld * d.rows + i0 * d.ld + j0, d.ld,
+                     slot + P.w_off + P.kk4 + 4 + ((l - 1) * 4 + s) * P.kk4, acc);
+  float* o = slot + z.off + j * z.ps + s * z.ld * z.rows + i0 * z.ld + j0;
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+    *reinterpret_cast<float4*>(o + a * z.ld) = make_float4(acc[a][0], acc[a][1], acc[a][2], acc[a][3]);
+}
+
+// t1 of a 4x4 tile of the level-1 grid at (i0, j0), i0 and j0 multiples of 4:
+//   t1(i,j) = sum_{l>=2} sum_s sigma_s(bit_{l-2}(i), bit_{l-2}(j)) Zd_l^s(i >> (l-1), j >> (l-1))
+// (reformulation (2) of arXiv:2608.10805, abstract: every level's share of
+// a position is indexed by the bits of its coordinates).  Added to z.
+__device__ __forceinline__ void main_add_t1(const MainPlan& P, const float* slot, int j, int i0, int j0,
+                                            float (&z)[4][4]) {
+  {
+    const BufDesc& zd = P.zd[2];
+    const int bz = zd.ld * zd.rows;
+    const float* q = slot + zd.off + j * zd.ps + (i0 >> 1) * zd.ld + (j0 >> 1);
+#pragma unroll
+    for (int a2 = 0; a2 < 2; ++a2) {
+      const float2 zl = *reinterpret_cast<const float2*>(q + a2 * zd.ld);
+      const float2 zh = *reinterpret_cast<const float2*>(q + a2 * zd.ld + bz);
+      const float2 zg = *reinterpret_cast<const float2*>(q + a2 * zd.ld + 2 * bz);
+      const float2 zk = *reinterpret_cast<const float2*>(q + a2 * zd.ld + 3 * bz);
+      float o00, o01, o10, o11;
+      synth4(zl.x, zh.x, zg.x, zk.x, o00, o01, o10, o11);
+      z[2 * a2][0] += o00;
+      z[2 * a2][1] += o01;
+      z[2 * a2 + 1][0] += o10;
+      z[2 * a2 + 1][1] += o11;
+      synth4(zl.y, zh.y, zg.y, zk.y, o00, o01, o10, o11);
+      z[2 * a2][2] += o00;
+      z[2 * a2][3] += o01;
+      z[2 * a2 + 1][2] += o10;
+      z[2 * a2 + 1][3] += o11;
+    }
+  }
+  for (int l = 3; l <= P.L; ++l) {
+    // i >> (l-1) and j >> (l-1) are the same for the whole tile
+    const BufDesc& zd = P.zd[l];
+    const int bz = zd.ld * zd.rows;
+    const float* q = slot + zd.off + j * zd.ps + (i0 >> (l - 1)) * zd.ld + (j0 >> (l - 1));
+    const float zl = q[0], zh = q[bz], zg = q[2 * bz], zk = q[3 * bz];
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+      const float sy = (((i0 + a) >> (l - 2)) & 1) ? -1.f : 1.f;
+      const float A = fmaf(sy, zh, zl), B = fmaf(sy, zk, zg);
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        const float sx = (((j0 + b) >> (l - 2)) & 1) ? -1.f : 1.f;
+        z[a][b] += fmaf(sx, B, A);
+      }
+    }
+  }
+}
+
 // Phase A, one tile: band s of plane j, a 4x4 tile of the level-1 grid:
 // the band conv with folded weights (reformulation (3) of arXiv:2608.10805,
 // abstract), t1 added to the LL band, stored to the band's Z plane.
@@ -198,7 +317,9 @@ __device__ __forceinline__ void main_band_tile(const MainPlan& P, float* slot, i
     for (int b = 0; b < 4; ++b) z[a][b] = 0.f;
   const float* s1 = slot + P.s1.off + j * P.s1.ps + s * P.s1.ld * P.s1.rows + i0 * P.s1.ld + j0;
   conv_tile<K, 4, 4>(s1, P.s1.ld, slot + P.w_off + P.kk4 + 4 + s * P.kk4, z);
-  if (s == 0 && P.L >= 2) {
+  if (s == 0 && P.fused) {
+    main_add_t1(P, slot, j, i0, j0, z);
+  } else if (s == 0 && P.L >= 2) {
     const float* t1 = slot + P.t1.off + j * P.t1.ps + i0 * P.t1.ld + j0;
 #pragma unroll
     for (int a = 0; a < 4; ++a) {
@@ -325,7 +446,21 @@ __global__ void __launch_bounds__(MAIN_NT, 4)
     const UnitGeo g = unit_geo(P, blockIdx.x + k * gridDim.x);
     // every thread waits on every phase in order, so a parity wait is exact
     mb_wait(full, k & 1, abort_flag);
-    const int n = g.npb * P.stage_pp;
+    const int n = P.fused ? 0 : g.npb * P.stage_pp;
+    if (P.fused) {
+      const int nb = g.npb * P.f_bpp.d;
+      for (int it = tid; it < nb; it += MAIN_NT) {
+        const int j = P.f_bpp.div(it);
+        const int rem = it - j * P.f_bpp.d;
+        const int by = P.f_bx4.div(rem);
+        const int bx = rem - by * P.f_bx4.d;
+        if (P.bulk_x)
+          main_stage_block<K, IO, true>(P, slot, j, reinterpret_cast<const IO*>(slot + P.raw_off + j * P.raw_pp),
+                                        by, bx);
+        else
+          main_stage_block<K, IO, false>(P, slot, j, x + plane_index(P, g, j) * P.H * P.W, by, bx);
+      }
+    }
     for (int it = tid; it < n; it += MAIN_NT) {
       const int j = P.f_spp.div(it);
       const int rem = it - j * P.stage_pp;
@@ -343,7 +478,7 @@ __global__ void __launch_bounds__(MAIN_NT, 4)
     // unit's copies overwrite while this unit computes
     for (int i = tid; i < (P.wblk >> 2); i += MAIN_NT)
       reinterpret_cast<float4*>(slot + P.w_off)[i] = reinterpret_cast<const float4*>(slot + P.wraw_off)[i];
-    if (P.L >= 2) {
+    if (P.L >= 2 && !P.fused) {
       const int rows = P.TH >> 1, q4 = (P.W1 + 3) >> 2;
       for (int it = tid; it < g.npb * rows * q4; it += MAIN_NT) {
         const int j = it / (rows * q4), rem = it - j * rows * q4;
@@ -362,6 +497,19 @@ __global__ void __launch_bounds__(MAIN_NT, 4)
     if (*abort_flag) break;  // uniform: read after the barrier
     if (tid == 0 && k + 1 < myunits)
       main_issue<IO>(P, slot, full, unit_geo(P, blockIdx.x + (k + 1) * gridDim.x), x, t1g, wfold);
+    if (P.fused) {
+      // levels 3..L of the pyramid, then every deep level's band convs
+      for (int l = 3; l <= P.L; ++l) {
+        const BufDesc& sb = P.sd[l - 1];
+        const BufDesc& d = P.sd[l];
+        pyramid_level(g.npb, P.H >> l, P.W >> l, slot + sb.off + (K / 2) * sb.ld + K / 2, sb.ld, sb.ps,
+                      slot + d.off + (K / 2) * d.ld + K / 2, d.ld, d.ld * d.rows, d.ps);
+        __syncthreads();
+      }
+      const int nd = g.npb * P.f_dper.d;
+      for (int it = tid; it < nd; it += MAIN_NT) main_deep_tile<K>(P, slot, it);
+      __syncthreads();
+    }
     if (P.L >= 1) {
       const int na = g.npb * P.a_pp;
       for (int it = tid; it < na; it += MAIN_NT) main_band_tile<K>(P, slot, it);

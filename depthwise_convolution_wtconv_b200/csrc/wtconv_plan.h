@@ -122,6 +122,11 @@ struct MainPlan {
   int w_off;                 // the current unit's folded weights
   BufDesc xf, s1, t1, zb;    // per-plane copies at ps stride (zb: the four level-1 Z planes)
   int a_pp;                  // phase-A tiles per plane: 4 bands x ceil(TH/8) x ceil(W1/4)
+  int fused;                 // whole planes with L >= 2: levels >= 2 computed here, t1 on the fly
+  BufDesc sd[MAXL + 1], zd[MAXL + 1];  // fused: subbands and band-conv outputs of levels 2..L
+  int dfirst[MAXL + 2];      // fused: first deep-conv tile of level l within a plane
+  FDiv f_dtiles[MAXL + 1], f_dtx[MAXL + 1], f_dper;  // fused: 4x4 tiles per band, per tile row; per plane
+  FDiv f_bpp, f_bx4;         // fused: 4x4 staging blocks per plane, per block row
   FDiv f_tiles, f_tpp, f_tx, f_stq, f_spp, f_bands, f_C;
   FDiv f_app, f_abt, f_atx;  // phase-A decomposition: per plane, per band, per tile row
   int smem_floats;

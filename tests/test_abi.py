@@ -51,12 +51,12 @@ def test_workspace_sizes(lib):
     d = _desc()
     V = 25 * (1 + 4 * 2) + 1
     t1 = 2 * 3 * 8 * 8 * 4  # level-1 resolution synthesis of levels >= 2
-    folded = 3 * (5 * 28 + 4) * 4  # per channel: base + 4 level-1 kernels (k*k padded to 28) + bias
+    folded = 3 * ((1 + 4 * 2) * 28 + 4) * 4  # per channel: base + 4 kernels per level (k*k padded to 28) + bias
     assert lib.wtconv_workspace_size(ctypes.byref(d), 0) == 16 + t1 + folded
     assert lib.wtconv_workspace_size(ctypes.byref(d), 1) == 16 + t1 + folded
     assert lib.wtconv_workspace_size(ctypes.byref(d), 2) == 16 + 2 * 3 * V * 4
     assert lib.wtconv_workspace_size(ctypes.byref(d), 3) == 16 + max(2 * 3 * V * 4, t1 + folded)
-    assert lib.wtconv_workspace_size(ctypes.byref(_desc(L=1)), 0) == 16 + folded
+    assert lib.wtconv_workspace_size(ctypes.byref(_desc(L=1)), 0) == 16 + 3 * (5 * 28 + 4) * 4
     assert lib.wtconv_workspace_size(ctypes.byref(_desc(L=0)), 0) == 16 + 3 * (28 + 4) * 4
     assert lib.wtconv_workspace_size(ctypes.byref(_desc(k=4)), 2) == 0
     assert lib.wtconv_workspace_size(None, 2) == 0
