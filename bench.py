@@ -58,19 +58,16 @@ def algorithmic_counts(wl):
     )
 
 
-def launches_per_step(wl):
-    """Kernels of this library launched per step: forward and backward-data
-    each run the weight-folding kernel, the deep-level kernel (L >= 2) and
-    the output kernel; backward-weight runs its partial-sum kernel and the
-    fixed-order finalize kernel."""
-    per_pass = 2 + (1 if wl.L >= 2 else 0)
-    return 2 * per_pass + 2
+def launches_per_step(wt, desc):
+    """Kernels of this library launched per step (forward, backward-data,
+    backward-weight), as the library reports them for the shape."""
+    return sum(wt.kernel_launches(desc, op) for op in (0, 1, 2))
 
 
 PASS_KERNELS = {
-    "fwd": "wtconv_fold_kernel + wtconv_deep_kernel (L >= 2) + wtconv_main_kernel",
-    "bwd_data": "wtconv_fold_kernel + wtconv_deep_kernel (L >= 2) + wtconv_main_kernel (flipped)",
-    "bwd_weight": "wtconv_bwdw_kernel + wtconv_bwdw_finalize",
+    "fwd": "wtconv_fold_kernel + wtconv_main_kernel (+ wtconv_deep_kernel for row-band planes)",
+    "bwd_data": "wtconv_fold_kernel + wtconv_main_kernel, flipped (+ wtconv_deep_kernel for row-band planes)",
+    "bwd_weight": "wtconv_bwdw_kernel + wtconv_bwdw_finalize (row-band planes: wtconv_bwband_kernel per level)",
 }
 
 
@@ -203,16 +200,16 @@ def run_ours(args, wl, world, rank, local):
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
     stream = torch.cuda.current_stream(device)
 
-    def step(ev=None, x=X, dy=dY, y=Y, dx=dX):
+    def step(ev=None, x=X, dy=dY, y=Y, dx=dX, st=stream):
         if ev is not None:
             ev[0].record(stream)
-        wt.forward(x, p["W0"], p["b0"], p["s0"], Wl, sl, y=y, ws=ws, stream=stream)
+        wt.forward(x, p["W0"], p["b0"], p["s0"], Wl, sl, y=y, ws=ws, stream=st)
         if ev is not None:
             ev[1].record(stream)
-        wt.backward_data(dy, p["W0"], p["s0"], Wl, sl, dx=dx, ws=ws, stream=stream)
+        wt.backward_data(dy, p["W0"], p["s0"], Wl, sl, dx=dx, ws=ws, stream=st)
         if ev is not None:
             ev[2].record(stream)
-        wt.backward_weight(x, dy, p["W0"], p["b0"], p["s0"], Wl, sl, grads=grads, ws=ws, stream=stream)
+        wt.backward_weight(x, dy, p["W0"], p["b0"], p["s0"], Wl, sl, grads=grads, ws=ws, stream=st)
         if ev is not None:
             ev[3].record(stream)
         allreduce_grads(gflat, world)
@@ -223,27 +220,66 @@ def run_ours(args, wl, world, rank, local):
         flush.fill_(0.0)
         step()
     torch.cuda.synchronize(device)
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize(device)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
-    sampler = ClockSampler(local)
-    sampler.start()
-    t_wall = time.perf_counter()
-    for i in range(args.steps):
-        flush.fill_(0.0)
-        step(evs[i])
-    torch.cuda.synchronize(device)
-    t_wall = time.perf_counter() - t_wall
-    clocks = sampler.stop()
-    if world > 1:
-        dist.barrier()
+
+    # each pass captured once as a CUDA graph (the same kernels, launched
+    # without per-call host work); the gradient all-reduce stays eager
+    graphs = []
+    if not args.eager:
+        cap = torch.cuda.Stream(device)
+        cap.wait_stream(stream)
+        for fn in (lambda: wt.forward(X, p["W0"], p["b0"], p["s0"], Wl, sl, y=Y, ws=ws, stream=cap),
+                   lambda: wt.backward_data(dY, p["W0"], p["s0"], Wl, sl, dx=dX, ws=ws, stream=cap),
+                   lambda: wt.backward_weight(X, dY, p["W0"], p["b0"], p["s0"], Wl, sl, grads=grads, ws=ws,
+                                              stream=cap)):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=cap):
+                fn()
+            graphs.append(g)
+        stream.wait_stream(cap)
+        for _ in range(args.warmup):
+            flush.fill_(0.0)
+            for g in graphs:
+                g.replay()
+        torch.cuda.synchronize(device)
+
+    def graph_step(ev):
+        ev[0].record(stream)
+        for i, g in enumerate(graphs):
+            g.replay()
+            ev[i + 1].record(stream)
+        allreduce_grads(gflat, world)
+        ev[4].record(stream)
+
+    def timed(run):
+        torch.cuda.synchronize(device)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(device)
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+        sampler = ClockSampler(local)
+        sampler.start()
+        t_wall = time.perf_counter()
+        for i in range(args.steps):
+            flush.fill_(0.0)
+            run(evs[i])
+        torch.cuda.synchronize(device)
+        t_wall = time.perf_counter() - t_wall
+        clocks = sampler.stop()
+        if world > 1:
+            dist.barrier()
+        return evs, clocks, t_wall
+
+    eager_evs, _, _ = timed(step) if graphs else (None, None, None)
+    evs, clocks, t_wall = timed(graph_step if graphs else step)
     per_step = [e[0].elapsed_time(e[4]) for e in evs]
     t_fwd = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
     t_bd = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
     t_bw = sum(e[2].elapsed_time(e[3]) for e in evs) / args.steps
     total_ms = max_over_ranks(sum(per_step), world, device)
     ms_per_step = total_ms / args.steps
+    eager_ms = None
+    if eager_evs is not None:
+        eager_ms = max_over_ranks(sum(e[0].elapsed_time(e[4]) for e in eager_evs), world, device) / args.steps
 
     # end to end through the public API: pinned host inputs in, results out
     hX = inp["X"].to(dt).pin_memory()
@@ -311,9 +347,13 @@ def run_ours(args, wl, world, rank, local):
         "hbm": {"achieved_gbs": hbm_gbs, "peak_gbs": hbm_peak, "frac": hbm_gbs / hbm_peak,
                 "algorithmic_bytes_per_step": step_bytes, "peak_source": peak_src},
         "kernels_ms": kernels,
+        "timing": ("each pass one CUDA graph replay" if graphs else "eager library calls") +
+                  ", CUDA events on the launching stream",
+        "eager": None if eager_ms is None else {"ms_per_step": eager_ms, "value": world * 1000.0 / eager_ms,
+                                                "unit": "steps/s"},
         "e2e": {"value": world * 1000.0 / e2e_ms, "unit": "steps/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
-        "gpu_launches": launches_per_step(wl) * args.steps,
+        "gpu_launches": launches_per_step(wt, desc) * args.steps,
         "clocks": clocks,
         "wall_s_timed_region": t_wall,
     }
@@ -426,6 +466,7 @@ def main(argv=None):
     ap.add_argument("--workload", default=BENCH_WORKLOAD, choices=list(WORKLOADS))
     ap.add_argument("--cpu-sample-n", type=int, default=32)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--eager", action="store_true", help="time eager library calls instead of CUDA graph replays")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

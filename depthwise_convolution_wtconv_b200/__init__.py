@@ -5,6 +5,6 @@ C ABI, see include/wtconv.h); `forward`, `backward_data`, `backward_weight`
 and `backward` are thin ctypes wrappers over it that take CUDA tensors.
 """
 from ._lib import (  # noqa: F401
-    forward, backward_data, backward_weight, backward, backward_weight_noalloc, workspace_size, make_desc, load,
+    forward, backward_data, backward_weight, backward, backward_weight_noalloc, workspace_size, kernel_launches, make_desc, load,
     WTConvError, EXPORTS, LIB_PATH,
 )

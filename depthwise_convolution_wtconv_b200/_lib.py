@@ -22,7 +22,7 @@ NOALLOC_SCRATCH_BYTES = 8 << 20
 
 # every symbol include/wtconv.h declares
 EXPORTS = ("wtconv_workspace_size", "wtconv_forward", "wtconv_backward_data", "wtconv_backward_weight",
-           "wtconv_backward", "wtconv_backward_weight_noalloc", "wtconv_status_string")
+           "wtconv_backward", "wtconv_backward_weight_noalloc", "wtconv_kernel_launches", "wtconv_status_string")
 
 
 class WTConvDesc(ctypes.Structure):
@@ -63,6 +63,8 @@ def load(path=LIB_PATH):
     lib.wtconv_backward_weight_noalloc.restype = ctypes.c_int
     lib.wtconv_status_string.argtypes = [ctypes.c_int]
     lib.wtconv_status_string.restype = ctypes.c_char_p
+    lib.wtconv_kernel_launches.argtypes = [dp, ctypes.c_int]
+    lib.wtconv_kernel_launches.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -73,6 +75,11 @@ def make_desc(N, C, H, W, k, L, io):
 
 def workspace_size(desc, op):
     return int(load().wtconv_workspace_size(ctypes.byref(desc), op))
+
+
+def kernel_launches(desc, op):
+    """Kernel launches one call of `op` makes for the shape `desc`."""
+    return int(load().wtconv_kernel_launches(ctypes.byref(desc), op))
 
 
 def _ptr(t):

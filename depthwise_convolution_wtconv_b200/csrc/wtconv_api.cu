@@ -7,11 +7,13 @@
 #include <cstdint>
 #include <initializer_list>
 #include <mutex>
+#include <vector>
 
 #include "wtconv.h"
 #include "wtconv_kernels.cuh"
 #include "wtconv_main.cuh"
 #include "wtconv_bwband.cuh"
+#include "wtconv_bwdw.cuh"
 
 namespace wt {
 namespace {
@@ -65,187 +67,9 @@ BufDesc make_plain(int& cur, int h, int w, std::initializer_list<TileShape> shap
   return d;
 }
 
-void relocate(BufDesc& d, int base, int slab) {
-  d.off += base;
-  d.ps = slab;
-}
 
 int io_bytes(const wtconv_desc* d) { return d->io == WTCONV_BF16 ? 2 : 4; }
 
-void fill_common(Plan& P, const wtconv_desc* d) {
-  P = Plan{};
-  P.N = d->N;
-  P.C = d->C;
-  P.H = d->H;
-  P.W = d->W;
-  P.K = d->k;
-  P.r = d->k / 2;
-  P.L = d->L;
-  P.H1 = d->L >= 1 ? d->H / 2 : d->H;
-  P.W1 = d->L >= 1 ? d->W / 2 : d->W;
-  P.kk4 = rup(d->k * d->k, 4);
-  P.vec_in = (d->W % 4) == 0;
-  P.vec_out = d->io == WTCONV_BF16 ? (d->W % 8) == 0 : (d->W % 4) == 0;
-  P.prefetch_ok = ((size_t)d->H * d->W * io_bytes(d)) % 16 == 0;
-  P.io_bytes = io_bytes(d);
-  P.nthreads = NT;
-  P.V = d->k * d->k * (1 + 4 * d->L) + 1;
-}
-
-// Per-plane slab of the forward / backward-data kernel.
-int forward_slab(Plan& P) {
-  const int r = P.r, L = P.L, RB = P.R3 / 2;
-  int cur = 0;
-  P.xf = make_shifted(cur, P.H, P.W, r, {{P.R3, C3_CW}}, 1);
-  if (L >= 1) P.s1 = make_shifted(cur, P.H1, P.W1, r, {{RB, 4}, {2, 2}}, 4);
-  if (L >= 2) {
-    P.t1 = make_plain(cur, P.H1, P.W1, {{RB, 4}, {1, 4}}, 1);
-    for (int l = 2; l <= L; ++l) P.sd[l] = make_shifted(cur, P.H >> l, P.W >> l, r, {{DP_R, DP_CW}, {2, 2}}, 4);
-    for (int l = 2; l <= L; ++l) P.zd[l] = make_plain(cur, P.H >> l, P.W >> l, {{DP_R, DP_CW}}, 4);
-  }
-  P.deep_off = 0;
-  P.deep_floats = 0;
-  return rup(cur, 4);
-}
-
-void forward_items(Plan& P) {
-  const int L = P.L;
-  int per, xdiv;
-  if (L >= 2) {
-    xdiv = P.W >> 2;
-    per = (P.H >> 2) * xdiv;
-  } else if (L == 1) {
-    xdiv = cdiv_h(P.W, 4);
-    per = P.H1 * xdiv;
-  } else {
-    xdiv = cdiv_h(P.W, 4);
-    per = P.H * xdiv;
-  }
-  P.f_stage_per = make_fdiv(per);
-  P.f_stage_x = make_fdiv(xdiv);
-  int first = 0;
-  for (int l = 0; l <= MAXL + 1; ++l) P.deep_first[l] = 0;
-  for (int l = 2; l <= L; ++l) {
-    const int tx = cdiv_h(P.W >> l, DP_CW), tiles = cdiv_h(P.H >> l, DP_R) * tx;
-    P.f_l_tiles[l] = make_fdiv(tiles);
-    P.f_l_tx[l] = make_fdiv(tx);
-    P.deep_first[l] = first;
-    first += 4 * tiles;
-  }
-  P.deep_items = first;
-  if (L >= 2) P.deep_first[L + 1] = first;
-  P.f_deep_per = make_fdiv(first > 0 ? first : 1);
-  const int tq = cdiv_h(P.W1, 4);
-  P.f_t1_x = make_fdiv(tq);
-  P.f_t1_per = make_fdiv(P.H1 * tq);
-  const int ox = cdiv_h(P.W, C3_CW);
-  P.f_out_x = make_fdiv(ox);
-  P.f_out_per = make_fdiv(cdiv_h(P.H, P.R3) * ox);
-}
-
-// Shared-memory header: mbarrier (8 bytes) and abort flag, 16 bytes.
-constexpr int HEADER_FLOATS = 4;
-
-void finish_forward_plan(Plan& P, int PB) {
-  const int slab = forward_slab(P);
-  P.PB = PB;
-  P.nbatch = (P.N + PB - 1) / PB;
-  P.w_off = HEADER_FLOATS;
-  P.use_bulk = P.prefetch_ok;
-  P.raw_off = rup(P.w_off + (1 + 4 * P.L) * P.kk4 + 4, 4);
-  const int raw_floats = P.use_bulk ? rup((int)((size_t)PB * P.H * P.W * P.io_bytes / 4), 4) : 0;
-  const int base = P.raw_off + raw_floats;
-  for (BufDesc* b : {&P.xf, &P.s1, &P.t1, &P.zb, &P.t2}) relocate(*b, base, slab);
-  for (int l = 0; l <= MAXL; ++l) {
-    relocate(P.sd[l], base, slab);
-    relocate(P.zd[l], base, slab);
-  }
-  P.smem_floats = base + PB * slab;
-  forward_items(P);
-}
-
-// Tiles of the output pass per plane, for the batch-size choice.
-int output_items(const Plan& P, int R3) { return ((P.H + R3 - 1) / R3) * ((P.W + C3_CW - 1) / C3_CW); }
-
-// Threads per CTA of the forward kernel: 128 when one plane has few
-// output tiles, so that a batch of one plane still keeps most threads busy.
-int forward_threads(const Plan& P) { return output_items(P, P.H >= 8 ? 4 : 2) <= 128 ? 128 : 256; }
-
-void build_forward_plan(Plan& P, const wtconv_desc* d, int max_smem) {
-  fill_common(P, d);
-  P.R3 = (P.H >= 8) ? 4 : 2;
-  P.nthreads = forward_threads(P);
-  const int items = output_items(P, P.R3);
-  int PB = std::max(1, std::min(d->N, P.nthreads / items));
-  const size_t budget = (size_t)max_smem / 2;
-  for (;;) {
-    finish_forward_plan(P, PB);
-    if (PB == 1 || (size_t)P.smem_floats * 4 <= budget) break;
-    --PB;
-  }
-}
-
-void bwdw_items(Plan& P) {
-  forward_items(P);  // staging and deep-level decompositions are shared
-  const int bx = cdiv_h(P.W, BW_CW);
-  P.f_bw_x = make_fdiv(bx);
-  P.f_bw_per = make_fdiv(cdiv_h(P.H, BW_R) * bx);
-  const int b1 = cdiv_h(P.W1, B1_CW);
-  P.f_b1_x = make_fdiv(b1);
-  P.f_b1_per = make_fdiv(cdiv_h(P.H1, B1_R) * b1);
-}
-
-int bwdw_slab(Plan& P) {
-  const int r = P.r, L = P.L;
-  int cur = 0;
-  P.xf = make_shifted(cur, P.H, P.W, r, {{BW_R, BW_CW}}, 1);
-  P.gf = make_plain(cur, P.H, P.W, {{BW_R, BW_CW}}, 1);
-  if (L >= 1) {
-    P.s1 = make_shifted(cur, P.H1, P.W1, r, {{B1_R, B1_CW}, {2, 2}}, 4);
-    P.g1 = make_plain(cur, P.H1, P.W1, {{B1_R, B1_CW}, {2, 2}}, 4);
-  }
-  for (int l = 2; l <= L; ++l) {
-    P.sd[l] = make_shifted(cur, P.H >> l, P.W >> l, r, {{DP_R, DP_CW}, {2, 2}}, 4);
-    P.gd[l] = make_plain(cur, P.H >> l, P.W >> l, {{DP_R, DP_CW}, {2, 2}}, 4);
-  }
-  return rup(cur, 4);
-}
-
-void finish_bwdw_plan(Plan& P, int PB) {
-  const int slab = bwdw_slab(P);
-  P.PB = PB;
-  const int ndeep = P.L >= 2 ? (P.L - 1) * 4 : 0;
-  P.gdeep_off = HEADER_FLOATS;
-  P.dpart_off = P.gdeep_off + ndeep * P.kk4;
-  P.use_bulk = P.prefetch_ok;
-  const int raw_floats = P.use_bulk ? rup((int)((size_t)PB * P.H * P.W * P.io_bytes / 4), 4) : 0;
-  P.raw_off = rup(P.dpart_off + ndeep * DSLOTS * P.kk4, 4);
-  P.rawg_off = P.raw_off + raw_floats;
-  const int base = P.rawg_off + raw_floats;
-  for (BufDesc* b : {&P.xf, &P.gf, &P.s1, &P.g1}) relocate(*b, base, slab);
-  for (int l = 0; l <= MAXL; ++l) {
-    relocate(P.sd[l], base, slab);
-    relocate(P.gd[l], base, slab);
-  }
-  P.red_off = base;
-  P.smem_floats = std::max(base + PB * slab, base + NT * P.kk4 + NT);
-  bwdw_items(P);
-}
-
-void build_bwdw_plan(Plan& P, const wtconv_desc* d, int max_smem) {
-  fill_common(P, d);
-  P.R3 = 2;
-  const int items = ((P.H + BW_R - 1) / BW_R) * ((P.W + BW_CW - 1) / BW_CW);
-  const int nbase = P.L >= 1 ? 128 : NT;
-  int PB = std::max(1, std::min(d->N, (nbase + items - 1) / items));
-  for (;;) {
-    finish_bwdw_plan(P, PB);
-    if (PB == 1 || (size_t)P.smem_floats * 4 <= (size_t)max_smem / 2) break;
-    --PB;
-  }
-}
-
-// ------------------------------------------------ pipelined output kernel
 constexpr int SM_SMEM = 233472;  // shared memory per SM on sm_100a (228 KB)
 
 // Floats of one channel's folded weights: the base kernel, the bias and
@@ -484,22 +308,72 @@ struct Device {
   int sms = 0, max_smem = 0;
 };
 
+// Launch set-up is cached so that a call costs little host time: the
+// device's SM count and shared-memory limit per device, and per (kernel,
+// device) the largest dynamic shared-memory size set so far (the attribute
+// only ever grows) and the occupancy per (shared memory, threads).
+constexpr int CACHE_DEVICES = 64;
+std::mutex g_setup_mutex;
+Device g_devices[CACHE_DEVICES];
+
+struct KernelSetup {
+  const void* func;
+  int device, nthreads;
+  size_t smem;
+  int occ;
+};
+std::vector<KernelSetup> g_occ;
+std::vector<std::pair<std::pair<const void*, int>, size_t>> g_smem_set;
+
 wtconv_status query_device(Device& dev) {
   int id = 0;
   if (cudaGetDevice(&id) != cudaSuccess) return WTCONV_ERR_CUDA;
+  if (id >= 0 && id < CACHE_DEVICES) {
+    std::lock_guard<std::mutex> lock(g_setup_mutex);
+    if (g_devices[id].sms > 0) {
+      dev = g_devices[id];
+      return WTCONV_OK;
+    }
+  }
   if (cudaDeviceGetAttribute(&dev.sms, cudaDevAttrMultiProcessorCount, id) != cudaSuccess) return WTCONV_ERR_CUDA;
   if (cudaDeviceGetAttribute(&dev.max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, id) != cudaSuccess)
     return WTCONV_ERR_CUDA;
+  if (id >= 0 && id < CACHE_DEVICES) {
+    std::lock_guard<std::mutex> lock(g_setup_mutex);
+    g_devices[id] = dev;
+  }
   return WTCONV_OK;
 }
 
+// Makes `kern` launchable with `smem` bytes of dynamic shared memory and
+// returns its resident CTAs per SM for `nthreads` threads.
 template <typename F>
 wtconv_status prepare(F kern, size_t smem, int& occ, int nthreads = NT) {
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-    return WTCONV_ERR_CUDA;
+  int id = 0;
+  if (cudaGetDevice(&id) != cudaSuccess) return WTCONV_ERR_CUDA;
+  const void* f = reinterpret_cast<const void*>(kern);
+  std::lock_guard<std::mutex> lock(g_setup_mutex);
+  for (const KernelSetup& k : g_occ)
+    if (k.func == f && k.device == id && k.nthreads == nthreads && k.smem == smem) {
+      occ = k.occ;
+      return occ < 1 ? WTCONV_ERR_UNSUPPORTED : WTCONV_OK;
+    }
+  size_t* set = nullptr;
+  for (auto& e : g_smem_set)
+    if (e.first.first == f && e.first.second == id) set = &e.second;
+  if (!set) {
+    g_smem_set.push_back({{f, id}, 0});
+    set = &g_smem_set.back().second;
+  }
+  if (smem > *set) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+      return WTCONV_ERR_CUDA;
+    *set = smem;
+  }
   occ = 0;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, nthreads, smem) != cudaSuccess)
     return WTCONV_ERR_CUDA;
+  g_occ.push_back(KernelSetup{f, id, nthreads, smem, occ});
   if (occ < 1) return WTCONV_ERR_UNSUPPORTED;
   return WTCONV_OK;
 }
@@ -583,11 +457,145 @@ constexpr size_t WS_HEADER = 16;
 constexpr int PLAN_SMEM = 232448;
 constexpr int PLAN_SMS = 148;
 
+// ---- whole-plane weight-gradient plan
+
+// Per-plane slab (floats): x padded and dy plain, and both pyramids.
+int bw_slab(BwPlan& B) {
+  const int r = B.r;
+  int cur = 0;
+  B.xf = make_shifted(cur, B.H, B.W, r, {{4, 4}}, 1);
+  B.gf = make_plain(cur, B.H, B.W, {{4, 4}}, 1);
+  B.s1 = B.g1 = BufDesc{0, 0, 0, 0};
+  for (int l = 0; l <= MAXL; ++l) B.sd[l] = B.gd[l] = BufDesc{0, 0, 0, 0};
+  if (B.L >= 1) {
+    B.s1 = make_shifted(cur, B.H1, B.W1, r, {{4, 4}}, 4);
+    B.g1 = make_plain(cur, B.H1, B.W1, {{4, 4}}, 4);
+  }
+  for (int l = 2; l <= B.L; ++l) {
+    B.sd[l] = make_shifted(cur, B.H >> l, B.W >> l, r, {{4, 4}}, 4);
+    B.gd[l] = make_plain(cur, B.H >> l, B.W >> l, {{4, 4}}, 4);
+  }
+  return rup(cur, 4);
+}
+
+// Layout for PB planes per unit; false when it needs more than max_smem.
+bool bw_layout(BwPlan& B, int PB, int max_smem) {
+  B.PB = PB;
+  B.ps = bw_slab(B);
+  const size_t plane_bytes = (size_t)B.H * B.W * B.io_bytes;
+  B.bulk = plane_bytes % 16 == 0;
+  B.raw_pp = B.bulk ? rup((int)((plane_bytes + 3) / 4), 4) : 0;
+  int cur = 0;  // relative to the slot, which starts after the header
+  B.raw_x = cur;
+  cur += PB * B.raw_pp;
+  B.raw_g = cur;
+  cur += PB * B.raw_pp;
+  const int base = cur;
+  for (BufDesc* bd : {&B.xf, &B.gf, &B.s1, &B.g1}) bd->off += base;
+  for (int l = 2; l <= B.L; ++l) {
+    B.sd[l].off += base;
+    B.gd[l].off += base;
+  }
+  B.red_off = base;
+  const int need = std::max(base + PB * B.ps, base + BW_NT * B.kk4 + BW_NT);
+  B.smem_floats = MAIN_HEADER + rup(need, 4);
+  return (size_t)B.smem_floats * 4 <= (size_t)max_smem;
+}
+
+// Branches and their threads: each of the 1 + 4L branches (base taps, then
+// band s of level l) gets a range of threads sized to its tiles, filled
+// greedily towards the branch with the most tiles per thread.
+void bw_branches(BwPlan& B) {
+  const int KK = B.K * B.K;
+  B.nbr = 1 + 4 * B.L;
+  int tiles[BW_MAXB], thr[BW_MAXB];
+  for (int b = 0; b < B.nbr; ++b) {
+    BwBranch& br = B.br[b];
+    const BufDesc* a;
+    const BufDesc* g;
+    int h, w, s = 0;
+    if (b == 0) {
+      a = &B.xf;
+      g = &B.gf;
+      h = B.H;
+      w = B.W;
+    } else {
+      const int l = 1 + (b - 1) / 4;
+      s = (b - 1) % 4;
+      a = l == 1 ? &B.s1 : &B.sd[l];
+      g = l == 1 ? &B.g1 : &B.gd[l];
+      h = B.H >> l;
+      w = B.W >> l;
+    }
+    br.a_off = a->off + s * a->ld * a->rows;
+    br.a_ld = a->ld;
+    br.g_off = g->off + s * g->ld * g->rows;
+    br.g_ld = g->ld;
+    br.seg = KK * b;
+    const int tx = cdiv_h(w, 4);
+    tiles[b] = cdiv_h(h, 4) * tx * B.PB;
+    br.f_tiles = make_fdiv(cdiv_h(h, 4) * tx);
+    br.f_tx = make_fdiv(tx);
+    thr[b] = 1;
+  }
+  for (int left = BW_NT - B.nbr; left > 0; --left) {
+    int best = -1;
+    long bestq = 1;
+    for (int b = 0; b < B.nbr; ++b) {
+      const long q = (tiles[b] + thr[b] - 1) / thr[b];
+      if (q > bestq || (q == bestq && best >= 0 && tiles[b] > tiles[best])) {
+        bestq = q;
+        best = b;
+      }
+    }
+    if (best < 0) break;  // every branch has one tile per thread at most
+    ++thr[best];
+  }
+  int first = 0;
+  for (int b = 0; b < B.nbr; ++b) {
+    B.br[b].first = first;
+    B.br[b].nthr = thr[b];
+    first += thr[b];
+  }
+}
+
+// Whole-plane plan: the most planes per unit (up to two tiles per thread)
+// that fit two CTAs per SM, else one.  False when one plane does not fit.
+bool build_bw_plan(BwPlan& B, const wtconv_desc* d, int max_smem) {
+  B = BwPlan{};
+  B.N = d->N;
+  B.C = d->C;
+  B.H = d->H;
+  B.W = d->W;
+  B.K = d->k;
+  B.r = d->k / 2;
+  B.L = d->L;
+  B.H1 = d->L >= 1 ? d->H / 2 : d->H;
+  B.W1 = d->L >= 1 ? d->W / 2 : d->W;
+  B.kk4 = rup(d->k * d->k, 4);
+  B.V = d->k * d->k * (1 + 4 * d->L) + 1;
+  B.io_bytes = io_bytes(d);
+  B.vec_in = (d->W % 4) == 0;
+  B.BH = d->L >= 2 ? 4 : (d->L == 1 ? 2 : 1);
+  int per_plane = cdiv_h(d->H, 4) * cdiv_h(d->W, 4);
+  for (int l = 1; l <= d->L; ++l) per_plane += 4 * cdiv_h(d->H >> l, 4) * cdiv_h(d->W >> l, 4);
+  const int pb0 = std::max(1, std::min(d->N, cdiv_h(2 * BW_NT, per_plane)));
+  bool ok = false;
+  for (const int budget : {(int)(SM_SMEM / 2 - 1024), max_smem}) {
+    for (int pb = pb0; pb >= 1 && !ok; --pb) ok = bw_layout(B, pb, std::min(budget, max_smem));
+    if (ok) break;
+  }
+  if (!ok) return false;
+  B.f_sx = make_fdiv(cdiv_h(d->W, 4));
+  B.f_spp = make_fdiv((d->H / B.BH) * cdiv_h(d->W, 4));
+  bw_branches(B);
+  return true;
+}
+
 // True when one plane's whole weight-gradient working set fits one SM.
 bool bwdw_whole_plane(const wtconv_desc* d) {
-  Plan P;
-  build_bwdw_plan(P, d, PLAN_SMEM);
-  return (size_t)P.smem_floats * 4 <= (size_t)PLAN_SMEM;
+  BwPlan B;
+  return build_bw_plan(B, d, PLAN_SMEM);
 }
 
 // ---- row-band weight-gradient path
@@ -703,60 +711,71 @@ size_t bwdw_ws_bytes(const wtconv_desc* d) {
   return WS_HEADER + band_part_bytes(d, G) + band_ll_floats(d) * sizeof(float);
 }
 
-template <int K, typename IO>
-wtconv_status launch_bwdw_t(Plan& P, const Device& dev, const void* x, const void* dy, const float* w0,
-                            const float* b0, const float* s0, const float* wl, const float* sl, float* dw0,
-                            float* db0, float* ds0, float* dwl, float* dsl, float* part, int* status,
-                            cudaStream_t st, int max_groups) {
-  auto kern = wtconv_bwdw_kernel<K, IO>;
-  const size_t smem = (size_t)P.smem_floats * 4;
-  int occ = 0;
-  wtconv_status e = prepare(kern, smem, occ);
-  if (e != WTCONV_OK) return e;
-  // planes per CTA: fewest sequential batches per CTA slot (waves x batches
-  // per CTA), ties broken towards longer CTAs (fewer partial sums)
-  const int slots = dev.sms * occ;
-  long best = -1;
-  for (int ppc = P.PB; ppc < P.N + P.PB; ppc += P.PB) {
-    const int p = std::min(ppc, P.N);
-    const int groups = (P.N + p - 1) / p;
-    if (groups > max_groups) continue;
-    const long ctas = (long)P.C * groups;
-    const long cost = ((ctas + slots - 1) / slots) * ((p + P.PB - 1) / P.PB);
-    if (best < 0 || cost <= best) {
-      best = cost;
-      P.planes_per_cta = p;
-    }
-    if (p == P.N) break;
-  }
-  P.ngroups = (P.N + P.planes_per_cta - 1) / P.planes_per_cta;
-  kern<<<P.C * P.ngroups, NT, smem, st>>>(P, static_cast<const IO*>(x), static_cast<const IO*>(dy), part,
-                                          status);
-  if (cudaGetLastError() != cudaSuccess) return WTCONV_ERR_CUDA;
-  const size_t fsmem = (size_t)P.V * sizeof(float);
+template <int K>
+wtconv_status launch_finalize(const wtconv_desc* d, int groups, const float* part, const float* w0, const float* b0,
+                              const float* s0, const float* wl, const float* sl, float* dw0, float* db0, float* ds0,
+                              float* dwl, float* dsl, cudaStream_t st) {
+  const FinalizeArgs F{d->C, d->L, d->k * d->k * (1 + 4 * d->L) + 1, groups};
+  const size_t fsmem = (size_t)F.V * sizeof(float);
   auto fin = wtconv_bwdw_finalize<K>;
-  if (fsmem > 48 * 1024 &&
-      cudaFuncSetAttribute(fin, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fsmem) != cudaSuccess)
-    return WTCONV_ERR_CUDA;
-  fin<<<P.C, 128, fsmem, st>>>(P, part, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl);
+  int occ = 0;
+  if (fsmem > 48 * 1024) {
+    const wtconv_status e = prepare(fin, fsmem, occ, 128);
+    if (e != WTCONV_OK) return e;
+  }
+  fin<<<F.C, 128, fsmem, st>>>(F, part, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl);
   return cudaGetLastError() == cudaSuccess ? WTCONV_OK : WTCONV_ERR_CUDA;
 }
 
-template <int K>
-wtconv_status launch_bwdw_k(Plan& P, const Device& dev, wtconv_dtype io, const void* x, const void* dy,
+template <int K, int LC, typename IO>
+wtconv_status launch_bwdw_t(BwPlan& B, const Device& dev, const wtconv_desc* d, const void* x, const void* dy,
                             const float* w0, const float* b0, const float* s0, const float* wl, const float* sl,
                             float* dw0, float* db0, float* ds0, float* dwl, float* dsl, float* part, int* status,
                             cudaStream_t st, int max_groups) {
-  if (io == WTCONV_F32)
-    return launch_bwdw_t<K, float>(P, dev, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, part, status, st,
-                                   max_groups);
-  return launch_bwdw_t<K, __nv_bfloat16>(P, dev, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, part, status,
-                                         st, max_groups);
+  auto kern = wtconv_bwdw_kernel<K, LC, IO>;
+  const size_t smem = (size_t)B.smem_floats * 4;
+  int occ = 0;
+  wtconv_status e = prepare(kern, smem, occ, BW_NT);
+  if (e != WTCONV_OK) return e;
+  // planes per CTA: fewest sequential units per CTA slot (waves x units per
+  // CTA), ties broken towards longer CTAs (fewer partial sums)
+  const int slots = dev.sms * occ;
+  long best = -1;
+  for (int ppc = B.PB; ppc < B.N + B.PB; ppc += B.PB) {
+    const int p = std::min(ppc, B.N);
+    const int groups = (B.N + p - 1) / p;
+    if (groups > max_groups) continue;
+    const long ctas = (long)B.C * groups;
+    const long cost = ((ctas + slots - 1) / slots) * ((p + B.PB - 1) / B.PB);
+    if (best < 0 || cost <= best) {
+      best = cost;
+      B.ppc = p;
+    }
+    if (p == B.N) break;
+  }
+  if (best < 0) return WTCONV_ERR_SCRATCH_LIMIT;
+  B.ngroups = (B.N + B.ppc - 1) / B.ppc;
+  kern<<<B.C * B.ngroups, BW_NT, smem, st>>>(B, static_cast<const IO*>(x), static_cast<const IO*>(dy), part, status);
+  if (cudaGetLastError() != cudaSuccess) return WTCONV_ERR_CUDA;
+  return launch_finalize<K>(d, B.ngroups, part, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, st);
 }
 
-// Runs the weight-gradient kernels with the per-CTA partial sums at `part`
-// and at most `max_groups` CTAs per channel (the partials then fill
-// max_groups * C * V floats).
+template <int K>
+wtconv_status launch_bwdw_k(BwPlan& B, const Device& dev, const wtconv_desc* d, const void* x, const void* dy,
+                            const float* w0, const float* b0, const float* s0, const float* wl, const float* sl,
+                            float* dw0, float* db0, float* ds0, float* dwl, float* dsl, float* part, int* status,
+                            cudaStream_t st, int max_groups) {
+#define WT_BW(LC, IO) \
+  launch_bwdw_t<K, LC, IO>(B, dev, d, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, part, status, st, max_groups)
+  const int lc = d->L >= 2 ? 2 : d->L;
+  if (d->io == WTCONV_F32) return lc == 2 ? WT_BW(2, float) : lc == 1 ? WT_BW(1, float) : WT_BW(0, float);
+  return lc == 2 ? WT_BW(2, __nv_bfloat16) : lc == 1 ? WT_BW(1, __nv_bfloat16) : WT_BW(0, __nv_bfloat16);
+#undef WT_BW
+}
+
+// Runs the whole-plane weight-gradient kernels with the per-CTA partial sums
+// at `part` and at most `max_groups` CTAs per channel (the partials then
+// fill max_groups * C * V floats).
 wtconv_status run_bwdw_part(const wtconv_desc* d, const void* x, const void* dy, const float* w0, const float* b0,
                             const float* s0, const float* wl, const float* sl, float* dw0, float* db0, float* ds0,
                             float* dwl, float* dsl, float* part, int* status, int max_groups, cudaStream_t st) {
@@ -764,21 +783,20 @@ wtconv_status run_bwdw_part(const wtconv_desc* d, const void* x, const void* dy,
   wtconv_status e = query_device(dev);
   if (e != WTCONV_OK) return e;
   if (dev.max_smem < PLAN_SMEM) return WTCONV_ERR_UNSUPPORTED;
-  Plan P;
-  build_bwdw_plan(P, d, dev.max_smem);
-  if ((size_t)P.smem_floats * 4 > (size_t)dev.max_smem) return WTCONV_ERR_UNSUPPORTED;
+  BwPlan B;
+  if (!build_bw_plan(B, d, dev.max_smem)) return WTCONV_ERR_UNSUPPORTED;
   switch (d->k) {
     case 1:
-      return launch_bwdw_k<1>(P, dev, d->io, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, part, status, st,
+      return launch_bwdw_k<1>(B, dev, d, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, part, status, st,
                               max_groups);
     case 3:
-      return launch_bwdw_k<3>(P, dev, d->io, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, part, status, st,
+      return launch_bwdw_k<3>(B, dev, d, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, part, status, st,
                               max_groups);
     case 5:
-      return launch_bwdw_k<5>(P, dev, d->io, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, part, status, st,
+      return launch_bwdw_k<5>(B, dev, d, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, part, status, st,
                               max_groups);
     default:
-      return launch_bwdw_k<7>(P, dev, d->io, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, part, status, st,
+      return launch_bwdw_k<7>(B, dev, d, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, part, status, st,
                               max_groups);
   }
 }
@@ -827,16 +845,7 @@ wtconv_status run_band_k(const wtconv_desc* d, const void* x, const void* dy, co
     prevx = llx;
     prevd = lld;
   }
-  Plan P;
-  fill_common(P, d);
-  P.ngroups = groups;
-  const size_t fsmem = (size_t)P.V * sizeof(float);
-  auto fin = wtconv_bwdw_finalize<K>;
-  if (fsmem > 48 * 1024 &&
-      cudaFuncSetAttribute(fin, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fsmem) != cudaSuccess)
-    return WTCONV_ERR_CUDA;
-  fin<<<P.C, 128, fsmem, st>>>(P, part, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl);
-  return cudaGetLastError() == cudaSuccess ? WTCONV_OK : WTCONV_ERR_CUDA;
+  return launch_finalize<K>(d, groups, part, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, st);
 }
 
 wtconv_status run_band(const wtconv_desc* d, const void* x, const void* dy, const float* w0, const float* b0,
@@ -1034,6 +1043,25 @@ wtconv_status wtconv_backward_weight_noalloc(const wtconv_desc* desc, const void
   if (G == 0) return WTCONV_ERR_UNSUPPORTED;
   float* ll = reinterpret_cast<float*>(static_cast<char*>(scratch) + WS_HEADER + band_part_bytes(desc, G));
   return run_band(desc, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, part, ll, G, st);
+}
+
+int wtconv_kernel_launches(const wtconv_desc* desc, int op) {
+  if (check_desc(desc) != WTCONV_OK) return 0;
+  MainPlan M;
+  const bool main_ok = build_main_plan(M, desc, PLAN_SMEM);
+  const int data = main_ok ? 2 + ((desc->L >= 2 && !M.fused) ? 1 : 0) : 0;  // fold, [deep], output
+  const int weight = bwdw_whole_plane(desc) ? 2 : (desc->L == 0 ? 1 : desc->L) + 1;  // kernel(s), finalize
+  switch (op) {
+    case WTCONV_OP_FORWARD:
+    case WTCONV_OP_BACKWARD_DATA:
+      return data;
+    case WTCONV_OP_BACKWARD_WEIGHT:
+      return weight;
+    case WTCONV_OP_BACKWARD:
+      return data + weight;
+    default:
+      return 0;
+  }
 }
 
 const char* wtconv_status_string(wtconv_status s) {

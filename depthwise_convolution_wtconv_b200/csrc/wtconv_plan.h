@@ -1,9 +1,7 @@
-// Shared-memory plan of the per-plane WTConv kernels.
-//
-// One CTA owns one (n, c) image plane at a time and keeps the whole plane,
-// its level-1 Haar subbands and the deeper pyramid in shared memory, so the
-// subbands never travel through HBM (reformulation (1) of arXiv:2608.10805,
-// abstract).  The host fills a Plan and passes it by value to the kernel.
+// Shared-memory plans of the WTConv kernels (the host fills one per launch
+// and passes it by value).  The kernels keep each plane's Haar subbands in
+// shared memory, so they never travel through HBM (reformulation (1) of
+// arXiv:2608.10805, abstract).
 //
 // Buffer conventions (all offsets and leading dimensions in floats):
 //  * "shifted" buffers (read at x0-r by the register tiles) store element
@@ -18,16 +16,13 @@
 
 namespace wt {
 
-constexpr int NT = 256;           // threads per CTA
+constexpr int NT = 256;           // threads per CTA of the row-band weight-gradient kernel
 constexpr int MAXL = WTCONV_MAX_LEVELS;
 
 // register-tile shapes (rows x cols of outputs per thread)
-constexpr int C3_CW = 8;          // base conv + synthesis, full resolution
-constexpr int C2_R = 4, C2_CW = 4;  // level-1 band conv, half resolution
-constexpr int DP_R = 2, DP_CW = 4;  // deep levels
-constexpr int BW_R = 4, BW_CW = 8;  // weight-gradient correlation, full resolution
-constexpr int B1_R = 4, B1_CW = 4;  // weight-gradient correlation, level 1
-constexpr int DSLOTS = 8;           // threads per deep (level, band) in the correlation pass
+constexpr int DP_R = 2, DP_CW = 4;  // deep-level kernel
+constexpr int BW_R = 4, BW_CW = 8;  // row-band weight gradients, full resolution
+constexpr int B1_R = 4, B1_CW = 4;  // row-band weight gradients, level grid
 
 // Division by a runtime divisor d >= 1 without an integer divide:
 // x / d == umulhi(x, m) >> s for 0 <= x < 2^31 (m, s set on the host).
@@ -51,52 +46,6 @@ struct BufDesc {
   int ps;              // stride between the copies of consecutive planes of a batch
 };
 
-struct Plan {
-  int N, C, H, W, K, r, L;
-  int H1, W1;
-  int R3;              // rows of the full-resolution register tile (2 or 4)
-  int kk4;             // K*K rounded up to 4
-  int vec_in, vec_out; // global rows allow 16-byte vector access
-  int prefetch_ok;     // plane bytes are a multiple of 16 (TMA bulk copies allowed)
-  int use_bulk;        // stage through TMA bulk copies into the raw buffer(s)
-  int raw_off, rawg_off;  // raw copies of x (and dy) of one batch, I/O dtype
-  int nthreads;        // threads per CTA of the forward kernel
-  int io_bytes;        // bytes per element of x, y, dy, dx
-  // weights (folded): w0 [kk4], b0 [4], wl[l][s] [kk4] for l = 1..L
-  int w_off;
-  BufDesc xf;          // shifted: input plane (fp32)
-  BufDesc s1;          // shifted: 4 bands of level-1 subbands
-  BufDesc zb;          // plain: 4 bands of folded level-1 conv outputs
-  BufDesc t1;          // plain: deep synthesis at level-1 resolution
-  int deep_off, deep_floats;   // region re-zeroed before every deep pass
-  BufDesc sd[MAXL + 1];        // shifted: level-l subbands (l >= 2), 4 bands
-  BufDesc zd[MAXL + 1];        // plain: folded level-l conv outputs (l >= 3)
-  BufDesc t2;                  // plain: deep synthesis at level-2 resolution
-  // weight-gradient kernel only
-  BufDesc gf;          // plain: dy plane (fp32)
-  BufDesc g1;          // plain: 4 bands of dy level-1 subbands
-  BufDesc gd[MAXL + 1];        // plain: dy level-l subbands (l >= 2)
-  int red_off;         // per-thread partial sums for the final reduction
-  int gdeep_off;       // deep-level accumulators [L-1][4][kk4]
-  int dpart_off;       // deep-level per-slot partials [L-1][4][DSLOTS][kk4]
-  // item decompositions of the forward phases (divisors per plane)
-  FDiv f_stage_per, f_stage_x;   // staging items per plane, per block row
-  FDiv f_deep_per;               // deep conv items per plane
-  FDiv f_t1_per, f_t1_x;         // t1 items per plane, per row
-  FDiv f_out_per, f_out_x;       // output tiles per plane, per tile row
-  FDiv f_bw_per, f_bw_x;         // weight-gradient base tiles per plane, per row
-  FDiv f_b1_per, f_b1_x;         // weight-gradient level-1 tiles per band, per row
-  FDiv f_l_tiles[MAXL + 1];      // deep conv tiles per band of level l
-  FDiv f_l_tx[MAXL + 1];         // deep conv tiles per tile row of level l
-  int deep_items;                // deep conv items per plane (levels 2..L)
-  int deep_first[MAXL + 2];      // first item of level l within a plane
-  int PB;              // planes of one channel processed together (a batch)
-  int nbatch;          // batches per channel: ceil(N / PB)
-  int planes_per_cta;  // weight-gradient kernel: consecutive n per CTA
-  int ngroups;         // weight-gradient kernel: CTAs per channel
-  int V;               // partial-sum entries per CTA: K*K*(1+4L) + 1
-  int smem_floats;
-};
 
 }  // namespace wt
 
@@ -168,6 +117,39 @@ struct BandPlan {
   int smem_floats;
   int vec, write_ll, seg;
   FDiv f_nb, f_bx, f_bper, f_sx, f_sper;
+};
+
+// One correlation branch of the whole-plane weight-gradient kernel: the
+// base taps (branch 0) or band s of level l (branch 1 + 4(l-1) + s).  Its
+// 4x4 tiles correlate the shifted operand a (x side, read at x0 - r) with the
+// plain operand g (dy side); the sums go to entries [seg, seg + K*K) of the
+// partial vector.  Threads [first, first + nthr) own the branch.
+struct BwBranch {
+  int a_off, a_ld, g_off, g_ld;  // band 0 of plane 0 of the slot; band offsets are added per branch
+  int first, nthr, seg;
+  FDiv f_tiles, f_tx;            // 4x4 tiles per plane, per tile row
+};
+
+// Plan of the whole-plane weight-gradient kernel: a CTA of BW_NT threads
+// owns channel c and planes [g*ppc, (g+1)*ppc) of it, PB planes per unit.
+// The slot holds the raw copies (bulk copies of the next unit) of x and dy,
+// and per plane: xf / gf (x padded, dy plain), the level-1 subbands of both
+// (s1x shifted, g1 plain) and, for l >= 2, sd[l] / gd[l].
+constexpr int BW_NT = 256;
+constexpr int BW_MAXB = 1 + 4 * MAXL;
+struct BwPlan {
+  int N, C, H, W, K, r, L, H1, W1, kk4, V, io_bytes, vec_in;
+  int PB, ppc, ngroups, units;     // planes per unit, planes per CTA, CTAs per channel
+  int bulk;                        // whole planes by bulk copies (plane bytes % 16 == 0)
+  int raw_x, raw_g, raw_pp;        // raw copies of one unit (floats; per-plane stride)
+  int ps;                          // per-plane slab stride (floats)
+  BufDesc xf, gf, s1, g1, sd[MAXL + 1], gd[MAXL + 1];
+  int BH;                          // staging block rows: 4 (L >= 2), 2 (L = 1), 1 (L = 0)
+  FDiv f_spp, f_sx;                // staging blocks per plane, per block row
+  int nbr;                         // branches: 1 + 4L
+  BwBranch br[BW_MAXB];
+  int red_off;                     // final reduction: BW_NT * kk4 + BW_NT floats (over the slab)
+  int smem_floats;
 };
 
 }  // namespace wt

@@ -187,6 +187,13 @@ wtconv_status wtconv_backward_weight_noalloc(const wtconv_desc* desc,
                                              float* db0, float* ds0, float* dwl,
                                              float* dsl, void* stream);
 
+/* Number of kernel launches one call of operation `op` makes for `desc`
+ * (the plan the library picks for the shape on sm_100a), so that a caller
+ * can count the kernels in a timed region or a captured graph; 0 when desc
+ * is invalid or op unknown.  No counterpart in the paper: an introspection
+ * helper of this library. */
+int wtconv_kernel_launches(const wtconv_desc* desc, int op);
+
 /* Static description of a status code (never NULL). */
 const char* wtconv_status_string(wtconv_status status);
 

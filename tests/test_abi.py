@@ -25,7 +25,7 @@ def lib():
 
 def declared_functions():
     text = open(HEADER).read()
-    return sorted(set(re.findall(r"^\s*(?:const char\*|size_t|wtconv_status)\s+(wtconv_\w+)\s*\(", text, re.M)))
+    return sorted(set(re.findall(r"^\s*(?:const char\*|size_t|int|wtconv_status)\s+(wtconv_\w+)\s*\(", text, re.M)))
 
 
 def test_header_declares_the_binding_exports():
@@ -75,6 +75,19 @@ def test_workspace_of_the_row_band_weight_gradient_path(lib):
     assert part % (C * V * 4) == 0
     assert 1 <= part // (C * V * 4) < N
     assert lib.wtconv_workspace_size(ctypes.byref(d), 3) == max(ws, lib.wtconv_workspace_size(ctypes.byref(d), 0))
+
+
+def test_kernel_launch_counts(lib):
+    """Whole 56x56 planes with L = 3: fold + output kernel per data pass, the
+    weight-gradient kernel + finalize; 256x256 planes with L = 5 run as row
+    bands: fold + deep + output kernel, and one launch per level + finalize."""
+    n = lambda d, op: lib.wtconv_kernel_launches(ctypes.byref(d), op)
+    whole = _lib.WTConvDesc(32, 96, 56, 56, 5, 3, 0)
+    assert [n(whole, op) for op in range(4)] == [2, 2, 2, 4]
+    bands = _lib.WTConvDesc(16, 64, 256, 256, 5, 5, 1)
+    assert [n(bands, op) for op in range(4)] == [3, 3, 6, 9]
+    assert n(_lib.WTConvDesc(2, 3, 16, 16, 4, 2, 0), 0) == 0
+    assert n(whole, 7) == 0
 
 
 def _fwd(lib, d, x=FAKE, y=FAKE, w0=FAKE, b0=FAKE, s0=FAKE, wl=FAKE, sl=FAKE, ws=FAKE, nws=1 << 30):
