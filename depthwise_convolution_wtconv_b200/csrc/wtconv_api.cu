@@ -406,19 +406,20 @@ wtconv_status launch_forward_t(const wtconv_desc* d, const Device& dev, const vo
   }
   const size_t smem = (size_t)M.smem_floats * 4;
   int occ = 0;
-  if (M.R3 == 8) {
-    auto km = wtconv_main_kernel<K, 8, IO>;
-    wtconv_status e = prepare(km, smem, occ, MAIN_NT);
-    if (e != WTCONV_OK) return e;
-    km<<<std::min(M.units, dev.sms * occ), MAIN_NT, smem, st>>>(M, static_cast<const IO*>(x), t1, wfold,
-                                                                static_cast<IO*>(y), status);
-  } else {
-    auto km = wtconv_main_kernel<K, 4, IO>;
-    wtconv_status e = prepare(km, smem, occ, MAIN_NT);
-    if (e != WTCONV_OK) return e;
-    km<<<std::min(M.units, dev.sms * occ), MAIN_NT, smem, st>>>(M, static_cast<const IO*>(x), t1, wfold,
-                                                                static_cast<IO*>(y), status);
+#define WT_MAIN(R3, FUSED)                                                                              \
+  {                                                                                                     \
+    auto km = wtconv_main_kernel<K, R3, IO, FUSED>;                                                     \
+    wtconv_status e = prepare(km, smem, occ, MAIN_NT);                                                  \
+    if (e != WTCONV_OK) return e;                                                                       \
+    km<<<std::min(M.units, dev.sms * occ), MAIN_NT, smem, st>>>(M, static_cast<const IO*>(x), t1, wfold, \
+                                                                static_cast<IO*>(y), status);           \
   }
+  if (M.fused) {
+    if (M.R3 == 8) WT_MAIN(8, true) else WT_MAIN(4, true)
+  } else {
+    if (M.R3 == 8) WT_MAIN(8, false) else WT_MAIN(4, false)
+  }
+#undef WT_MAIN
   return cudaGetLastError() == cudaSuccess ? WTCONV_OK : WTCONV_ERR_CUDA;
 }
 
@@ -560,7 +561,8 @@ void bw_branches(BwPlan& B) {
 }
 
 // Whole-plane plan: the most planes per unit (up to two tiles per thread)
-// that fit two CTAs per SM, else one.  False when one plane does not fit.
+// that fit two CTAs per SM, else one.  False when one plane does not fit;
+// such shapes run on the row-band path.
 bool build_bw_plan(BwPlan& B, const wtconv_desc* d, int max_smem) {
   B = BwPlan{};
   B.N = d->N;
@@ -581,11 +583,13 @@ bool build_bw_plan(BwPlan& B, const wtconv_desc* d, int max_smem) {
   for (int l = 1; l <= d->L; ++l) per_plane += 4 * cdiv_h(d->H >> l, 4) * cdiv_h(d->W >> l, 4);
   const int pb0 = std::max(1, std::min(d->N, cdiv_h(2 * BW_NT, per_plane)));
   bool ok = false;
+  // two CTAs per SM if possible; else one (still faster than row bands,
+  // which stage halo rows twice and hand the LL planes through HBM)
   for (const int budget : {(int)(SM_SMEM / 2 - 1024), max_smem}) {
     for (int pb = pb0; pb >= 1 && !ok; --pb) ok = bw_layout(B, pb, std::min(budget, max_smem));
     if (ok) break;
   }
-  if (!ok) return false;
+  if (!ok) return false;  // the row-band path takes the shape
   B.f_sx = make_fdiv(cdiv_h(d->W, 4));
   B.f_spp = make_fdiv((d->H / B.BH) * cdiv_h(d->W, 4));
   bw_branches(B);

@@ -302,7 +302,7 @@ __device__ __forceinline__ void main_add_t1(const MainPlan& P, const float* slot
 // Phase A, one tile: band s of plane j, a 4x4 tile of the level-1 grid:
 // the band conv with folded weights (reformulation (3) of arXiv:2608.10805,
 // abstract), t1 added to the LL band, stored to the band's Z plane.
-template <int K>
+template <int K, bool FUSED>
 __device__ __forceinline__ void main_band_tile(const MainPlan& P, float* slot, int it) {
   const int j = P.f_app.div(it);
   int rem = it - j * P.a_pp;
@@ -317,8 +317,8 @@ __device__ __forceinline__ void main_band_tile(const MainPlan& P, float* slot, i
     for (int b = 0; b < 4; ++b) z[a][b] = 0.f;
   const float* s1 = slot + P.s1.off + j * P.s1.ps + s * P.s1.ld * P.s1.rows + i0 * P.s1.ld + j0;
   conv_tile<K, 4, 4>(s1, P.s1.ld, slot + P.w_off + P.kk4 + 4 + s * P.kk4, z);
-  if (s == 0 && P.fused) {
-    main_add_t1(P, slot, j, i0, j0, z);
+  if constexpr (FUSED) {
+    if (s == 0) main_add_t1(P, slot, j, i0, j0, z);
   } else if (s == 0 && P.L >= 2) {
     const float* t1 = slot + P.t1.off + j * P.t1.ps + i0 * P.t1.ld + j0;
 #pragma unroll
@@ -422,7 +422,7 @@ __device__ __forceinline__ void main_issue(const MainPlan& P, float* slot, uint6
   }
 }
 
-template <int K, int R3, typename IO>
+template <int K, int R3, typename IO, bool FUSED>
 __global__ void __launch_bounds__(MAIN_NT, 4)
     wtconv_main_kernel(const MainPlan P, const IO* __restrict__ x, const float* __restrict__ t1g,
                        const float* __restrict__ wfold, IO* __restrict__ y, int* __restrict__ status) {
@@ -446,8 +446,8 @@ __global__ void __launch_bounds__(MAIN_NT, 4)
     const UnitGeo g = unit_geo(P, blockIdx.x + k * gridDim.x);
     // every thread waits on every phase in order, so a parity wait is exact
     mb_wait(full, k & 1, abort_flag);
-    const int n = P.fused ? 0 : g.npb * P.stage_pp;
-    if (P.fused) {
+    const int n = FUSED ? 0 : g.npb * P.stage_pp;
+    if constexpr (FUSED) {
       const int nb = g.npb * P.f_bpp.d;
       for (int it = tid; it < nb; it += MAIN_NT) {
         const int j = P.f_bpp.div(it);
@@ -478,7 +478,7 @@ __global__ void __launch_bounds__(MAIN_NT, 4)
     // unit's copies overwrite while this unit computes
     for (int i = tid; i < (P.wblk >> 2); i += MAIN_NT)
       reinterpret_cast<float4*>(slot + P.w_off)[i] = reinterpret_cast<const float4*>(slot + P.wraw_off)[i];
-    if (P.L >= 2 && !P.fused) {
+    if (!FUSED && P.L >= 2) {
       const int rows = P.TH >> 1, q4 = (P.W1 + 3) >> 2;
       for (int it = tid; it < g.npb * rows * q4; it += MAIN_NT) {
         const int j = it / (rows * q4), rem = it - j * rows * q4;
@@ -497,7 +497,7 @@ __global__ void __launch_bounds__(MAIN_NT, 4)
     if (*abort_flag) break;  // uniform: read after the barrier
     if (tid == 0 && k + 1 < myunits)
       main_issue<IO>(P, slot, full, unit_geo(P, blockIdx.x + (k + 1) * gridDim.x), x, t1g, wfold);
-    if (P.fused) {
+    if constexpr (FUSED) {
       // levels 3..L of the pyramid, then every deep level's band convs
       for (int l = 3; l <= P.L; ++l) {
         const BufDesc& sb = P.sd[l - 1];
@@ -512,7 +512,7 @@ __global__ void __launch_bounds__(MAIN_NT, 4)
     }
     if (P.L >= 1) {
       const int na = g.npb * P.a_pp;
-      for (int it = tid; it < na; it += MAIN_NT) main_band_tile<K>(P, slot, it);
+      for (int it = tid; it < na; it += MAIN_NT) main_band_tile<K, FUSED>(P, slot, it);
       __syncthreads();
     }
     for (int it = tid; it < P.tiles; it += MAIN_NT) {
