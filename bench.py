@@ -320,7 +320,17 @@ def run_ours(args, wl, world, rank, local):
     kernels = {"fwd": t_fwd, "bwd_data": t_bd, "bwd_weight": t_bw}
     dom = max(kernels, key=kernels.get)
     dom_ms = kernels[dom]
-    achieved_tflops = 2 * counts[dom]["fma"] / (dom_ms * 1e-3) / 1e12
+    # the bound of the pass: FP32 ALUs or HBM, whichever needs more time
+    t_alu = 2 * counts[dom]["fma"] / (fp32_peak_tflops * 1e12)
+    t_hbm = counts[dom]["bytes"] / (hbm_peak * 1e9)
+    if t_hbm > t_alu:
+        bound, unit, peak = "hbm", "GB/s", hbm_peak
+        achieved = counts[dom]["bytes"] / (dom_ms * 1e-3) / 1e9
+        peak_source = f"{peak_src} copy bandwidth"
+    else:
+        bound, unit, peak = "alu", "TFLOP/s", fp32_peak_tflops
+        achieved = 2 * counts[dom]["fma"] / (dom_ms * 1e-3) / 1e12
+        peak_source = f"{sms} SMs x {FP32_LANES_PER_SM} FP32 lanes x 2 x {sm_max:.0f} MHz"
     step_bytes = sum(c["bytes"] for c in counts.values())
     hbm_gbs = step_bytes / (ms_per_step * 1e-3) / 1e9
     traffic = load_traffic(dom, wl.name)
@@ -340,10 +350,9 @@ def run_ours(args, wl, world, rank, local):
         "config": {"workload": wl.name, **{k: v for k, v in wl.as_dict().items() if k != "name"},
                    "global_batch": wl.N * world, "parallelism": f"dp{world}",
                    "l2": "flushed before every timed step (256 MiB write)"},
-        "roofline": {"bound": "alu", "kernel": f"{dom} pass: {PASS_KERNELS[dom]}", "achieved": achieved_tflops,
-                     "peak": fp32_peak_tflops, "unit": "TFLOP/s", "frac": achieved_tflops / fp32_peak_tflops,
-                     "traffic": traffic,
-                     "peak_source": f"{sms} SMs x {FP32_LANES_PER_SM} FP32 lanes x 2 x {sm_max:.0f} MHz"},
+        "roofline": {"bound": bound, "kernel": f"{dom} pass: {PASS_KERNELS[dom]}", "achieved": achieved,
+                     "peak": peak, "unit": unit, "frac": achieved / peak, "traffic": traffic,
+                     "peak_source": peak_source},
         "hbm": {"achieved_gbs": hbm_gbs, "peak_gbs": hbm_peak, "frac": hbm_gbs / hbm_peak,
                 "algorithmic_bytes_per_step": step_bytes, "peak_source": peak_src},
         "kernels_ms": kernels,
@@ -357,6 +366,9 @@ def run_ours(args, wl, world, rank, local):
         "clocks": clocks,
         "wall_s_timed_region": t_wall,
     }
+    if rank == 0 and not args.no_comparators:
+        extra = (Y.numel() + dX.numel()) * Y.element_size() + gflat.numel() * 4 + ws.numel()
+        line["comparators"] = comparators(wl, device, inp, lambda: step(), extra)
     if rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl, args.cpu_sample_n)
     return line
@@ -368,6 +380,102 @@ def sources_sha256():
     import hashlib
     paths = sorted(glob.glob(os.path.join(ROOT, "depthwise_convolution_wtconv_b200", "csrc", "*")))
     return hashlib.sha256(b"".join(open(p, "rb").read() for p in paths)).hexdigest()
+
+
+def torch_cascade(X, W0, b0, s0, Wl, sl):
+    """The layer composed from plain PyTorch GPU ops, written here as a
+    comparator (the unfused cascade, as a framework user would write it):
+    grouped conv2d for the depthwise convs, a stride-2 grouped conv2d with
+    the +-1/2 Haar taps for the analysis, conv_transpose2d for the synthesis;
+    autograd for the backward.  Every subband, Z and LL tensor goes through
+    HBM and is kept for the backward."""
+    import torch.nn.functional as F
+    C, k = X.shape[1], W0.shape[-1]
+    L = 0 if Wl is None else Wl.shape[0]
+    h = 0.5
+    filt = torch.tensor([[[h, h], [h, h]], [[h, h], [-h, -h]], [[h, -h], [h, -h]], [[h, -h], [-h, h]]],
+                        dtype=X.dtype, device=X.device).repeat(C, 1, 1).unsqueeze(1)
+    Y = s0.view(1, C, 1, 1) * F.conv2d(X, W0.unsqueeze(1), b0, padding=k // 2, groups=C)
+    cur, Zs = X, []
+    for lv in range(L):
+        sub = F.conv2d(cur, filt, stride=2, groups=C)
+        Zs.append(F.conv2d(sub, Wl[lv].reshape(4 * C, 1, k, k), padding=k // 2, groups=4 * C)
+                  * sl[lv].reshape(1, 4 * C, 1, 1))
+        cur = sub[:, 0::4]
+    t = None
+    for lv in reversed(range(L)):
+        Z = Zs[lv]
+        if t is not None:
+            Z = torch.cat([(Z[:, 0::4] + t).unsqueeze(2), Z.view(Z.shape[0], C, 4, *Z.shape[2:])[:, :, 1:]],
+                          dim=2).view_as(Z)
+        t = F.conv_transpose2d(Z, filt, stride=2, groups=C)
+    return Y if t is None else Y + t
+
+
+def comparators(wl, device, inp, ours_step, ours_extra_bytes, steps=20):
+    """Same-GPU comparators of one fwd+bwd step (not part of the timed
+    metric): the plain PyTorch cascade (time and peak memory beyond the
+    inputs), and for L = 0 a diagonalwise-refactorized conv (channels in
+    blocks of 32, each block one dense conv with a block-diagonal weight, as
+    in "Diagonalwise Refactorization: An Efficient Training Method for
+    Depthwise Convolutions").  fp32 arithmetic on fp32 copies of the inputs."""
+    import torch.nn.functional as F
+    X = inp["X"].float().to(device).requires_grad_(True)
+    dY = inp["dY"].float().to(device)
+    P = {kk: inp[kk].to(device).requires_grad_(True) for kk in ("W0", "b0", "s0")}
+    Wl = inp["Wl"].to(device).requires_grad_(True) if wl.L else None
+    sl = inp["sl"].to(device).requires_grad_(True) if wl.L else None
+    leaves = [X, P["W0"], P["b0"], P["s0"]] + ([Wl, sl] if wl.L else [])
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize(device)
+        base = torch.cuda.memory_allocated(device)
+        torch.cuda.reset_peak_memory_stats(device)
+        fn()
+        torch.cuda.synchronize(device)
+        peak = torch.cuda.max_memory_allocated(device) - base
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(steps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize(device)
+        return e0.elapsed_time(e1) / steps, peak
+
+    def cascade_step():
+        for t in leaves:
+            t.grad = None
+        Y = torch_cascade(X, P["W0"], P["b0"], P["s0"], Wl, sl)
+        Y.backward(dY)
+
+    out = {}
+    ms, peak = timed(cascade_step)
+    ours_ms, _ = timed(ours_step)
+    out["torch_cascade"] = {"ms_per_step": ms, "peak_extra_bytes": peak,
+                            "what": "plain PyTorch ops (grouped conv2d, Haar as stride-2 conv, conv_transpose2d) "
+                                    "+ autograd, fp32"}
+    out["ours_eager_ms_per_step"] = ours_ms
+    out["ours_extra_bytes"] = ours_extra_bytes
+    out["speedup_vs_torch_cascade"] = ms / ours_ms
+    out["memory_ratio_vs_torch_cascade"] = peak / max(1, ours_extra_bytes)
+    if wl.L == 0:
+        G = min(32, wl.C)
+        groups = wl.C // G
+        k = wl.k
+        eye = torch.eye(G, device=device).view(1, G, G, 1, 1)
+
+        def diag_step():
+            for t in leaves:
+                t.grad = None
+            w = (P["W0"].view(groups, G, 1, k, k) * eye).reshape(wl.C, G, k, k)
+            Y = P["s0"].view(1, -1, 1, 1) * F.conv2d(X, w, P["b0"], padding=k // 2, groups=groups)
+            Y.backward(dY)
+
+        dms, dpeak = timed(diag_step)
+        out["diagonalwise_refactorization"] = {"ms_per_step": dms, "peak_extra_bytes": dpeak, "block": G}
+    return out
 
 
 def load_traffic(kernel, workload):
@@ -467,6 +575,7 @@ def main(argv=None):
     ap.add_argument("--cpu-sample-n", type=int, default=32)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--eager", action="store_true", help="time eager library calls instead of CUDA graph replays")
+    ap.add_argument("--no-comparators", action="store_true", help="skip the same-GPU PyTorch comparators")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
