@@ -99,6 +99,10 @@ EDGE = [
     Workload("band_L1_bf16", 1, 2, 192, 160, 5, 1, "bf16"),
     Workload("band_L3_k7", 2, 2, 256, 128, 7, 3, "f32"),
     Workload("band_ragged_L2", 1, 2, 200, 180, 3, 2, "f32"),
+    # level-0 weight gradients in row bands: rows not 16-byte multiples (no
+    # bulk copies), and bf16
+    Workload("band_L0_nobulk", 1, 2, 150, 146, 5, 0, "f32"),
+    Workload("band_L0_bf16", 2, 2, 160, 132, 3, 0, "bf16"),
 ]
 
 
