@@ -741,8 +741,10 @@ wtconv_status launch_bwdw_t(BwPlan& B, const Device& dev, const wtconv_desc* d, 
   int occ = 0;
   wtconv_status e = prepare(kern, smem, occ, BW_NT);
   if (e != WTCONV_OK) return e;
-  // planes per CTA: fewest sequential units per CTA slot (waves x units per
-  // CTA), ties broken towards longer CTAs (fewer partial sums)
+  // planes per CTA: fewest sequential units per CTA slot, counting one more
+  // unit per CTA for its fixed costs (clearing its shared memory, the first
+  // copy that nothing overlaps, the final reduction and partial write); ties
+  // broken towards longer CTAs (fewer partial sums)
   const int slots = dev.sms * occ;
   long best = -1;
   for (int ppc = B.PB; ppc < B.N + B.PB; ppc += B.PB) {
@@ -750,7 +752,7 @@ wtconv_status launch_bwdw_t(BwPlan& B, const Device& dev, const wtconv_desc* d, 
     const int groups = (B.N + p - 1) / p;
     if (groups > max_groups) continue;
     const long ctas = (long)B.C * groups;
-    const long cost = ((ctas + slots - 1) / slots) * ((p + B.PB - 1) / B.PB);
+    const long cost = ((ctas + slots - 1) / slots) * ((p + B.PB - 1) / B.PB + 1);
     if (best < 0 || cost <= best) {
       best = cost;
       B.ppc = p;
