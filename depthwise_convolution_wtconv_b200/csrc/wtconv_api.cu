@@ -76,8 +76,9 @@ constexpr int SM_SMEM = 233472;  // shared memory per SM on sm_100a (228 KB)
 // four kernels per level (kk4 floats each).
 int main_wblk(const wtconv_desc* d) { return rup((1 + 4 * d->L) * rup(d->k * d->k, 4) + 4, 4); }
 
-// Output tile rows for band height TH: 8, unless 4 wastes fewer padded rows.
-int main_r3(int TH) { return rup(TH, 8) == rup(TH, 4) ? 8 : 4; }
+// Output tile rows for band height TH: 8, unless 4 wastes fewer padded rows
+// or the band is at most 8 rows (twice the tiles for the CTA's threads).
+int main_r3(int TH) { return TH > 8 && rup(TH, 8) == rup(TH, 4) ? 8 : 4; }
 
 // Slot layout for band height TH and PB planes per unit; returns the slot
 // size in floats.
@@ -625,7 +626,13 @@ void band_layout(BandPlan& B, int TB) {
   } else {
     B.s_ld = B.s_rows = B.d_ld = B.d_rows = 0;
   }
-  int cur = 0;
+  int cur = 4;  // header: mbarrier (8 bytes), abort flag
+  // raw copies of the next unit's rows (bulk copies), when rows are 16-byte aligned
+  B.bulk = ((size_t)B.W * B.in_bytes) % 16 == 0;
+  B.raw_a = cur;
+  cur += B.bulk ? rup((int)(((size_t)(B.FR + 2 * B.ha) * B.W * B.in_bytes + 3) / 4), 4) : 0;
+  B.raw_b = cur;
+  cur += B.bulk ? rup((int)(((size_t)B.FR * B.W * B.in_bytes + 3) / 4), 4) : 0;
   B.a_off = cur;
   cur += rup(B.a_ld * B.a_rows, 4);
   B.b_off = cur;
@@ -664,6 +671,7 @@ bool build_band_plan(BandPlan& B, const wtconv_desc* d, int lvl) {
   B.Hl = lvl == 0 ? B.H : B.H / 2;
   B.Wl = lvl == 0 ? B.W : B.W / 2;
   B.ha = lvl == 0 ? B.r : 2 * B.r;
+  B.in_bytes = lvl <= 1 ? io_bytes(d) : 4;
   B.vec = (B.W % 4) == 0;
   B.write_ll = lvl >= 1 && lvl < d->L;
   B.seg = lvl >= 1 ? d->k * d->k * (1 + 4 * (lvl - 1)) : 0;
@@ -809,13 +817,14 @@ wtconv_status run_bwdw_part(const wtconv_desc* d, const void* x, const void* dy,
 
 template <int K, typename IN>
 wtconv_status launch_band_level(const BandPlan& B, const void* a, const void* b, float* llx, float* lld, float* part,
-                                cudaStream_t st) {
+                                int* status, cudaStream_t st) {
   auto kern = wtconv_bwband_kernel<K, IN>;
   const size_t smem = (size_t)B.smem_floats * 4;
   int occ = 0;
   wtconv_status e = prepare(kern, smem, occ);
   if (e != WTCONV_OK) return e;
-  kern<<<B.C * B.ngroups, NT, smem, st>>>(B, static_cast<const IN*>(a), static_cast<const IN*>(b), llx, lld, part);
+  kern<<<B.C * B.ngroups, NT, smem, st>>>(B, static_cast<const IN*>(a), static_cast<const IN*>(b), llx, lld, part,
+                                          status);
   return cudaGetLastError() == cudaSuccess ? WTCONV_OK : WTCONV_ERR_CUDA;
 }
 
@@ -825,7 +834,8 @@ wtconv_status launch_band_level(const BandPlan& B, const void* a, const void* b,
 template <int K>
 wtconv_status run_band_k(const wtconv_desc* d, const void* x, const void* dy, const float* w0, const float* b0,
                          const float* s0, const float* wl, const float* sl, float* dw0, float* db0, float* ds0,
-                         float* dwl, float* dsl, float* part, float* ll, int groups, cudaStream_t st) {
+                         float* dwl, float* dsl, float* part, float* ll, int groups, int* status,
+                         cudaStream_t st) {
   const float* prevx = nullptr;
   const float* prevd = nullptr;
   size_t off = 0;
@@ -843,10 +853,10 @@ wtconv_status run_band_k(const wtconv_desc* d, const void* x, const void* dy, co
     }
     wtconv_status e;
     if (lvl <= 1)
-      e = d->io == WTCONV_F32 ? launch_band_level<K, float>(B, x, dy, llx, lld, part, st)
-                              : launch_band_level<K, __nv_bfloat16>(B, x, dy, llx, lld, part, st);
+      e = d->io == WTCONV_F32 ? launch_band_level<K, float>(B, x, dy, llx, lld, part, status, st)
+                              : launch_band_level<K, __nv_bfloat16>(B, x, dy, llx, lld, part, status, st);
     else
-      e = launch_band_level<K, float>(B, prevx, prevd, llx, lld, part, st);
+      e = launch_band_level<K, float>(B, prevx, prevd, llx, lld, part, status, st);
     if (e != WTCONV_OK) return e;
     prevx = llx;
     prevd = lld;
@@ -856,20 +866,21 @@ wtconv_status run_band_k(const wtconv_desc* d, const void* x, const void* dy, co
 
 wtconv_status run_band(const wtconv_desc* d, const void* x, const void* dy, const float* w0, const float* b0,
                        const float* s0, const float* wl, const float* sl, float* dw0, float* db0, float* ds0,
-                       float* dwl, float* dsl, float* part, float* ll, int groups, cudaStream_t st) {
+                       float* dwl, float* dsl, float* part, float* ll, int groups, int* status,
+                       cudaStream_t st) {
   Device dev;
   wtconv_status e = query_device(dev);
   if (e != WTCONV_OK) return e;
   if (dev.max_smem < PLAN_SMEM) return WTCONV_ERR_UNSUPPORTED;
   switch (d->k) {
     case 1:
-      return run_band_k<1>(d, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, part, ll, groups, st);
+      return run_band_k<1>(d, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, part, ll, groups, status, st);
     case 3:
-      return run_band_k<3>(d, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, part, ll, groups, st);
+      return run_band_k<3>(d, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, part, ll, groups, status, st);
     case 5:
-      return run_band_k<5>(d, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, part, ll, groups, st);
+      return run_band_k<5>(d, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, part, ll, groups, status, st);
     default:
-      return run_band_k<7>(d, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, part, ll, groups, st);
+      return run_band_k<7>(d, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, part, ll, groups, status, st);
   }
 }
 
@@ -885,7 +896,7 @@ wtconv_status run_bwdw(const wtconv_desc* d, const void* x, const void* dy, cons
   const int G = band_groups(d);
   if (G == 0) return WTCONV_ERR_UNSUPPORTED;
   float* ll = reinterpret_cast<float*>(static_cast<char*>(ws) + WS_HEADER + band_part_bytes(d, G));
-  return run_band(d, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, part, ll, G, st);
+  return run_band(d, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, part, ll, G, status, st);
 }
 
 wtconv_status check_ws(void* ws, size_t ws_bytes, size_t need) {
@@ -1048,7 +1059,7 @@ wtconv_status wtconv_backward_weight_noalloc(const wtconv_desc* desc, const void
   const int G = std::min<int>(band_groups(desc), (int)std::min<size_t>(groups, 1u << 20));
   if (G == 0) return WTCONV_ERR_UNSUPPORTED;
   float* ll = reinterpret_cast<float*>(static_cast<char*>(scratch) + WS_HEADER + band_part_bytes(desc, G));
-  return run_band(desc, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, part, ll, G, st);
+  return run_band(desc, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, part, ll, G, nullptr, st);
 }
 
 int wtconv_kernel_launches(const wtconv_desc* desc, int op) {

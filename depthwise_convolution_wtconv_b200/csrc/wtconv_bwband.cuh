@@ -25,7 +25,7 @@
 // launch uses the same G, so the fixed-order finalize applies unchanged.
 #pragma once
 
-#include "wtconv_kernels.cuh"
+#include "wtconv_main.cuh"
 
 namespace wt {
 
@@ -37,17 +37,24 @@ __device__ __forceinline__ float warp_sum(float v) {
 
 // Stages `rows` rows of a plane (row y0 first; rows outside [0, h) are
 // written as zeros) into shared memory at dst + i*ld + col0, converting to
-// fp32.  Returns this thread's sum of the staged in-image values when SUM.
-template <typename IN, bool SUM>
-__device__ __forceinline__ float stage_band_rows(const IN* __restrict__ src, int h, int w, int y0, int rows,
-                                                 float* __restrict__ dst, int ld, int col0, bool vec) {
+// fp32.  The rows come from the plane in global memory, or (SMEM) from a
+// raw copy in shared memory holding row i of the window at raw + i*w.
+// Returns this thread's sum of the staged in-image values when SUM.
+template <typename IN, bool SUM, bool SMEM>
+__device__ __forceinline__ float stage_band_rows(const IN* __restrict__ src, const IN* raw, int h, int w, int y0,
+                                                 int rows, float* __restrict__ dst, int ld, int col0, bool vec) {
   float sum = 0.f;
   const int q4 = (w + 3) >> 2;
   for (int it = threadIdx.x; it < rows * q4; it += NT) {
     const int i = it / q4, q = it - i * q4;
     const int y = y0 + i, x = 4 * q;
     float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (y >= 0 && y < h) v = load4(src + (size_t)y * w + x, x, w, vec);
+    if (y >= 0 && y < h) {
+      if constexpr (SMEM)
+        v = lds4(raw + (size_t)i * w + x, x, w, vec);
+      else
+        v = load4(src + (size_t)y * w + x, x, w, vec);
+    }
     float* o = dst + i * ld + col0 + x;
     o[0] = v.x;
     if (x + 1 < w) o[1] = v.y;
@@ -61,12 +68,20 @@ __device__ __forceinline__ float stage_band_rows(const IN* __restrict__ src, int
 template <int K, typename IN>
 __global__ void __launch_bounds__(NT, 2) wtconv_bwband_kernel(const BandPlan P, const IN* __restrict__ A,
                                                               const IN* __restrict__ B, float* __restrict__ llx,
-                                                              float* __restrict__ lld, float* __restrict__ part) {
+                                                              float* __restrict__ lld, float* __restrict__ part,
+                                                              int* __restrict__ status) {
   constexpr int KK = K * K;
   constexpr int r = K / 2;
   extern __shared__ float4 smem4[];
   float* sm = reinterpret_cast<float*>(smem4);
+  uint64_t* full = reinterpret_cast<uint64_t*>(sm);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + 2);
   for (int i = threadIdx.x; i < (P.smem_floats >> 2); i += NT) smem4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    mb_init(full, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
   __syncthreads();
   const int c = blockIdx.x % P.C, g = blockIdx.x / P.C;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -81,17 +96,52 @@ __global__ void __launch_bounds__(NT, 2) wtconv_bwband_kernel(const BandPlan P, 
   float G[KK];
   zero_taps<K>(G);
   float sumdy = 0.f;
-
-  for (int u = g; u < P.units; u += P.ngroups) {
+  const IN* rawa = reinterpret_cast<const IN*>(sm + P.raw_a);
+  const IN* rawb = reinterpret_cast<const IN*>(sm + P.raw_b);
+  // bulk copies of a unit's rows: the A rows of its window that lie in the
+  // image (at their row of the window) and its B rows
+  auto issue = [&](int u) {
+    const int n = P.f_nb.div(u), b = u - n * P.nb;
+    const int y0 = P.lvl == 0 ? b * P.TB : 2 * b * P.TB;
+    const int y_lo = max(0, y0 - P.ha), y_hi = min(P.H, y0 + P.FR + P.ha);
+    const unsigned ba = (unsigned)((y_hi - y_lo) * P.W * sizeof(IN));
+    const unsigned bbytes = (unsigned)(P.FR * P.W * sizeof(IN));
+    const size_t po = ((size_t)n * P.C + c) * plane;
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(full)), "r"(ba + bbytes)
+                 : "memory");
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(rawa + (size_t)(y_lo - (y0 - P.ha)) * P.W)),
+        "l"(A + po + (size_t)y_lo * P.W), "r"(ba), "r"(smem_u32(full))
+        : "memory");
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(rawb)),
+        "l"(B + po + (size_t)y0 * P.W), "r"(bbytes), "r"(smem_u32(full))
+        : "memory");
+  };
+  if (P.bulk && threadIdx.x == 0 && g < P.units) issue(g);
+  int k = 0;
+  for (int u = g; u < P.units; u += P.ngroups, ++k) {
     const int n = P.f_nb.div(u), b = u - n * P.nb;
     const int i0 = b * P.TB;                     // first row of the level grid
     const int y0 = P.lvl == 0 ? i0 : 2 * i0;     // first input row of the band
     const IN* a = A + ((size_t)n * P.C + c) * plane;
     const IN* bb = B + ((size_t)n * P.C + c) * plane;
-    stage_band_rows<IN, false>(a, P.H, P.W, y0 - P.ha, P.FR + 2 * P.ha, sa, P.a_ld, r, P.vec);
-    const float sdy = stage_band_rows<IN, true>(bb, P.H, P.W, y0, P.FR, sb, P.b_ld, 0, P.vec);
+    float sdy;
+    if (P.bulk) {
+      mb_wait(full, k & 1, abort_flag);
+      stage_band_rows<IN, false, true>(a, rawa, P.H, P.W, y0 - P.ha, P.FR + 2 * P.ha, sa, P.a_ld, r, P.vec);
+      sdy = stage_band_rows<IN, true, true>(bb, rawb, P.H, P.W, y0, P.FR, sb, P.b_ld, 0, P.vec);
+    } else {
+      stage_band_rows<IN, false, false>(a, nullptr, P.H, P.W, y0 - P.ha, P.FR + 2 * P.ha, sa, P.a_ld, r, P.vec);
+      sdy = stage_band_rows<IN, true, false>(bb, nullptr, P.H, P.W, y0, P.FR, sb, P.b_ld, 0, P.vec);
+    }
     if (P.lvl <= 1) sumdy += sdy;
     __syncthreads();
+    if (*abort_flag) break;  // uniform: read after the barrier
+    if (P.bulk && threadIdx.x == 0 && u + P.ngroups < P.units) issue(u + P.ngroups);
     if (P.lvl >= 1) {
       // subbands of x over TB + 2r level rows (the halo rows outside the
       // image come out zero from the zero rows staged above) and of dy over
@@ -147,6 +197,13 @@ __global__ void __launch_bounds__(NT, 2) wtconv_bwband_kernel(const BandPlan P, 
     __syncthreads();
   }
 
+  if (*abort_flag) {
+    if (threadIdx.x == 0) {
+      mb_drain(full, k & 1);  // the copies of unit k were issued; let them land before exit
+      if (status) atomicExch(status, 1);
+    }
+    return;
+  }
   // fixed-order reduction: shuffle tree within each warp, then warps in order
   float* red = sm + P.red_off;
 #pragma unroll

@@ -27,7 +27,7 @@ namespace wt {
 
 constexpr int MAIN_NT = 128;
 constexpr int MAIN_HEADER = 4;       // floats: mbarrier (8 bytes), abort flag
-constexpr int DEEP_NT = 128;
+constexpr int DEEP_NT = 256;
 
 // ------------------------------------------------------------ mbarriers
 __device__ __forceinline__ unsigned smem_u32(const void* p) { return (unsigned)__cvta_generic_to_shared(p); }

@@ -114,6 +114,8 @@ struct BandPlan {
   int s_off, s_ld, s_rows;
   int d_off, d_ld, d_rows;
   int red_off;               // (NT/32) * kk4 + NT/32 floats of the final reduction
+  int raw_a, raw_b;          // raw copies of the next unit's A window and B rows (bulk copies)
+  int in_bytes, bulk;        // bytes per input element; rows 16-byte aligned for bulk copies
   int smem_floats;
   int vec, write_ll, seg;
   FDiv f_nb, f_bx, f_bper, f_sx, f_sper;
