@@ -201,3 +201,21 @@ def test_stream_argument_and_preallocated_outputs(cuda_ok):
     ref = wt.forward(d["X"], d["W0"], d["b0"], d["s0"], d["Wl"], d["sl"])
     torch.cuda.synchronize()
     assert torch.equal(y, ref)
+
+
+@pytest.mark.parametrize("wl", [Workload("status_whole", 2, 3, 32, 32, 5, 3, "f32"),
+                                Workload("status_bands", 1, 2, 256, 128, 5, 3, "bf16")],
+                         ids=["whole_planes", "row_bands"])
+def test_status_word_stays_clear(cuda_ok, wl):
+    """The workspace header's status word is set only when a bounded wait for
+    an asynchronous copy runs out; after ordinary calls of every entry point
+    (whole-plane and row-band paths) it must still read 0."""
+    d = _dev(make_inputs(wl, 6), wl.io)
+    desc = wt.make_desc(wl.N, wl.C, wl.H, wl.W, wl.k, wl.L, wl.io)
+    ws = torch.zeros(wt.workspace_size(desc, 3), dtype=torch.uint8, device="cuda")
+    wt.forward(d["X"], d["W0"], d["b0"], d["s0"], d["Wl"], d["sl"], ws=ws)
+    wt.backward_data(d["dY"], d["W0"], d["s0"], d["Wl"], d["sl"], ws=ws)
+    wt.backward_weight(d["X"], d["dY"], d["W0"], d["b0"], d["s0"], d["Wl"], d["sl"], ws=ws)
+    wt.backward(d["X"], d["dY"], d["W0"], d["b0"], d["s0"], d["Wl"], d["sl"], ws=ws)
+    torch.cuda.synchronize()
+    assert int(ws[:4].view(torch.int32).item()) == 0
