@@ -1,7 +1,7 @@
 """WTConv layer fwd+bwd benchmark on B200 (prints one JSON line on rank 0).
 
 A step is one pass of the whole layer hot path over one batch: forward,
-backward-data and backward-weight (the fused kernels of libwtconv) on the
+backward-data and backward-weight (the kernels of libwtconv) on the
 ConvNeXt-T stage-1 shape (N=32, C=96, 56x56, k=5, L=3, fp32) by default.
 
   python bench.py --gpus N --steps K --warmup W [--impl reference]
@@ -374,12 +374,22 @@ def run_ours(args, wl, world, rank, local):
     return line
 
 
+def _code_only(text):
+    """C/C++ source without comments and whitespace (a comment edit does not
+    change a kernel)."""
+    import re
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return "".join(text.split())
+
+
 def sources_sha256():
-    """Hash of the CUDA sources, to tell whether committed counters still apply."""
+    """Hash of the CUDA sources' code, to tell whether committed counters
+    still apply."""
     import glob
     import hashlib
     paths = sorted(glob.glob(os.path.join(ROOT, "depthwise_convolution_wtconv_b200", "csrc", "*")))
-    return hashlib.sha256(b"".join(open(p, "rb").read() for p in paths)).hexdigest()
+    return hashlib.sha256("".join(_code_only(open(p).read()) for p in paths).encode()).hexdigest()
 
 
 def torch_cascade(X, W0, b0, s0, Wl, sl):

@@ -117,7 +117,8 @@ __global__ void wtconv_fold_kernel(int C, int L, int kk4, int wblk, const float*
   }
 }
 
-// Stager work for one plane of a unit: padded fp32 rows xf (band rows
+// Staging of one plane of a unit (paths other than the fused-deep one): padded
+// fp32 rows xf (band rows
 // [-r, TH+r)) and level-1 subbands s1 (half rows [-r, TH/2+r)), zero outside
 // the plane.  SMEM: rows come from the raw copy (row y at src + (y - y_lo) * W).
 template <int K, typename IO, bool SMEM>
