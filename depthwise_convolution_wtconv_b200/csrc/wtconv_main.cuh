@@ -117,10 +117,10 @@ __global__ void wtconv_fold_kernel(int C, int L, int kk4, int wblk, const float*
   }
 }
 
-// Staging of one plane of a unit (paths other than the fused-deep one): padded
-// fp32 rows xf (band rows
-// [-r, TH+r)) and level-1 subbands s1 (half rows [-r, TH/2+r)), zero outside
-// the plane.  SMEM: rows come from the raw copy (row y at src + (y - y_lo) * W).
+// Staging of one plane of a unit (paths other than the fused-deep one):
+// padded fp32 rows xf (band rows [-r, TH+r)) and level-1 subbands s1 (half
+// rows [-r, TH/2+r)), zero outside the plane.  SMEM: rows come from the raw
+// copy (row y at src + (y - y_lo) * W).
 template <int K, typename IO, bool SMEM>
 __device__ __forceinline__ void main_stage_item(const MainPlan& P, float* xf, float* s1, const IO* __restrict__ src,
                                                 const UnitGeo& g, int ri, int x0) {
