@@ -7,6 +7,7 @@
 #include <cstdint>
 #include <initializer_list>
 #include <mutex>
+#include <type_traits>
 #include <vector>
 
 #include "wtconv.h"
@@ -92,7 +93,7 @@ int main_slot(MainPlan& M, int TH, int PB) {
   M.wraw_off = cur;
   cur += M.wblk;
   M.raw_off = cur;
-  M.raw_pp = rup((int)(((size_t)std::min(M.H, TH + 2 * hx) * M.W * M.io_bytes + 3) / 4), 4);
+  M.raw_pp = M.direct ? 0 : rup((int)(((size_t)std::min(M.H, TH + 2 * hx) * M.W * M.io_bytes + 3) / 4), 4);
   cur += PB * M.raw_pp;
   M.rawt_off = cur;
   M.rawt_pp = (M.L >= 2 && M.bulk_t) ? rup(TH1 * M.W1, 4) : 0;
@@ -101,7 +102,14 @@ int main_slot(MainPlan& M, int TH, int PB) {
   M.w_off = cur;
   cur += M.wblk;
   int pcur = 0;  // per-plane buffers, PB copies each
-  M.xf = make_shifted(pcur, TH, M.W, r, {{R3, 4}}, 1);
+  if (M.direct) {
+    // rows land here straight from the bulk copies: column x at x + 4 (16-byte
+    // aligned), zero columns on both sides; two buffers, one per phase
+    M.xf = BufDesc{pcur, rup(M.W, 4) + 8, rup(TH, R3) + 2 * r, 0};
+    pcur += M.xf.ld * M.xf.rows;
+  } else {
+    M.xf = make_shifted(pcur, TH, M.W, r, {{R3, 4}}, 1);
+  }
   M.s1 = BufDesc{0, 0, 0, 0};
   M.t1 = BufDesc{0, 0, 0, 0};
   M.zb = BufDesc{0, 0, 0, 0};
@@ -127,6 +135,11 @@ int main_slot(MainPlan& M, int TH, int PB) {
       bd->ps = pstride;
     }
   cur += PB * pstride;
+  M.xbuf = 0;
+  if (M.direct) {
+    M.xbuf = PB * pstride;
+    cur += PB * pstride;
+  }
   return rup(cur, 4);
 }
 
@@ -141,6 +154,9 @@ bool build_main_plan(MainPlan& M, const wtconv_desc* d, int max_smem) {
   M.vec_out = (d->W % 4) == 0;
   M.wblk = main_wblk(d);
   M.bulk_t = d->L >= 2 && (M.W1 % 4) == 0;
+  // level-0 fp32 rows of at least 256 bytes go straight to the padded row
+  // buffers (shorter rows: many small copies cost more than staging saves)
+  M.direct = d->L == 0 && d->io == WTCONV_F32 && (d->W % 4) == 0 && d->W >= 64;
   const int tx = cdiv_h(d->W, 4);
   // Whole planes when at least three CTAs fit per SM (no halo rows staged
   // twice); else the most CTAs per SM (four, then three, two, one) with the
@@ -407,18 +423,24 @@ wtconv_status launch_forward_t(const wtconv_desc* d, const Device& dev, const vo
   }
   const size_t smem = (size_t)M.smem_floats * 4;
   int occ = 0;
-#define WT_MAIN(R3, FUSED)                                                                              \
+#define WT_MAIN(R3, FUSED, DIRECT)                                                                      \
   {                                                                                                     \
-    auto km = wtconv_main_kernel<K, R3, IO, FUSED>;                                                     \
+    auto km = wtconv_main_kernel<K, R3, IO, FUSED, DIRECT>;                                             \
     wtconv_status e = prepare(km, smem, occ, MAIN_NT);                                                  \
     if (e != WTCONV_OK) return e;                                                                       \
     km<<<std::min(M.units, dev.sms * occ), MAIN_NT, smem, st>>>(M, static_cast<const IO*>(x), t1, wfold, \
                                                                 static_cast<IO*>(y), status);           \
   }
   if (M.fused) {
-    if (M.R3 == 8) WT_MAIN(8, true) else WT_MAIN(4, true)
+    if (M.R3 == 8) WT_MAIN(8, true, false) else WT_MAIN(4, true, false)
+  } else if constexpr (std::is_same<IO, float>::value) {
+    if (M.direct) {
+      if (M.R3 == 8) WT_MAIN(8, false, true) else WT_MAIN(4, false, true)
+    } else {
+      if (M.R3 == 8) WT_MAIN(8, false, false) else WT_MAIN(4, false, false)
+    }
   } else {
-    if (M.R3 == 8) WT_MAIN(8, false) else WT_MAIN(4, false)
+    if (M.R3 == 8) WT_MAIN(8, false, false) else WT_MAIN(4, false, false)
   }
 #undef WT_MAIN
   return cudaGetLastError() == cudaSuccess ? WTCONV_OK : WTCONV_ERR_CUDA;

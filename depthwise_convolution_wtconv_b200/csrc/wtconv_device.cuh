@@ -115,11 +115,13 @@ __device__ __forceinline__ void store4(__nv_bfloat16* __restrict__ p, const floa
 // acc[R][CW] += sum_{u,v<K} w[u*K+v] * in[(orow+u)*ld + (j+v)]
 // `in` points at the input element (y0-r, x0-r) of the tile and must be
 // 16-byte aligned; ld is a multiple of 4 floats.  Each input row is read
-// once (NV float4 loads) and used by every output row it touches.
-template <int K, int R, int CW>
+// once (NV float4 loads) and used by every output row it touches.  With
+// OFF > 0, `in` points OFF elements before (y0-r, x0-r) (an aligned window
+// start when the row layout's column padding is not r).
+template <int K, int R, int CW, int OFF = 0>
 __device__ __forceinline__ void conv_tile(const float* __restrict__ in, int ld,
                                           const float* __restrict__ w, float (&acc)[R][CW]) {
-  constexpr int NIN = CW + K - 1;
+  constexpr int NIN = CW + K - 1 + OFF;
   constexpr int NV = (NIN + 3) / 4;
   float wr[K * K];
 #pragma unroll
@@ -143,7 +145,7 @@ __device__ __forceinline__ void conv_tile(const float* __restrict__ in, int ld,
 #pragma unroll
         for (int v = 0; v < K; ++v) {
 #pragma unroll
-          for (int j = 0; j < CW; ++j) acc[orow][j] = fmaf(wr[u * K + v], xv[j + v], acc[orow][j]);
+          for (int j = 0; j < CW; ++j) acc[orow][j] = fmaf(wr[u * K + v], xv[j + v + OFF], acc[orow][j]);
         }
       }
     }

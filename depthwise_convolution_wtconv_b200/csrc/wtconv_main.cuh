@@ -340,9 +340,9 @@ __device__ __forceinline__ void main_band_tile(const MainPlan& P, float* slot, i
 // Phase B, one tile: R3 x 4 outputs of plane j: bias, the level-1 synthesis
 // of the four Z planes (signs sigma_s(py, px); the 1/2 is in the weights),
 // the base conv, and the store.
-template <int K, int R3, typename IO>
+template <int K, int R3, typename IO, bool DIRECT>
 __device__ __forceinline__ void main_out_tile(const MainPlan& P, const float* slot, const UnitGeo& g, int j, int tile,
-                                              IO* __restrict__ y) {
+                                              int buf, IO* __restrict__ y) {
   const int ti = P.f_tx.div(tile);
   const int yy0 = ti * R3, xx0 = (tile - ti * P.f_tx.d) * 4;
   const float* sw = slot + P.w_off;
@@ -373,7 +373,14 @@ __device__ __forceinline__ void main_out_tile(const MainPlan& P, const float* sl
       acc[2 * a + 1][3] += o11;
     }
   }
-  conv_tile<K, R3, 4>(slot + P.xf.off + j * P.xf.ps + yy0 * P.xf.ld + xx0, P.xf.ld, sw, acc);
+  if constexpr (DIRECT) {
+    // rows copied straight into the buffer: column x at x + 4, so the aligned
+    // window starts 4 - r columns before the tile's first tap
+    conv_tile<K, R3, 4, 4 - K / 2>(slot + P.xf.off + buf * P.xbuf + j * P.xf.ps + yy0 * P.xf.ld + xx0, P.xf.ld, sw,
+                                   acc);
+  } else {
+    conv_tile<K, R3, 4>(slot + P.xf.off + j * P.xf.ps + yy0 * P.xf.ld + xx0, P.xf.ld, sw, acc);
+  }
   const int n = P.W - xx0 < 4 ? P.W - xx0 : 4;
   IO* yp = y + plane_index(P, g, j) * P.H * P.W;
 #pragma unroll
@@ -423,7 +430,42 @@ __device__ __forceinline__ void main_issue(const MainPlan& P, float* slot, uint6
   }
 }
 
-template <int K, int R3, typename IO, bool FUSED>
+// Level-0 fp32 planes at least 32 wide: one unit's bulk copies straight into
+// row buffer `buf` (row y of plane j at (y - y0 + r) * ld + 4, 16-byte
+// aligned), no staging pass; issued by the lanes of warp 0 after lane 0 has
+// set the phase's byte count.  The folded weights come as for the other
+// paths.
+__device__ __forceinline__ void main_issue_direct(const MainPlan& P, float* slot, uint64_t* full, const UnitGeo& g,
+                                                  int buf, const float* __restrict__ x,
+                                                  const float* __restrict__ wfold) {
+  const int lane = threadIdx.x & 31;
+  const int nrows = g.y_hi - g.y_lo;
+  const unsigned brow = (unsigned)(P.W * 4);
+  if (lane == 0) {
+    const unsigned bw = (unsigned)(P.wblk * 4);
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(full)),
+                 "r"(bw + brow * nrows * g.npb)
+                 : "memory");
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(slot + P.wraw_off)),
+        "l"(wfold + (size_t)g.c * P.wblk), "r"(bw), "r"(smem_u32(full))
+        : "memory");
+  }
+  __syncwarp();
+  for (int q = lane; q < g.npb * nrows; q += 32) {
+    const int j = q / nrows, yy = g.y_lo + (q - j * nrows);
+    float* dst = slot + P.xf.off + buf * P.xbuf + j * P.xf.ps + (yy - g.y0 + P.r) * P.xf.ld + 4;
+    const float* src = x + plane_index(P, g, j) * P.H * P.W + (size_t)yy * P.W;
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_u32(dst)),
+                 "l"(src), "r"(brow), "r"(smem_u32(full))
+                 : "memory");
+  }
+}
+
+template <int K, int R3, typename IO, bool FUSED, bool DIRECT>
 __global__ void __launch_bounds__(MAIN_NT, 4)
     wtconv_main_kernel(const MainPlan P, const IO* __restrict__ x, const float* __restrict__ t1g,
                        const float* __restrict__ wfold, IO* __restrict__ y, int* __restrict__ status) {
@@ -441,13 +483,37 @@ __global__ void __launch_bounds__(MAIN_NT, 4)
   __syncthreads();
   const int myunits = (int)blockIdx.x < P.units ? (P.units - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
   float* slot = sm + P.slot0;
-  if (tid == 0 && myunits > 0) main_issue<IO>(P, slot, full, unit_geo(P, blockIdx.x), x, t1g, wfold);
+  if constexpr (DIRECT) {
+    if (tid < 32 && myunits > 0)
+      main_issue_direct(P, slot, full, unit_geo(P, blockIdx.x), 0, reinterpret_cast<const float*>(x), wfold);
+  } else {
+    if (tid == 0 && myunits > 0) main_issue<IO>(P, slot, full, unit_geo(P, blockIdx.x), x, t1g, wfold);
+  }
   int k = 0;
   for (; k < myunits; ++k) {
     const UnitGeo g = unit_geo(P, blockIdx.x + k * gridDim.x);
     // every thread waits on every phase in order, so a parity wait is exact
     mb_wait(full, k & 1, abort_flag);
-    const int n = FUSED ? 0 : g.npb * P.stage_pp;
+    const int n = (FUSED || DIRECT) ? 0 : g.npb * P.stage_pp;
+    if constexpr (DIRECT) {
+      // The halo rows of the first and last band lie outside the image and
+      // must read as zero, but the buffer may hold another band's rows there
+      // (bands divide H, so no other row is outside; whole planes never
+      // write those rows at all).  The fence orders these generic stores
+      // before the bulk copies that later refill the rows.
+      constexpr int hx = K / 2;
+      if (P.nbands > 1 && (g.y0 == 0 || g.y0 + P.TH == P.H)) {
+        const int rr0 = g.y0 == 0 ? 0 : P.TH + hx;
+        const int q = P.xf.ld >> 2;
+        for (int it = tid; it < g.npb * hx * q; it += MAIN_NT) {
+          const int j = it / (hx * q), rem = it - j * hx * q;
+          const int rr = rem / q, cx = (rem - rr * q) << 2;
+          *reinterpret_cast<float4*>(slot + P.xf.off + (k & 1) * P.xbuf + j * P.xf.ps + (rr0 + rr) * P.xf.ld + cx) =
+              make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      }
+    }
     if constexpr (FUSED) {
       const int nb = g.npb * P.f_bpp.d;
       for (int it = tid; it < nb; it += MAIN_NT) {
@@ -496,8 +562,14 @@ __global__ void __launch_bounds__(MAIN_NT, 4)
     }
     __syncthreads();
     if (*abort_flag) break;  // uniform: read after the barrier
-    if (tid == 0 && k + 1 < myunits)
-      main_issue<IO>(P, slot, full, unit_geo(P, blockIdx.x + (k + 1) * gridDim.x), x, t1g, wfold);
+    if constexpr (DIRECT) {
+      if (tid < 32 && k + 1 < myunits)
+        main_issue_direct(P, slot, full, unit_geo(P, blockIdx.x + (k + 1) * gridDim.x), (k + 1) & 1,
+                          reinterpret_cast<const float*>(x), wfold);
+    } else {
+      if (tid == 0 && k + 1 < myunits)
+        main_issue<IO>(P, slot, full, unit_geo(P, blockIdx.x + (k + 1) * gridDim.x), x, t1g, wfold);
+    }
     if constexpr (FUSED) {
       // levels 3..L of the pyramid, then every deep level's band convs
       for (int l = 3; l <= P.L; ++l) {
@@ -518,7 +590,7 @@ __global__ void __launch_bounds__(MAIN_NT, 4)
     }
     for (int it = tid; it < P.tiles; it += MAIN_NT) {
       const int j = P.f_tpp.div(it);
-      if (j < g.npb) main_out_tile<K, R3, IO>(P, slot, g, j, it - j * P.tiles_pp, y);
+      if (j < g.npb) main_out_tile<K, R3, IO, DIRECT>(P, slot, g, j, it - j * P.tiles_pp, k & 1, y);
     }
     __syncthreads();
   }

@@ -72,6 +72,7 @@ struct MainPlan {
   BufDesc xf, s1, t1, zb;    // per-plane copies at ps stride (zb: the four level-1 Z planes)
   int a_pp;                  // phase-A tiles per plane: 4 bands x ceil(TH/8) x ceil(W1/4)
   int fused;                 // whole planes with L >= 2: levels >= 2 computed here, t1 on the fly
+  int direct, xbuf;          // level-0 fp32 rows copied straight into two xf buffers xbuf floats apart
   BufDesc sd[MAXL + 1], zd[MAXL + 1];  // fused: subbands and band-conv outputs of levels 2..L
   int dfirst[MAXL + 2];      // fused: first deep-conv tile of level l within a plane
   FDiv f_dtiles[MAXL + 1], f_dtx[MAXL + 1], f_dper;  // fused: 4x4 tiles per band, per tile row; per plane

@@ -103,6 +103,14 @@ EDGE = [
     # bulk copies), and bf16
     Workload("band_L0_nobulk", 1, 2, 150, 146, 5, 0, "f32"),
     Workload("band_L0_bf16", 2, 2, 160, 132, 3, 0, "bf16"),
+    # level-0 fp32 rows of 64 or more floats: input rows copied straight
+    # into the padded row buffers (row bands with k = 7; batched whole planes
+    # with a partial last batch; many units per CTA alternating the two
+    # buffers; k = 1)
+    Workload("rows_L0_k7_bands", 2, 2, 256, 96, 7, 0, "f32"),
+    Workload("rows_L0_k5_batched", 5, 4, 8, 64, 5, 0, "f32"),
+    Workload("rows_L0_k3_reuse", 6, 1000, 8, 64, 3, 0, "f32"),
+    Workload("rows_L0_k1", 2, 3, 12, 64, 1, 0, "f32"),
 ]
 
 
