@@ -79,12 +79,17 @@ int main_wblk(const wtconv_desc* d) { return rup((1 + 4 * d->L) * rup(d->k * d->
 
 // Output tile rows for band height TH: 8, unless 4 wastes fewer padded rows
 // or the band is at most 8 rows (twice the tiles for the CTA's threads).
-int main_r3(int TH) { return TH > 8 && rup(TH, 8) == rup(TH, 4) ? 8 : 4; }
+// Level-0 whole planes of at most 16 rows take 4: these units are short and
+// latency-bound, and the smaller register tile lets more CTAs share an SM.
+int main_r3(int H, int L, int TH) {
+  if (L == 0 && TH == H && H <= 16) return 4;
+  return TH > 8 && rup(TH, 8) == rup(TH, 4) ? 8 : 4;
+}
 
 // Slot layout for band height TH and PB planes per unit; returns the slot
 // size in floats.
 int main_slot(MainPlan& M, int TH, int PB) {
-  const int r = M.r, R3 = main_r3(TH), TH1 = TH / 2;
+  const int r = M.r, R3 = main_r3(M.H, M.L, TH), TH1 = TH / 2;
   const int hx = M.L >= 1 ? 2 * r : r;
   M.fused = TH == M.H && M.L >= 2;
   if (M.fused) M.bulk_t = 0;
@@ -169,7 +174,7 @@ bool build_main_plan(MainPlan& M, const wtconv_desc* d, int max_smem) {
     const size_t budget = std::min((size_t)max_smem, (size_t)SM_SMEM / occ - 1024);
     for (int cand = d->H; cand >= (pass == 0 ? d->H : 2) && TH < 0; --cand) {
       if (d->H % cand || (cand != d->H && (cand & 1))) continue;
-      const int tpp = cdiv_h(cand, main_r3(cand)) * tx;
+      const int tpp = cdiv_h(cand, main_r3(d->H, d->L, cand)) * tx;
       int pb = cand == d->H ? std::max(1, std::min(d->N, MAIN_NT / tpp)) : 1;
       for (; pb >= 1 && TH < 0; --pb) {
         MainPlan T = M;
@@ -184,7 +189,7 @@ bool build_main_plan(MainPlan& M, const wtconv_desc* d, int max_smem) {
   if (TH < 0) return false;
   M.TH = TH;
   M.PB = PB;
-  M.R3 = main_r3(TH);
+  M.R3 = main_r3(d->H, d->L, TH);
   M.nbands = d->H / TH;
   M.units = d->C * ((d->N + PB - 1) / PB) * M.nbands;
   M.slot_floats = main_slot(M, TH, PB);
@@ -521,7 +526,7 @@ bool bw_layout(BwPlan& B, int PB, int max_smem) {
     B.gd[l].off += base;
   }
   B.red_off = base;
-  const int need = std::max(base + PB * B.ps, base + BW_NT * B.kk4 + BW_NT);
+  const int need = std::max(base + PB * B.ps, base + BW_NT * (B.kk4 + 1) + BW_NT);
   B.smem_floats = MAIN_HEADER + rup(need, 4);
   return (size_t)B.smem_floats * 4 <= (size_t)max_smem;
 }
@@ -583,9 +588,9 @@ void bw_branches(BwPlan& B) {
   }
 }
 
-// Whole-plane plan: the most planes per unit (up to two tiles per thread)
-// that fit two CTAs per SM, else one.  False when one plane does not fit;
-// such shapes run on the row-band path.
+// Whole-plane plan: the most planes per unit (up to two tiles per thread,
+// one at level 0) that fit two CTAs per SM, else one.  False when one plane
+// does not fit; such shapes run on the row-band path.
 bool build_bw_plan(BwPlan& B, const wtconv_desc* d, int max_smem) {
   B = BwPlan{};
   B.N = d->N;
@@ -604,7 +609,10 @@ bool build_bw_plan(BwPlan& B, const wtconv_desc* d, int max_smem) {
   B.BH = d->L >= 2 ? 4 : (d->L == 1 ? 2 : 1);
   int per_plane = cdiv_h(d->H, 4) * cdiv_h(d->W, 4);
   for (int l = 1; l <= d->L; ++l) per_plane += 4 * cdiv_h(d->H >> l, 4) * cdiv_h(d->W >> l, 4);
-  const int pb0 = std::max(1, std::min(d->N, cdiv_h(2 * BW_NT, per_plane)));
+  // up to two tiles per thread; level 0 (one branch, short units) up to one,
+  // which leaves each CTA several units whose copies overlap the compute
+  const int tpt = d->L == 0 ? 1 : 2;
+  const int pb0 = std::max(1, std::min(d->N, cdiv_h(tpt * BW_NT, per_plane)));
   bool ok = false;
   // two CTAs per SM if possible; else one (still faster than row bands,
   // which stage halo rows twice and hand the LL planes through HBM)

@@ -29,12 +29,6 @@
 
 namespace wt {
 
-__device__ __forceinline__ float warp_sum(float v) {
-#pragma unroll
-  for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
-}
-
 // Stages `rows` rows of a plane (row y0 first; rows outside [0, h) are
 // written as zeros) into shared memory at dst + i*ld + col0, converting to
 // fp32.  The rows come from the plane in global memory, or (SMEM) from a

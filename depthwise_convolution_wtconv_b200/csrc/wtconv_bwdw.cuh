@@ -223,23 +223,43 @@ __global__ void __launch_bounds__(BW_NT, 2) wtconv_bwdw_kernel(const __grid_cons
     }
     return;
   }
-  // fixed-order reduction: the threads of each branch in index order
+  // Fixed-order reduction.  An entry of a branch with at most 32 threads is
+  // summed by one thread over the branch's threads in index order; an entry
+  // of a larger branch (and the sum of dy, over all threads) by one warp,
+  // lane l summing threads l, l + 32, ... in order, then a fixed butterfly.
+  // The row stride kk4 + 1 (odd) keeps the strided reads free of bank
+  // conflicts.
   float* red = slot + P.red_off;
+  const int rld = P.kk4 + 1;
 #pragma unroll
-  for (int t = 0; t < KK; ++t) red[tid * P.kk4 + t] = G[t];
-  red[BW_NT * P.kk4 + tid] = sumdy;
+  for (int t = 0; t < KK; ++t) red[tid * rld + t] = G[t];
+  red[BW_NT * rld + tid] = sumdy;
   __syncthreads();
   float* out = part + (size_t)blockIdx.x * P.V;
-  for (int e = tid; e < P.V; e += BW_NT) {
+  for (int e = tid; e < P.V - 1; e += BW_NT) {
+    const int bb = e / KK, t = e - bb * KK;
+    const BwBranch& Bb = P.br[bb];
+    if (Bb.nthr > 32) continue;
     float acc = 0.f;
-    if (e == P.V - 1) {
-      for (int th = 0; th < BW_NT; ++th) acc += red[BW_NT * P.kk4 + th];
-    } else {
-      const int bb = e / KK, t = e - bb * KK;
-      const BwBranch& Bb = P.br[bb];
-      for (int th = Bb.first; th < Bb.first + Bb.nthr; ++th) acc += red[th * P.kk4 + t];
-    }
+    for (int th = Bb.first; th < Bb.first + Bb.nthr; ++th) acc += red[th * rld + t];
     out[e] = acc;
+  }
+  const int warp = tid >> 5, lane = tid & 31;
+  for (int bb = 0; bb < P.nbr; ++bb) {
+    const BwBranch& Bb = P.br[bb];
+    if (Bb.nthr <= 32) continue;  // uniform
+    for (int t = warp; t < KK; t += BW_NT / 32) {
+      float acc = 0.f;
+      for (int th = lane; th < Bb.nthr; th += 32) acc += red[(Bb.first + th) * rld + t];
+      acc = warp_sum(acc);
+      if (lane == 0) out[bb * KK + t] = acc;
+    }
+  }
+  if (warp == BW_NT / 32 - 1) {
+    float acc = 0.f;
+    for (int th = lane; th < BW_NT; th += 32) acc += red[BW_NT * rld + th];
+    acc = warp_sum(acc);
+    if (lane == 0) out[P.V - 1] = acc;
   }
 }
 

@@ -112,6 +112,14 @@ __device__ __forceinline__ void store4(__nv_bfloat16* __restrict__ p, const floa
 }
 
 // ------------------------------------------------------ register-tiled conv
+// Sum over the 32 lanes of a warp by a fixed butterfly: the same order on
+// every run, so reductions built on it are deterministic.
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
 // acc[R][CW] += sum_{u,v<K} w[u*K+v] * in[(orow+u)*ld + (j+v)]
 // `in` points at the input element (y0-r, x0-r) of the tile and must be
 // 16-byte aligned; ld is a multiple of 4 floats.  Each input row is read

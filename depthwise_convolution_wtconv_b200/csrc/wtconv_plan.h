@@ -151,7 +151,7 @@ struct BwPlan {
   FDiv f_spp, f_sx;                // staging blocks per plane, per block row
   int nbr;                         // branches: 1 + 4L
   BwBranch br[BW_MAXB];
-  int red_off;                     // final reduction: BW_NT * kk4 + BW_NT floats (over the slab)
+  int red_off;                     // final reduction: BW_NT * (kk4 + 1) + BW_NT floats (over the slab)
   int smem_floats;
 };
 
