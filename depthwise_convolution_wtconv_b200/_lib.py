@@ -15,6 +15,7 @@ LIB_PATH = os.path.join(_PKG, "libwtconv.so")
 
 F32, BF16 = 0, 1
 OP_FORWARD, OP_BACKWARD_DATA, OP_BACKWARD_WEIGHT, OP_BACKWARD = 0, 1, 2, 3
+OP_FORWARD_FOLDED, OP_FOLD = 4, 5
 STATUS_NAMES = {0: "WTCONV_OK", 1: "WTCONV_ERR_ARG", 2: "WTCONV_ERR_SHAPE", 3: "WTCONV_ERR_ALIGN",
                 4: "WTCONV_ERR_WORKSPACE", 5: "WTCONV_ERR_CUDA", 6: "WTCONV_ERR_UNSUPPORTED",
                 7: "WTCONV_ERR_SCRATCH_LIMIT"}
@@ -22,7 +23,8 @@ NOALLOC_SCRATCH_BYTES = 8 << 20
 
 # every symbol include/wtconv.h declares
 EXPORTS = ("wtconv_workspace_size", "wtconv_forward", "wtconv_backward_data", "wtconv_backward_weight",
-           "wtconv_backward", "wtconv_backward_weight_noalloc", "wtconv_kernel_launches", "wtconv_status_string")
+           "wtconv_backward", "wtconv_backward_weight_noalloc", "wtconv_folded_size", "wtconv_fold_weights",
+           "wtconv_forward_folded", "wtconv_kernel_launches", "wtconv_status_string")
 
 
 class WTConvDesc(ctypes.Structure):
@@ -63,6 +65,12 @@ def load(path=LIB_PATH):
     lib.wtconv_backward_weight_noalloc.restype = ctypes.c_int
     lib.wtconv_status_string.argtypes = [ctypes.c_int]
     lib.wtconv_status_string.restype = ctypes.c_char_p
+    lib.wtconv_folded_size.argtypes = [dp]
+    lib.wtconv_folded_size.restype = sz
+    lib.wtconv_fold_weights.argtypes = [dp, fp, fp, fp, fp, fp, ctypes.c_int, vp, sz, vp]
+    lib.wtconv_fold_weights.restype = ctypes.c_int
+    lib.wtconv_forward_folded.argtypes = [dp, vp, vp, vp, vp, sz, vp]
+    lib.wtconv_forward_folded.restype = ctypes.c_int
     lib.wtconv_kernel_launches.argtypes = [dp, ctypes.c_int]
     lib.wtconv_kernel_launches.restype = ctypes.c_int
     _lib = lib
@@ -216,3 +224,37 @@ def backward(x, dy, w0, b0, s0, wl=None, sl=None, dx=None, grads=None, ws=None, 
                                _ptr(sl), _ptr(dx), _ptr(g["dw0"]), _ptr(g["db0"]), _ptr(g["ds0"]), _ptr(g["dwl"]),
                                _ptr(g["dsl"]), _ptr(ws), nws, _stream(stream)), "wtconv_backward")
     return dx, g
+
+
+def fold_weights(w0, b0, s0, wl=None, sl=None, adjoint=False, folded=None, stream=None):
+    """The scales folded into the weights once (for fixed parameters, e.g.
+    inference): a uint8 CUDA tensor holding the library's folded block; with
+    adjoint=True the backward-data block (flipped kernels, no bias)."""
+    lib = load()
+    wl, sl = _params(w0, None if adjoint else b0, s0, wl, sl)
+    C, k = w0.shape[0], w0.shape[-1]
+    desc = make_desc(1, C, 1 << _levels(wl), 1 << _levels(wl), k, _levels(wl), "f32")
+    need = lib.wtconv_folded_size(ctypes.byref(desc))
+    if folded is None:
+        folded = torch.empty(max(need, 16), dtype=torch.uint8, device="cuda")
+    _check(lib.wtconv_fold_weights(ctypes.byref(desc), _ptr(w0), _ptr(None if adjoint else b0), _ptr(s0),
+                                   _ptr(wl), _ptr(sl), int(bool(adjoint)), _ptr(folded),
+                                   folded.numel() * folded.element_size(), _stream(stream)), "wtconv_fold_weights")
+    return folded
+
+
+def forward_folded(x, folded, k, L, y=None, ws=None, stream=None):
+    """y = WTConv(x) over a block from fold_weights (kernel size k, L levels);
+    with an adjoint block and dy for x, the backward-data pass."""
+    lib = load()
+    _cuda(x, "x")
+    _cuda(folded, "folded")
+    N, C, H, W = x.shape
+    desc = make_desc(N, C, H, W, k, L, "bf16" if x.dtype == torch.bfloat16 else "f32")
+    if folded.numel() * folded.element_size() < lib.wtconv_folded_size(ctypes.byref(desc)):
+        raise ValueError("folded block too small for this shape")
+    y = torch.empty_like(x) if y is None else _cuda(y, "y", x.dtype)
+    ws, nws = _workspace(desc, OP_FORWARD_FOLDED, ws)
+    _check(lib.wtconv_forward_folded(ctypes.byref(desc), _ptr(x), _ptr(folded), _ptr(y), _ptr(ws), nws,
+                                     _stream(stream)), "wtconv_forward_folded")
+    return y

@@ -254,6 +254,8 @@ bool build_deep_plan(DeepPlan& D, const wtconv_desc* d, int max_smem) {
   D.kk4 = rup(d->k * d->k, 4);
   D.io_bytes = io_bytes(d);
   D.vec_in = (d->W % 4) == 0;
+  D.wblk = main_wblk(d);
+  D.wdeep = 5 * D.kk4 + 4;
   int slab = 0;
   deep_slab_items(D, slab);
   D.w_off = 0;
@@ -400,18 +402,22 @@ wtconv_status prepare(F kern, size_t smem, int& occ, int nthreads = NT) {
   return WTCONV_OK;
 }
 
+// The folded weight block of every channel (reformulation (3)), one launch.
+template <int K>
+wtconv_status launch_fold(const wtconv_desc* d, const Device& dev, const float* w0, const float* b0, const float* s0,
+                          const float* wl, const float* sl, int flip, float* wfold, cudaStream_t st) {
+  const int kk4 = rup(d->k * d->k, 4), wblk = main_wblk(d);
+  const int n = d->C * wblk;
+  wtconv_fold_kernel<K><<<std::min((n + 255) / 256, dev.sms * 4), 256, 0, st>>>(d->C, d->L, kk4, wblk, w0, b0, s0,
+                                                                                 wl, sl, flip, wfold);
+  return cudaGetLastError() == cudaSuccess ? WTCONV_OK : WTCONV_ERR_CUDA;
+}
+
+// Deep kernel (row-band planes with L >= 2) and output kernel over folded
+// weights `wfold`.
 template <int K, typename IO>
-wtconv_status launch_forward_t(const wtconv_desc* d, const Device& dev, const void* x, const float* w0,
-                               const float* b0, const float* s0, const float* wl, const float* sl, void* y, int flip,
+wtconv_status launch_forward_t(const wtconv_desc* d, const Device& dev, const void* x, const float* wfold, void* y,
                                int* status, float* t1, cudaStream_t st) {
-  float* wfold = reinterpret_cast<float*>(reinterpret_cast<char*>(t1) + t1_bytes(d));
-  {
-    const int kk4 = rup(d->k * d->k, 4), wblk = main_wblk(d);
-    const int n = d->C * wblk;
-    wtconv_fold_kernel<K><<<std::min((n + 255) / 256, dev.sms * 4), 256, 0, st>>>(d->C, d->L, kk4, wblk, w0, b0, s0,
-                                                                                   wl, sl, flip, wfold);
-    if (cudaGetLastError() != cudaSuccess) return WTCONV_ERR_CUDA;
-  }
   MainPlan M;
   if (!build_main_plan(M, d, dev.max_smem)) return WTCONV_ERR_UNSUPPORTED;
   if (d->L >= 2 && !M.fused) {
@@ -423,7 +429,7 @@ wtconv_status launch_forward_t(const wtconv_desc* d, const Device& dev, const vo
     wtconv_status e = prepare(kd, smem, occ, DEEP_NT);
     if (e != WTCONV_OK) return e;
     const int units = D.C * D.nbatch;
-    kd<<<std::min(units, dev.sms * occ), DEEP_NT, smem, st>>>(D, static_cast<const IO*>(x), wl, sl, t1, flip);
+    kd<<<std::min(units, dev.sms * occ), DEEP_NT, smem, st>>>(D, static_cast<const IO*>(x), wfold, t1);
     if (cudaGetLastError() != cudaSuccess) return WTCONV_ERR_CUDA;
   }
   const size_t smem = (size_t)M.smem_floats * 4;
@@ -452,28 +458,50 @@ wtconv_status launch_forward_t(const wtconv_desc* d, const Device& dev, const vo
 }
 
 template <int K>
-wtconv_status launch_forward_k(const wtconv_desc* d, const Device& dev, const void* x, const float* w0,
-                               const float* b0, const float* s0, const float* wl, const float* sl, void* y, int flip,
+wtconv_status launch_forward_k(const wtconv_desc* d, const Device& dev, const void* x, const float* wfold, void* y,
                                int* status, float* t1, cudaStream_t st) {
-  if (d->io == WTCONV_F32) return launch_forward_t<K, float>(d, dev, x, w0, b0, s0, wl, sl, y, flip, status, t1, st);
-  return launch_forward_t<K, __nv_bfloat16>(d, dev, x, w0, b0, s0, wl, sl, y, flip, status, t1, st);
+  if (d->io == WTCONV_F32) return launch_forward_t<K, float>(d, dev, x, wfold, y, status, t1, st);
+  return launch_forward_t<K, __nv_bfloat16>(d, dev, x, wfold, y, status, t1, st);
 }
 
-// Forward (flip = 0) or backward-data (flip = 1).  ws: 16-byte header (status
-// word) followed by t1 when L >= 2 (ws may be NULL when L < 2).
-wtconv_status run_forward(const wtconv_desc* d, const void* x, const float* w0, const float* b0, const float* s0,
-                          const float* wl, const float* sl, void* y, int flip, void* ws, cudaStream_t st) {
+// Folds the weights into `wfold` (flip = 1: the adjoint's block).
+wtconv_status run_fold(const wtconv_desc* d, const float* w0, const float* b0, const float* s0, const float* wl,
+                       const float* sl, int flip, float* wfold, cudaStream_t st) {
+  Device dev;
+  wtconv_status e = query_device(dev);
+  if (e != WTCONV_OK) return e;
+  switch (d->k) {
+    case 1: return launch_fold<1>(d, dev, w0, b0, s0, wl, sl, flip, wfold, st);
+    case 3: return launch_fold<3>(d, dev, w0, b0, s0, wl, sl, flip, wfold, st);
+    case 5: return launch_fold<5>(d, dev, w0, b0, s0, wl, sl, flip, wfold, st);
+    default: return launch_fold<7>(d, dev, w0, b0, s0, wl, sl, flip, wfold, st);
+  }
+}
+
+// The data pass over a folded block.  ws: 16-byte header (status word)
+// followed by t1 when L >= 2.
+wtconv_status run_folded(const wtconv_desc* d, const void* x, const float* wfold, void* y, void* ws, cudaStream_t st) {
   Device dev;
   wtconv_status e = query_device(dev);
   if (e != WTCONV_OK) return e;
   int* status = static_cast<int*>(ws);
   float* t1 = reinterpret_cast<float*>(static_cast<char*>(ws) + 16);
   switch (d->k) {
-    case 1: return launch_forward_k<1>(d, dev, x, w0, b0, s0, wl, sl, y, flip, status, t1, st);
-    case 3: return launch_forward_k<3>(d, dev, x, w0, b0, s0, wl, sl, y, flip, status, t1, st);
-    case 5: return launch_forward_k<5>(d, dev, x, w0, b0, s0, wl, sl, y, flip, status, t1, st);
-    default: return launch_forward_k<7>(d, dev, x, w0, b0, s0, wl, sl, y, flip, status, t1, st);
+    case 1: return launch_forward_k<1>(d, dev, x, wfold, y, status, t1, st);
+    case 3: return launch_forward_k<3>(d, dev, x, wfold, y, status, t1, st);
+    case 5: return launch_forward_k<5>(d, dev, x, wfold, y, status, t1, st);
+    default: return launch_forward_k<7>(d, dev, x, wfold, y, status, t1, st);
   }
+}
+
+// Forward (flip = 0) or backward-data (flip = 1): the weights are folded into
+// the workspace after t1, then the data pass runs over them.
+wtconv_status run_forward(const wtconv_desc* d, const void* x, const float* w0, const float* b0, const float* s0,
+                          const float* wl, const float* sl, void* y, int flip, void* ws, cudaStream_t st) {
+  float* wfold = reinterpret_cast<float*>(static_cast<char*>(ws) + 16 + t1_bytes(d));
+  wtconv_status e = run_fold(d, w0, b0, s0, wl, sl, flip, wfold, st);
+  if (e != WTCONV_OK) return e;
+  return run_folded(d, x, wfold, y, ws, st);
 }
 
 // Workspace: a 16-byte header whose first int is the device status word,
@@ -962,9 +990,39 @@ size_t wtconv_workspace_size(const wtconv_desc* desc, int op) {
       return bwdw_ws_bytes(desc);
     case WTCONV_OP_BACKWARD:
       return std::max(bwdw_ws_bytes(desc), fwd_ws_bytes(desc));
+    case WTCONV_OP_FORWARD_FOLDED:
+      return 16 + t1_bytes(desc);
     default:
       return 0;
   }
+}
+
+size_t wtconv_folded_size(const wtconv_desc* desc) {
+  if (check_desc(desc) != WTCONV_OK) return 0;
+  return (size_t)desc->C * main_wblk(desc) * sizeof(float);
+}
+
+wtconv_status wtconv_fold_weights(const wtconv_desc* desc, const float* w0, const float* b0, const float* s0,
+                                  const float* wl, const float* sl, int adjoint, void* folded,
+                                  size_t folded_bytes, void* stream) {
+  wtconv_status e = check_desc(desc);
+  if (e != WTCONV_OK) return e;
+  if (adjoint != 0 && adjoint != 1) return WTCONV_ERR_ARG;
+  if ((e = check_params(desc, w0, adjoint ? nullptr : b0, s0, wl, sl, !adjoint)) != WTCONV_OK) return e;
+  if (!folded) return WTCONV_ERR_ARG;
+  if (!aligned16(folded)) return WTCONV_ERR_ALIGN;
+  if (folded_bytes < wtconv_folded_size(desc)) return WTCONV_ERR_WORKSPACE;
+  return run_fold(desc, w0, b0, s0, wl, sl, adjoint, static_cast<float*>(folded), static_cast<cudaStream_t>(stream));
+}
+
+wtconv_status wtconv_forward_folded(const wtconv_desc* desc, const void* x, const void* folded, void* y, void* ws,
+                                    size_t ws_bytes, void* stream) {
+  wtconv_status e = check_desc(desc);
+  if (e != WTCONV_OK) return e;
+  if (!x || !y || !folded) return WTCONV_ERR_ARG;
+  if (!aligned16(x) || !aligned16(y) || !aligned16(folded)) return WTCONV_ERR_ALIGN;
+  if ((e = check_ws(ws, ws_bytes, 16 + t1_bytes(desc))) != WTCONV_OK) return e;
+  return run_folded(desc, x, static_cast<const float*>(folded), y, ws, static_cast<cudaStream_t>(stream));
 }
 
 wtconv_status wtconv_forward(const wtconv_desc* desc, const void* x, const float* w0, const float* b0,
@@ -1096,7 +1154,8 @@ int wtconv_kernel_launches(const wtconv_desc* desc, int op) {
   if (check_desc(desc) != WTCONV_OK) return 0;
   MainPlan M;
   const bool main_ok = build_main_plan(M, desc, PLAN_SMEM);
-  const int data = main_ok ? 2 + ((desc->L >= 2 && !M.fused) ? 1 : 0) : 0;  // fold, [deep], output
+  const int pass = main_ok ? 1 + ((desc->L >= 2 && !M.fused) ? 1 : 0) : 0;  // [deep], output
+  const int data = main_ok ? 1 + pass : 0;                                  // fold first
   const int weight = bwdw_whole_plane(desc) ? 2 : (desc->L == 0 ? 1 : desc->L) + 1;  // kernel(s), finalize
   switch (op) {
     case WTCONV_OP_FORWARD:
@@ -1106,6 +1165,10 @@ int wtconv_kernel_launches(const wtconv_desc* desc, int op) {
       return weight;
     case WTCONV_OP_BACKWARD:
       return data + weight;
+    case WTCONV_OP_FORWARD_FOLDED:
+      return pass;
+    case WTCONV_OP_FOLD:
+      return 1;
     default:
       return 0;
   }

@@ -110,7 +110,7 @@ __global__ void wtconv_fold_kernel(int C, int L, int kk4, int wblk, const float*
       if (t < KK) {
         const int l = (blk >> 2) + 1, s = blk & 3;
         const size_t base = ((size_t)(l - 1) * C + c) * 4 + s;
-        v = (sl[base] * wl[base * KK + (flip ? KK - 1 - t : t)]) * __int_as_float((127 - l) << 23);
+        v = (sl[base] * wl[base * KK + (flip ? KK - 1 - t : t)]) * pow2neg(l);
       }
     }
     out[i] = v;
@@ -606,11 +606,9 @@ __global__ void __launch_bounds__(MAIN_NT, 4)
 // 2^-l s_l W_l), then t1 by the closed form, stored to global memory.
 template <int K, typename IO>
 __global__ void __launch_bounds__(DEEP_NT) wtconv_deep_kernel(const DeepPlan P, const IO* __restrict__ x,
-                                                              const float* __restrict__ wl,
-                                                              const float* __restrict__ sl, float* __restrict__ t1g,
-                                                              int flip) {
+                                                              const float* __restrict__ wfold,
+                                                              float* __restrict__ t1g) {
   constexpr int r = K / 2;
-  constexpr int KK = K * K;
   extern __shared__ float4 smem4[];
   float* sm = reinterpret_cast<float*>(smem4);
   for (int i = threadIdx.x; i < (P.smem_floats >> 2); i += DEEP_NT) smem4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -624,17 +622,8 @@ __global__ void __launch_bounds__(DEEP_NT) wtconv_deep_kernel(const DeepPlan P, 
     const int c = u - bt * P.C;
     const int nb0 = bt * P.PB;
     const int npb = (P.N - nb0) < P.PB ? (P.N - nb0) : P.PB;
-    for (int i = threadIdx.x; i < (P.L - 1) * 4 * kk4; i += DEEP_NT) {
-      const int blk = i / kk4, e = i - blk * kk4;
-      float v = 0.f;
-      if (e < KK) {
-        const int l = blk / 4 + 2, s = blk & 3;
-        const int tt = flip ? (KK - 1 - e) : e;
-        const size_t base = ((size_t)(l - 1) * P.C + c) * 4 + s;
-        v = (sl[base] * wl[base * KK + tt]) * pow2neg(l);
-      }
-      sw[i] = v;
-    }
+    // the channel's folded level-2..L weights (contiguous in its block)
+    for (int i = threadIdx.x; i < (P.L - 1) * 4 * kk4; i += DEEP_NT) sw[i] = wfold[(size_t)c * P.wblk + P.wdeep + i];
     // level-2 subbands straight from 4x4 blocks of x (two blocks in flight)
     {
       const int bw = P.W >> 2, per = (P.H >> 2) * bw, n = npb * per;

@@ -88,6 +88,7 @@ struct MainPlan {
 struct DeepPlan {
   int N, C, H, W, K, r, L, H1, W1, kk4, io_bytes, vec_in;
   int PB, nbatch;
+  int wblk, wdeep;           // floats per channel of the folded block; offset of its level-2 kernels
   int w_off;                 // folded weights of levels 2..L
   BufDesc sd[MAXL + 1], zd[MAXL + 1];
   FDiv f_stage_per, f_stage_x, f_deep_per, f_t1_per, f_t1_x;

@@ -92,12 +92,15 @@ typedef enum {
   WTCONV_ERR_SCRATCH_LIMIT = 7
 } wtconv_status;
 
-/* Operation codes for wtconv_workspace_size. */
+/* Operation codes for wtconv_workspace_size and wtconv_kernel_launches
+ * (WTCONV_OP_FOLD: wtconv_fold_weights, which needs no workspace). */
 enum {
   WTCONV_OP_FORWARD = 0,
   WTCONV_OP_BACKWARD_DATA = 1,
   WTCONV_OP_BACKWARD_WEIGHT = 2,
-  WTCONV_OP_BACKWARD = 3
+  WTCONV_OP_BACKWARD = 3,
+  WTCONV_OP_FORWARD_FOLDED = 4,
+  WTCONV_OP_FOLD = 5
 };
 
 /* Bytes of device workspace the operation `op` uses for `desc` (0 when desc
@@ -186,6 +189,39 @@ wtconv_status wtconv_backward_weight_noalloc(const wtconv_desc* desc,
                                              const float* sl, float* dw0,
                                              float* db0, float* ds0, float* dwl,
                                              float* dsl, void* stream);
+
+/* Bytes of the folded-weight block of `desc` (0 when desc is invalid): per
+ * channel, s0*w0 and s0*b0, then 2^-l s_l[s] w_l[s] for every level l and
+ * band s (2^-l: the synthesis factors 1/2 between level l and the image),
+ * each k x k kernel padded to a multiple of 4 floats. */
+size_t wtconv_folded_size(const wtconv_desc* desc);
+
+/* Folds the per-channel scales into the convolution weights once
+ * (arXiv:2608.10805, abstract, reformulation (3)), for callers whose
+ * parameters stay fixed over many calls (inference).  adjoint = 0 gives the
+ * forward block; adjoint = 1 the backward-data block (every kernel flipped,
+ * no bias; b0 may then be NULL).  folded: caller-owned device memory of at
+ * least wtconv_folded_size bytes, 16-byte aligned, overwritten.  One kernel
+ * launch, asynchronous on `stream`.  Errors as for wtconv_forward;
+ * WTCONV_ERR_WORKSPACE when folded_bytes is too small, WTCONV_ERR_ARG for an
+ * adjoint flag other than 0 or 1. */
+wtconv_status wtconv_fold_weights(const wtconv_desc* desc, const float* w0,
+                                  const float* b0, const float* s0,
+                                  const float* wl, const float* sl,
+                                  int adjoint, void* folded,
+                                  size_t folded_bytes, void* stream);
+
+/* The forward pass over a block from wtconv_fold_weights: y equals what
+ * wtconv_forward gives for the same parameters, bit for bit, without the
+ * folding launch, so that planes held whole in one SM take one kernel
+ * launch (row-band planes with L >= 2 take two: the deep levels, then the
+ * output).  Given an adjoint block and dy in place of x, it computes the
+ * backward-data pass dx.  x, y: NCHW device memory, 16-byte aligned; the
+ * block is only read.  Needs wtconv_workspace_size(desc, 4) bytes of ws
+ * (the status header and, for L >= 2, the level >= 2 synthesis). */
+wtconv_status wtconv_forward_folded(const wtconv_desc* desc, const void* x,
+                                    const void* folded, void* y, void* ws,
+                                    size_t ws_bytes, void* stream);
 
 /* Number of kernel launches one call of operation `op` makes for `desc`
  * (the plan the library picks for the shape on sm_100a), so that a caller

@@ -90,6 +90,45 @@ def test_kernel_launch_counts(lib):
     assert n(whole, 7) == 0
 
 
+def test_folded_block_size_and_launches(lib):
+    """The folded block: per channel k*k padded to 4, then the bias slot (4
+    floats), then 4 padded kernels per level.  forward_folded launches the
+    data pass alone (output kernel; deep kernel first for row-band planes
+    with L >= 2); folding is one launch; its workspace is the status header
+    plus the level >= 2 synthesis."""
+    d = _desc()
+    assert lib.wtconv_folded_size(ctypes.byref(d)) == 3 * ((1 + 4 * 2) * 28 + 4) * 4
+    assert lib.wtconv_folded_size(ctypes.byref(_desc(L=0, k=3))) == 3 * (12 + 4) * 4
+    assert lib.wtconv_folded_size(ctypes.byref(_desc(k=4))) == 0
+    assert lib.wtconv_workspace_size(ctypes.byref(d), 4) == 16 + 2 * 3 * 8 * 8 * 4
+    assert lib.wtconv_workspace_size(ctypes.byref(_desc(L=1)), 4) == 16
+    n = lambda d, op: lib.wtconv_kernel_launches(ctypes.byref(d), op)
+    assert n(_lib.WTConvDesc(32, 96, 56, 56, 5, 3, 0), 4) == 1
+    assert n(_lib.WTConvDesc(16, 64, 256, 256, 5, 5, 1), 4) == 2
+    assert n(_lib.WTConvDesc(16, 64, 256, 256, 5, 5, 1), 5) == 1
+
+
+def test_fold_and_forward_folded_checks(lib):
+    d = _desc()
+    need = lib.wtconv_folded_size(ctypes.byref(d))
+    f = lib.wtconv_fold_weights
+    assert f(ctypes.byref(_desc(k=4)), FAKE, FAKE, FAKE, FAKE, FAKE, 0, FAKE, need, None) == ARG
+    assert f(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, 2, FAKE, need, None) == ARG
+    assert f(ctypes.byref(d), FAKE, None, FAKE, FAKE, FAKE, 0, FAKE, need, None) == ARG  # forward needs b0
+    assert f(ctypes.byref(d), FAKE, FAKE, FAKE, None, FAKE, 0, FAKE, need, None) == ARG
+    assert f(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, 0, None, need, None) == ARG
+    assert f(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, 0, FAKE + 4, need, None) == ALIGN
+    assert f(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, 0, FAKE, need - 4, None) == WS
+    g = lib.wtconv_forward_folded
+    ws = lib.wtconv_workspace_size(ctypes.byref(d), 4)
+    assert g(ctypes.byref(_desc(H=18, L=2)), FAKE, FAKE, FAKE, FAKE, ws, None) == SHAPE
+    assert g(ctypes.byref(d), None, FAKE, FAKE, FAKE, ws, None) == ARG
+    assert g(ctypes.byref(d), FAKE, None, FAKE, FAKE, ws, None) == ARG
+    assert g(ctypes.byref(d), FAKE, FAKE + 8, FAKE, FAKE, ws, None) == ALIGN
+    assert g(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, ws - 4, None) == WS
+    assert g(ctypes.byref(d), FAKE, FAKE, FAKE, None, ws, None) == WS
+
+
 def _fwd(lib, d, x=FAKE, y=FAKE, w0=FAKE, b0=FAKE, s0=FAKE, wl=FAKE, sl=FAKE, ws=FAKE, nws=1 << 30):
     return lib.wtconv_forward(ctypes.byref(d) if d is not None else None, x, w0, b0, s0, wl, sl, y, ws, nws, None)
 
