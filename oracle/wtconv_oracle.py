@@ -23,6 +23,13 @@ What it computes (the plain, unfused definition of the layer):
   * t = 0; for l = L..1: t = IWT(Z_l with t added to its LL band)
   * Y = Ybase + t
 
+Planes whose sides are not divisible by 2^L: the pages are silent.  Reading
+taken here: at every level the plane entering the analysis (X, then the raw
+LL band) gets one zero row at the bottom and / or one zero column at the
+right when that side is odd, and the synthesis output of that level is
+cropped back to the size the plane had before the padding.  With even sides
+throughout this is the plain definition above.
+
 The backward pass is the hand-derived adjoint of those steps in reverse order
 (IWT^T = Haar and Haar^T = IWT because the +-1/2 Haar is orthonormal;
 dwconv^T is the correlation with the spatially flipped kernel).
@@ -122,9 +129,21 @@ def _check(X, W0, Wl, L):
     N, C, H, W = X.shape
     k = W0.shape[-1]
     assert k % 2 == 1 and W0.shape == (C, k, k)
-    assert H % (1 << L) == 0 and W % (1 << L) == 0
     if L:
         assert Wl.shape == (L, C, 4, k, k)
+
+
+def pad_even(A):
+    """Zero row at the bottom / zero column at the right of the last two
+    axes where that side is odd (the plane entering one analysis level)."""
+    h, w = A.shape[-2:]
+    pad = [(0, 0)] * (A.ndim - 2) + [(0, h % 2), (0, w % 2)]
+    return np.pad(A, pad)
+
+
+def crop(A, shape):
+    """The top-left shape[0] x shape[1] corner of the last two axes."""
+    return A[..., :shape[0], :shape[1]]
 
 
 def forward(X, W0, b0, s0, Wl, sl, return_intermediates=False):
@@ -138,10 +157,11 @@ def forward(X, W0, b0, s0, Wl, sl, return_intermediates=False):
     _check(X, W0, Wl, L)
     base_pre = dwconv(X, W0[None]) + b0[None, :, None, None]
     Y = s0[None, :, None, None] * base_pre
-    subs, convs = [], []
+    subs, convs, shapes = [], [], []
     cur = X
     for l in range(L):
-        sub = haar_analysis(cur)                 # [N, C, 4, h, w]
+        shapes.append(cur.shape[-2:])            # size before this level's padding
+        sub = haar_analysis(pad_even(cur))       # [N, C, 4, h, w]
         conv = dwconv(sub, Wl[l][None])          # unscaled level conv
         subs.append(sub)
         convs.append(conv)
@@ -152,11 +172,11 @@ def forward(X, W0, b0, s0, Wl, sl, return_intermediates=False):
         if t is not None:
             Z = Z.copy()
             Z[:, :, 0] += t
-        t = haar_synthesis(Z)
+        t = crop(haar_synthesis(Z), shapes[l])
     if t is not None:
         Y = Y + t
     if return_intermediates:
-        return Y, dict(base_pre=base_pre, subs=subs, convs=convs)
+        return Y, dict(base_pre=base_pre, subs=subs, convs=convs, shapes=shapes)
     return Y
 
 
@@ -169,7 +189,7 @@ def backward(X, dY, W0, b0, s0, Wl, sl):
     """
     L = 0 if Wl is None else Wl.shape[0]
     _, inter = forward(X, W0, b0, s0, Wl, sl, return_intermediates=True)
-    base_pre, subs, convs = inter["base_pre"], inter["subs"], inter["convs"]
+    base_pre, subs, convs, shapes = inter["base_pre"], inter["subs"], inter["convs"], inter["shapes"]
     k = W0.shape[-1]
 
     # base branch: Y += s0 * base_pre
@@ -179,11 +199,12 @@ def backward(X, dY, W0, b0, s0, Wl, sl):
     dW0 = dwcorr_weight(X, dbase, k)
     dX = dwconv(dbase, W0[None, :, ::-1, ::-1])
 
-    # synthesis cascade, reversed: t_{l-1} = IWT(Z_l + t_l on LL)
+    # synthesis cascade, reversed: t_{l-1} = crop(IWT(Z_l + t_l on LL));
+    # crop^T pads with zeros, IWT^T = Haar
     dZ = []
     dt = dY
     for l in range(L):
-        g = haar_analysis(dt)                    # IWT^T
+        g = haar_analysis(pad_even(dt))
         dZ.append(g)
         dt = g[:, :, 0]
     dWl = np.zeros_like(Wl) if L else None
@@ -194,14 +215,15 @@ def backward(X, dY, W0, b0, s0, Wl, sl):
         dconv = sl[l][None, :, :, None, None] * dZ[l]
         dWl[l] = dwcorr_weight(subs[l], dconv, k)
         dsub.append(dwconv(dconv, Wl[l][None, :, :, ::-1, ::-1]))
-    # analysis chain, reversed: sub_l = Haar(cur_{l-1}), cur_l = sub_l[LL]
+    # analysis chain, reversed: sub_l = Haar(pad(cur_{l-1})), cur_l = sub_l[LL];
+    # Haar^T = IWT, pad^T crops
     dcur = None
     for l in reversed(range(L)):
         g = dsub[l]
         if dcur is not None:
             g = g.copy()
             g[:, :, 0] += dcur
-        dcur = haar_synthesis(g)                 # Haar^T
+        dcur = crop(haar_synthesis(g), shapes[l])
     if dcur is not None:
         dX = dX + dcur
     return dict(dX=dX, dW0=dW0, db0=db0, ds0=ds0, dWl=dWl, dsl=dsl)

@@ -357,3 +357,126 @@ def test_regression_fixture_tiny_workload():
         arr = outs[key].reshape(-1)
         np.testing.assert_allclose(arr[entry["index"]], entry["value"], rtol=1e-12, atol=1e-12, err_msg=key)
         assert abs(float(np.sum(arr)) - entry["sum"]) <= 1e-9 * max(1.0, abs(entry["sum"]))
+
+
+# ------------------------------------------- sides not multiples of 2^L
+# The pages are silent on such sides; the oracle pads each level's plane to
+# even sides with zeros (bottom, right) and crops each level's synthesis back.
+
+RAGGED = [(2, 3, 13, 11, 5, 2), (1, 2, 7, 9, 3, 3), (2, 2, 5, 6, 3, 1), (1, 3, 9, 14, 1, 2), (1, 2, 3, 3, 3, 3)]
+
+
+def torch_wtconv_ragged(X, W0, b0, s0, Wl, sl):
+    """The layer with per-level padding composed from library routines
+    (F.pad, grouped conv2d, conv_transpose2d and slicing), differentiated by
+    autograd."""
+    C = X.shape[1]
+    k = W0.shape[-1]
+    L = 0 if Wl is None else Wl.shape[0]
+    h = 0.5
+    filt = torch.tensor([[[h, h], [h, h]], [[h, h], [-h, -h]], [[h, -h], [h, -h]], [[h, -h], [-h, h]]],
+                        dtype=X.dtype).repeat(C, 1, 1).unsqueeze(1)
+    Y = s0.view(1, C, 1, 1) * F.conv2d(X, W0.unsqueeze(1), b0, padding=k // 2, groups=C)
+    cur, Zs, sizes = X, [], []
+    for l in range(L):
+        H, W = cur.shape[-2:]
+        sizes.append((H, W))
+        sub = F.conv2d(F.pad(cur, (0, W % 2, 0, H % 2)), filt, stride=2, groups=C)
+        Zs.append(F.conv2d(sub, Wl[l].reshape(4 * C, 1, k, k), padding=k // 2, groups=4 * C)
+                  * sl[l].reshape(1, 4 * C, 1, 1))
+        cur = sub[:, 0::4]
+    t = None
+    for l in reversed(range(L)):
+        Z = Zs[l]
+        if t is not None:
+            Z = Z.clone()
+            Z[:, 0::4] = Z[:, 0::4] + t
+        H, W = sizes[l]
+        t = F.conv_transpose2d(Z, filt, stride=2, groups=C)[..., :H, :W]
+    return Y if t is None else Y + t
+
+
+@pytest.mark.parametrize("shape", RAGGED)
+def test_ragged_torch_composition_matches_forward_and_all_gradients(shape):
+    N, C, H, W, k, L = shape
+    p = _params(N, C, H, W, k, L, seed=11)
+    t = {key: (None if v is None else torch.tensor(v, requires_grad=True)) for key, v in p.items()}
+    Yt = torch_wtconv_ragged(t["X"], t["W0"], t["b0"], t["s0"], t["Wl"], t["sl"])
+    Y = oracle.forward(p["X"], p["W0"], p["b0"], p["s0"], p["Wl"], p["sl"])
+    assert Y.shape == (N, C, H, W)
+    np.testing.assert_allclose(Y, Yt.detach().numpy(), rtol=0, atol=1e-10)
+    (Yt * torch.from_numpy(p["dY"])).sum().backward()
+    g = oracle.backward(p["X"], p["dY"], p["W0"], p["b0"], p["s0"], p["Wl"], p["sl"])
+    for gk, tk in [("dX", "X"), ("dW0", "W0"), ("db0", "b0"), ("ds0", "s0"), ("dWl", "Wl"), ("dsl", "sl")]:
+        np.testing.assert_allclose(g[gk], t[tk].grad.numpy(), rtol=0, atol=1e-10, err_msg=gk)
+
+
+@pytest.mark.parametrize("shape", [(2, 3, 13, 11), (1, 2, 7, 5), (1, 1, 3, 9)])
+def test_ragged_delta_kernels_reproduce_zero_padded_block_means(shape):
+    """Delta kernels, b0 = 0, equal band scales: Y = s0 X + sum_l s_l U_{l-1}(X)
+    with U_m the mean over the aligned 2^m x 2^m block, pixels outside the
+    image counting as zeros (brute force over each block)."""
+    N, C, H, W = shape
+    L, k = 3, 3
+    X = rng.standard_normal((N, C, H, W))
+    W0 = np.zeros((C, k, k)); W0[:, 1, 1] = 1.0
+    Wl = np.zeros((L, C, 4, k, k)); Wl[:, :, :, 1, 1] = 1.0
+    s0 = rng.uniform(0.5, 1.5, C)
+    sc = rng.uniform(0.5, 1.5, (L, C))
+    Y = oracle.forward(X, W0, np.zeros(C), s0, Wl, np.repeat(sc[:, :, None], 4, axis=2))
+    ref = s0[None, :, None, None] * X
+    for l in range(1, L + 1):
+        b = 1 << (l - 1)
+        U = np.zeros_like(X)
+        for i in range(H):
+            for j in range(W):
+                i0, j0 = i // b * b, j // b * b
+                U[:, :, i, j] = X[:, :, i0:i0 + b, j0:j0 + b].sum(axis=(2, 3)) / (b * b)
+        ref = ref + sc[l - 1][None, :, None, None] * U
+    np.testing.assert_allclose(Y, ref, rtol=0, atol=1e-12)
+
+
+def test_ragged_adjoint_dot_product_and_finite_differences():
+    p = _params(N=2, C=2, H=11, W=7, k=3, L=2, seed=13)
+    Y = oracle.forward(p["X"], p["W0"], p["b0"], p["s0"], p["Wl"], p["sl"])
+    Y0 = oracle.forward(np.zeros_like(p["X"]), p["W0"], p["b0"], p["s0"], p["Wl"], p["sl"])
+    g = oracle.backward(p["X"], p["dY"], p["W0"], p["b0"], p["s0"], p["Wl"], p["sl"])
+    lhs, rhs = np.sum((Y - Y0) * p["dY"]), np.sum(p["X"] * g["dX"])
+    assert abs(lhs - rhs) < 1e-10 * max(1.0, abs(lhs))
+
+    def loss(q):
+        return float(np.sum(oracle.forward(q["X"], q["W0"], q["b0"], q["s0"], q["Wl"], q["sl"]) * p["dY"]))
+
+    h = 1e-6
+    fd_rng = np.random.default_rng(17)
+    for name, gname in [("X", "dX"), ("W0", "dW0"), ("s0", "ds0"), ("Wl", "dWl"), ("sl", "dsl")]:
+        flat = p[name].reshape(-1)
+        for idx in fd_rng.choice(flat.size, size=min(4, flat.size), replace=False):
+            q = {key: (None if v is None else v.copy()) for key, v in p.items()}
+            q[name].reshape(-1)[idx] += h
+            lp = loss(q)
+            q[name].reshape(-1)[idx] -= 2 * h
+            fd = (lp - loss(q)) / (2 * h)
+            an = g[gname].reshape(-1)[idx]
+            assert abs(fd - an) <= 1e-6 * max(1.0, abs(an)), (name, idx, fd, an)
+
+
+@pytest.mark.parametrize("shape", RAGGED)
+def test_ragged_equals_one_padding_to_multiples_of_2L(shape):
+    """Zero-padding X once to multiples of 2^L (bottom, right), running the
+    layer on the padded planes and cropping gives the per-level reading's
+    output; dY zero-padded the same way gives its gradients (dX cropped).
+    This is how the CUDA library computes such sides."""
+    N, C, H, W, k, L = shape
+    p = _params(N, C, H, W, k, L, seed=19)
+    m = 1 << L
+    Hp, Wp = -(-H // m) * m, -(-W // m) * m
+    pad = lambda A: np.pad(A, [(0, 0), (0, 0), (0, Hp - H), (0, Wp - W)])
+    Y = oracle.forward(p["X"], p["W0"], p["b0"], p["s0"], p["Wl"], p["sl"])
+    Yp = oracle.forward(pad(p["X"]), p["W0"], p["b0"], p["s0"], p["Wl"], p["sl"])
+    np.testing.assert_allclose(Yp[:, :, :H, :W], Y, rtol=0, atol=1e-12)
+    g = oracle.backward(p["X"], p["dY"], p["W0"], p["b0"], p["s0"], p["Wl"], p["sl"])
+    gp = oracle.backward(pad(p["X"]), pad(p["dY"]), p["W0"], p["b0"], p["s0"], p["Wl"], p["sl"])
+    np.testing.assert_allclose(gp["dX"][:, :, :H, :W], g["dX"], rtol=0, atol=1e-12)
+    for key in ("dW0", "db0", "ds0", "dWl", "dsl"):
+        np.testing.assert_allclose(gp[key], g[key], rtol=0, atol=1e-11, err_msg=key)
