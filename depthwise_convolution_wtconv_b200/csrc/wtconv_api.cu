@@ -310,10 +310,55 @@ wtconv_status check_desc(const wtconv_desc* d) {
   if (d->L < 0 || d->L > WTCONV_MAX_LEVELS) return WTCONV_ERR_ARG;
   if (d->N <= 0 || d->C <= 0 || d->H <= 0 || d->W <= 0) return WTCONV_ERR_ARG;
   if (d->io != WTCONV_F32 && d->io != WTCONV_BF16) return WTCONV_ERR_ARG;
-  if ((long long)d->H * d->W > (1LL << 30) || (long long)d->N * d->C > (1LL << 30)) return WTCONV_ERR_ARG;
-  const int m = 1 << d->L;
-  if ((d->H % m) != 0 || (d->W % m) != 0) return WTCONV_ERR_SHAPE;
+  const long long m = 1LL << d->L;
+  const long long Hp = (d->H + m - 1) / m * m, Wp = (d->W + m - 1) / m * m;
+  if (Hp * Wp > (1LL << 30) || (long long)d->N * d->C > (1LL << 30)) return WTCONV_ERR_ARG;
   return WTCONV_OK;
+}
+
+// Sides not multiples of 2^L: the passes run on zero-padded copies of the
+// planes (the padded descriptor) in the workspace, and outputs are cropped.
+bool ragged(const wtconv_desc* d) {
+  const int m = 1 << d->L;
+  return (d->H % m) != 0 || (d->W % m) != 0;
+}
+wtconv_desc padded(const wtconv_desc* d) {
+  wtconv_desc p = *d;
+  const int m = 1 << d->L;
+  p.H = (d->H + m - 1) / m * m;
+  p.W = (d->W + m - 1) / m * m;
+  return p;
+}
+size_t rup16(size_t b) { return (b + 15) / 16 * 16; }
+// bytes of one padded activation tensor in the workspace
+size_t act_bytes(const wtconv_desc* p) {
+  return rup16((size_t)p->N * p->C * p->H * p->W * (p->io == WTCONV_BF16 ? 2 : 4));
+}
+
+wtconv_status launch_pad_crop(const wtconv_desc* d, const wtconv_desc* p, const void* src, void* dst, bool pad,
+                              cudaStream_t st) {
+  const long long planes = (long long)d->N * d->C;
+  const int per = pad ? p->H * p->W : d->H * d->W;
+  const int cpp = (per + PADC - 1) / PADC;
+  const int grid = (int)std::min<long long>(planes * cpp, 148LL * 8);
+  const FDiv f = make_fdiv(pad ? p->W : d->W);
+  if (d->io == WTCONV_F32) {
+    if (pad)
+      wtconv_pad_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float*>(src), static_cast<float*>(dst), d->H,
+                                                     d->W, p->H, p->W, f, planes, cpp);
+    else
+      wtconv_crop_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float*>(src), static_cast<float*>(dst), d->H,
+                                                      d->W, p->H, p->W, f, planes, cpp);
+  } else {
+    using B = __nv_bfloat16;
+    if (pad)
+      wtconv_pad_kernel<B><<<grid, 256, 0, st>>>(static_cast<const B*>(src), static_cast<B*>(dst), d->H, d->W, p->H,
+                                                 p->W, f, planes, cpp);
+    else
+      wtconv_crop_kernel<B><<<grid, 256, 0, st>>>(static_cast<const B*>(src), static_cast<B*>(dst), d->H, d->W, p->H,
+                                                  p->W, f, planes, cpp);
+  }
+  return cudaGetLastError() == cudaSuccess ? WTCONV_OK : WTCONV_ERR_CUDA;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -980,8 +1025,11 @@ using namespace wt;
 
 extern "C" {
 
-size_t wtconv_workspace_size(const wtconv_desc* desc, int op) {
-  if (check_desc(desc) != WTCONV_OK) return 0;
+}  // extern "C"
+
+namespace {
+// workspace of `op` for sides that are multiples of 2^L
+size_t op_ws(const wtconv_desc* desc, int op) {
   switch (op) {
     case WTCONV_OP_FORWARD:
     case WTCONV_OP_BACKWARD_DATA:
@@ -995,6 +1043,26 @@ size_t wtconv_workspace_size(const wtconv_desc* desc, int op) {
     default:
       return 0;
   }
+}
+
+// padded activation tensors a ragged call of `op` keeps in its workspace:
+// input and output (both backward passes: x, dy and dx)
+int op_acts(int op) { return op == WTCONV_OP_BACKWARD ? 3 : 2; }
+
+// Ragged shapes: the workspace of the padded shape, then the padded
+// activations, each 16-byte aligned.  Returns the i-th one.
+void* act_slot(const wtconv_desc* p, int op, void* ws, int i) {
+  return static_cast<char*>(ws) + rup16(op_ws(p, op)) + (size_t)i * act_bytes(p);
+}
+}  // namespace
+
+extern "C" {
+
+size_t wtconv_workspace_size(const wtconv_desc* desc, int op) {
+  if (check_desc(desc) != WTCONV_OK || op < 0 || op > WTCONV_OP_FORWARD_FOLDED) return 0;
+  if (!ragged(desc)) return op_ws(desc, op);
+  const wtconv_desc p = padded(desc);
+  return rup16(op_ws(&p, op)) + (size_t)op_acts(op) * act_bytes(&p);
 }
 
 size_t wtconv_folded_size(const wtconv_desc* desc) {
@@ -1021,8 +1089,16 @@ wtconv_status wtconv_forward_folded(const wtconv_desc* desc, const void* x, cons
   if (e != WTCONV_OK) return e;
   if (!x || !y || !folded) return WTCONV_ERR_ARG;
   if (!aligned16(x) || !aligned16(y) || !aligned16(folded)) return WTCONV_ERR_ALIGN;
-  if ((e = check_ws(ws, ws_bytes, 16 + t1_bytes(desc))) != WTCONV_OK) return e;
-  return run_folded(desc, x, static_cast<const float*>(folded), y, ws, static_cast<cudaStream_t>(stream));
+  if ((e = check_ws(ws, ws_bytes, wtconv_workspace_size(desc, WTCONV_OP_FORWARD_FOLDED))) != WTCONV_OK) return e;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const float* wf = static_cast<const float*>(folded);
+  if (!ragged(desc)) return run_folded(desc, x, wf, y, ws, st);
+  const wtconv_desc p = padded(desc);
+  void* xp = act_slot(&p, WTCONV_OP_FORWARD_FOLDED, ws, 0);
+  void* yp = act_slot(&p, WTCONV_OP_FORWARD_FOLDED, ws, 1);
+  if ((e = launch_pad_crop(desc, &p, x, xp, true, st)) != WTCONV_OK) return e;
+  if ((e = run_folded(&p, xp, wf, yp, ws, st)) != WTCONV_OK) return e;
+  return launch_pad_crop(desc, &p, yp, y, false, st);
 }
 
 wtconv_status wtconv_forward(const wtconv_desc* desc, const void* x, const float* w0, const float* b0,
@@ -1033,8 +1109,15 @@ wtconv_status wtconv_forward(const wtconv_desc* desc, const void* x, const float
   if (!x || !y) return WTCONV_ERR_ARG;
   if ((e = check_params(desc, w0, b0, s0, wl, sl, true)) != WTCONV_OK) return e;
   if (!aligned16(x) || !aligned16(y)) return WTCONV_ERR_ALIGN;
-  if ((e = check_ws(ws, ws_bytes, fwd_ws_bytes(desc))) != WTCONV_OK) return e;
-  return run_forward(desc, x, w0, b0, s0, wl, sl, y, 0, ws, static_cast<cudaStream_t>(stream));
+  if ((e = check_ws(ws, ws_bytes, wtconv_workspace_size(desc, WTCONV_OP_FORWARD))) != WTCONV_OK) return e;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (!ragged(desc)) return run_forward(desc, x, w0, b0, s0, wl, sl, y, 0, ws, st);
+  const wtconv_desc p = padded(desc);
+  void* xp = act_slot(&p, WTCONV_OP_FORWARD, ws, 0);
+  void* yp = act_slot(&p, WTCONV_OP_FORWARD, ws, 1);
+  if ((e = launch_pad_crop(desc, &p, x, xp, true, st)) != WTCONV_OK) return e;
+  if ((e = run_forward(&p, xp, w0, b0, s0, wl, sl, yp, 0, ws, st)) != WTCONV_OK) return e;
+  return launch_pad_crop(desc, &p, yp, y, false, st);
 }
 
 wtconv_status wtconv_backward_data(const wtconv_desc* desc, const void* dy, const float* w0, const float* s0,
@@ -1045,8 +1128,15 @@ wtconv_status wtconv_backward_data(const wtconv_desc* desc, const void* dy, cons
   if (!dy || !dx) return WTCONV_ERR_ARG;
   if ((e = check_params(desc, w0, nullptr, s0, wl, sl, false)) != WTCONV_OK) return e;
   if (!aligned16(dy) || !aligned16(dx)) return WTCONV_ERR_ALIGN;
-  if ((e = check_ws(ws, ws_bytes, fwd_ws_bytes(desc))) != WTCONV_OK) return e;
-  return run_forward(desc, dy, w0, nullptr, s0, wl, sl, dx, 1, ws, static_cast<cudaStream_t>(stream));
+  if ((e = check_ws(ws, ws_bytes, wtconv_workspace_size(desc, WTCONV_OP_BACKWARD_DATA))) != WTCONV_OK) return e;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (!ragged(desc)) return run_forward(desc, dy, w0, nullptr, s0, wl, sl, dx, 1, ws, st);
+  const wtconv_desc p = padded(desc);
+  void* dyp = act_slot(&p, WTCONV_OP_BACKWARD_DATA, ws, 0);
+  void* dxp = act_slot(&p, WTCONV_OP_BACKWARD_DATA, ws, 1);
+  if ((e = launch_pad_crop(desc, &p, dy, dyp, true, st)) != WTCONV_OK) return e;
+  if ((e = run_forward(&p, dyp, w0, nullptr, s0, wl, sl, dxp, 1, ws, st)) != WTCONV_OK) return e;
+  return launch_pad_crop(desc, &p, dxp, dx, false, st);
 }
 
 wtconv_status wtconv_backward_weight(const wtconv_desc* desc, const void* x, const void* dy, const float* w0,
@@ -1059,9 +1149,15 @@ wtconv_status wtconv_backward_weight(const wtconv_desc* desc, const void* x, con
   if ((e = check_params(desc, w0, b0, s0, wl, sl, true)) != WTCONV_OK) return e;
   if ((e = check_grad_outputs(desc, dw0, db0, ds0, dwl, dsl)) != WTCONV_OK) return e;
   if (!aligned16(x) || !aligned16(dy)) return WTCONV_ERR_ALIGN;
-  if ((e = check_ws(ws, ws_bytes, bwdw_ws_bytes(desc))) != WTCONV_OK) return e;
-  return run_bwdw(desc, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, ws,
-                  static_cast<cudaStream_t>(stream));
+  if ((e = check_ws(ws, ws_bytes, wtconv_workspace_size(desc, WTCONV_OP_BACKWARD_WEIGHT))) != WTCONV_OK) return e;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (!ragged(desc)) return run_bwdw(desc, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, ws, st);
+  const wtconv_desc p = padded(desc);
+  void* xp = act_slot(&p, WTCONV_OP_BACKWARD_WEIGHT, ws, 0);
+  void* dyp = act_slot(&p, WTCONV_OP_BACKWARD_WEIGHT, ws, 1);
+  if ((e = launch_pad_crop(desc, &p, x, xp, true, st)) != WTCONV_OK) return e;
+  if ((e = launch_pad_crop(desc, &p, dy, dyp, true, st)) != WTCONV_OK) return e;
+  return run_bwdw(&p, xp, dyp, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, ws, st);
 }
 
 wtconv_status wtconv_backward(const wtconv_desc* desc, const void* x, const void* dy, const float* w0,
@@ -1076,9 +1172,20 @@ wtconv_status wtconv_backward(const wtconv_desc* desc, const void* x, const void
   if (!aligned16(x) || !aligned16(dy) || !aligned16(dx)) return WTCONV_ERR_ALIGN;
   if ((e = check_ws(ws, ws_bytes, wtconv_workspace_size(desc, WTCONV_OP_BACKWARD))) != WTCONV_OK) return e;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  e = run_forward(desc, dy, w0, nullptr, s0, wl, sl, dx, 1, ws, st);
-  if (e != WTCONV_OK) return e;
-  return run_bwdw(desc, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, ws, st);
+  if (!ragged(desc)) {
+    e = run_forward(desc, dy, w0, nullptr, s0, wl, sl, dx, 1, ws, st);
+    if (e != WTCONV_OK) return e;
+    return run_bwdw(desc, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, ws, st);
+  }
+  const wtconv_desc p = padded(desc);
+  void* xp = act_slot(&p, WTCONV_OP_BACKWARD, ws, 0);
+  void* dyp = act_slot(&p, WTCONV_OP_BACKWARD, ws, 1);
+  void* dxp = act_slot(&p, WTCONV_OP_BACKWARD, ws, 2);
+  if ((e = launch_pad_crop(desc, &p, dy, dyp, true, st)) != WTCONV_OK) return e;
+  if ((e = run_forward(&p, dyp, w0, nullptr, s0, wl, sl, dxp, 1, ws, st)) != WTCONV_OK) return e;
+  if ((e = launch_pad_crop(desc, &p, dxp, dx, false, st)) != WTCONV_OK) return e;
+  if ((e = launch_pad_crop(desc, &p, x, xp, true, st)) != WTCONV_OK) return e;
+  return run_bwdw(&p, xp, dyp, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, ws, st);
 }
 
 // ------------------------------------------------------------------------
@@ -1127,6 +1234,7 @@ wtconv_status wtconv_backward_weight_noalloc(const wtconv_desc* desc, const void
   if ((e = check_params(desc, w0, b0, s0, wl, sl, true)) != WTCONV_OK) return e;
   if ((e = check_grad_outputs(desc, dw0, db0, ds0, dwl, dsl)) != WTCONV_OK) return e;
   if (!aligned16(x) || !aligned16(dy)) return WTCONV_ERR_ALIGN;
+  if (ragged(desc)) return WTCONV_ERR_SHAPE;  // no workspace for padded copies
   // one group of partial sums is C * V floats; at least one must fit, with
   // the LL planes of the row-band path when the planes need it
   const size_t V = (size_t)desc->k * desc->k * (1 + 4 * desc->L) + 1;
@@ -1152,6 +1260,12 @@ wtconv_status wtconv_backward_weight_noalloc(const wtconv_desc* desc, const void
 
 int wtconv_kernel_launches(const wtconv_desc* desc, int op) {
   if (check_desc(desc) != WTCONV_OK) return 0;
+  if (ragged(desc)) {
+    const wtconv_desc p = padded(desc);
+    const int inner = wtconv_kernel_launches(&p, op);
+    if (inner == 0 || op == WTCONV_OP_FOLD) return inner;
+    return inner + (op == WTCONV_OP_BACKWARD ? 3 : 2);  // pads of the inputs, crop of the output
+  }
   MainPlan M;
   const bool main_ok = build_main_plan(M, desc, PLAN_SMEM);
   const int pass = main_ok ? 1 + ((desc->L >= 2 && !M.fused) ? 1 : 0) : 0;  // [deep], output

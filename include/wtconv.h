@@ -20,6 +20,12 @@
  *       Z_l[c,s] = sl[l][c][s] * dwconv(sub_l[c,s], Wl[l][c][s]); cur = raw LL.
  *   t = 0; for l = L..1: t = IWT(Z_l with t added to its LL band)
  *   Y = Ybase + t
+ *   Sides that are not multiples of 2^L (the paper does not cover them; this
+ *   is the library's reading): at every level an odd side of the plane
+ *   entering the analysis gets one zero row (bottom) or column (right), and
+ *   that level's synthesis output is cropped back to the plane's size.  The
+ *   library computes this on copies of the planes zero-padded to multiples
+ *   of 2^L, which gives the same outputs and gradients, and crops.
  *
  * Layouts (all contiguous, row-major):
  *   x, y, dy, dx : [N][C][H][W] in the I/O dtype (fp32 or bf16)
@@ -41,7 +47,10 @@
  *     forward and backward-data passes keep the folded weights of every
  *     channel and, for L >= 2, the synthesis of levels >= 2 at level-1
  *     resolution (fp32, N*C*(H/2)*(W/2)); the weight-gradient passes keep
- *     their per-CTA partial sums.  The workspace is required.
+ *     their per-CTA partial sums.  For sides that are not multiples of 2^L
+ *     it also holds the zero-padded copies of the call's input and output
+ *     planes (two, or three for wtconv_backward).  The workspace is
+ *     required.
  *   - Arithmetic is fp32 throughout; bf16 I/O is rounded to nearest even on
  *     output.  Results are deterministic run to run (fixed reduction order).
  *   - Gradients are overwritten, not accumulated.
@@ -49,7 +58,9 @@
  *       WTCONV_ERR_ARG       null desc/pointer, k even or outside 1..7,
  *                            L < 0 or L > WTCONV_MAX_LEVELS, N,C,H,W <= 0,
  *                            element counts that overflow 32-bit indexing
- *       WTCONV_ERR_SHAPE     H or W not divisible by 2^L
+ *       WTCONV_ERR_SHAPE     (no-allocation variant only) H or W not a
+ *                            multiple of 2^L: it has no workspace for the
+ *                            padded copies
  *       WTCONV_ERR_ALIGN     a tensor pointer not 16-byte aligned
  *       WTCONV_ERR_WORKSPACE ws_bytes < wtconv_workspace_size(desc, op)
  *       WTCONV_ERR_UNSUPPORTED  the shape needs more on-chip memory than

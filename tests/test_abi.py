@@ -90,6 +90,36 @@ def test_kernel_launch_counts(lib):
     assert n(whole, 7) == 0
 
 
+def test_workspace_of_ragged_sides(lib):
+    """Sides not multiples of 2^L: the workspace of the padded shape (H and W
+    rounded up to multiples of 2^L), then the padded input and output planes
+    (x, dy and dx for both backward passes), each rounded to 16 bytes."""
+    d = _desc(H=18, W=13, L=2)                       # padded to 20 x 16
+    t1 = 2 * 3 * 10 * 8 * 4
+    folded = 3 * ((1 + 4 * 2) * 28 + 4) * 4
+    act = 2 * 3 * 20 * 16 * 4
+    V = 25 * (1 + 4 * 2) + 1
+    fwd = 16 + t1 + folded                           # 5008, a multiple of 16
+    bw = 16 + 2 * 3 * V * 4
+    assert lib.wtconv_workspace_size(ctypes.byref(d), 0) == fwd + 2 * act
+    assert lib.wtconv_workspace_size(ctypes.byref(d), 1) == fwd + 2 * act
+    assert lib.wtconv_workspace_size(ctypes.byref(d), 2) == bw + 2 * act
+    assert lib.wtconv_workspace_size(ctypes.byref(d), 3) == (max(bw, fwd) + 15) // 16 * 16 + 3 * act
+    assert lib.wtconv_workspace_size(ctypes.byref(d), 4) == 16 + t1 + 2 * act
+    bf = _desc(H=7, W=5, L=1, io=1)                  # 8 x 6 bf16: 2*3*8*6*2 = 576 bytes
+    assert lib.wtconv_workspace_size(ctypes.byref(bf), 0) == 16 + 3 * (5 * 28 + 4) * 4 + 2 * 576
+
+
+def test_ragged_launch_counts_and_noalloc(lib):
+    """Ragged sides add the pads of the inputs and the crop of the output;
+    the no-allocation weight gradients refuse them (no room for the copies)."""
+    n = lambda d, op: lib.wtconv_kernel_launches(ctypes.byref(d), op)
+    d = _lib.WTConvDesc(32, 96, 55, 54, 5, 3, 0)      # padded to 56 x 56
+    assert [n(d, op) for op in range(6)] == [4, 4, 4, 7, 3, 1]
+    args = [FAKE] * 12
+    assert lib.wtconv_backward_weight_noalloc(ctypes.byref(d), *args, None) == SHAPE
+
+
 def test_folded_block_size_and_launches(lib):
     """The folded block: per channel k*k padded to 4, then the bias slot (4
     floats), then 4 padded kernels per level.  forward_folded launches the
@@ -121,7 +151,7 @@ def test_fold_and_forward_folded_checks(lib):
     assert f(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, 0, FAKE, need - 4, None) == WS
     g = lib.wtconv_forward_folded
     ws = lib.wtconv_workspace_size(ctypes.byref(d), 4)
-    assert g(ctypes.byref(_desc(H=18, L=2)), FAKE, FAKE, FAKE, FAKE, ws, None) == SHAPE
+    assert g(ctypes.byref(_desc(H=18, L=2)), FAKE, FAKE, FAKE, FAKE, ws, None) == WS  # padded copies need more
     assert g(ctypes.byref(d), None, FAKE, FAKE, FAKE, ws, None) == ARG
     assert g(ctypes.byref(d), FAKE, None, FAKE, FAKE, ws, None) == ARG
     assert g(ctypes.byref(d), FAKE, FAKE + 8, FAKE, FAKE, ws, None) == ALIGN
@@ -136,7 +166,7 @@ def _fwd(lib, d, x=FAKE, y=FAKE, w0=FAKE, b0=FAKE, s0=FAKE, wl=FAKE, sl=FAKE, ws
 @pytest.mark.parametrize("kw,status", [
     (dict(k=4), ARG), (dict(k=9), ARG), (dict(k=0), ARG), (dict(L=-1), ARG), (dict(L=9), ARG),
     (dict(N=0), ARG), (dict(C=-1), ARG), (dict(H=0), ARG), (dict(io=7), ARG),
-    (dict(H=18, L=2), SHAPE), (dict(W=20, L=3), SHAPE), (dict(H=3, W=4, L=1), SHAPE),
+    (dict(H=1 << 16, W=(1 << 14) + 1, L=1), ARG),  # padded plane beyond 32-bit indexing
 ])
 def test_forward_rejects_bad_descriptors(lib, kw, status):
     assert _fwd(lib, _desc(**kw)) == status
@@ -167,7 +197,9 @@ def test_backward_data_checks(lib):
     f = lib.wtconv_backward_data
     assert f(ctypes.byref(d), None, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 30, None) == ARG
     assert f(ctypes.byref(d), FAKE_MIS, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 30, None) == ALIGN
-    assert f(ctypes.byref(_desc(W=10, L=2)), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 30, None) == SHAPE
+    ragged = _desc(W=10, L=2)
+    need = lib.wtconv_workspace_size(ctypes.byref(ragged), 1)
+    assert f(ctypes.byref(ragged), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, need - 16, None) == WS
     assert f(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, 0, None) == WS
 
 

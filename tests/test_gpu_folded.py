@@ -22,6 +22,7 @@ CASES = [
     Workload("rows_L0_k3", 2, 3, 112, 112, 3, 0, "f32"),
     Workload("small_L0_k5", 4, 5, 14, 14, 5, 0, "f32"),
     Workload("L1_k1", 2, 3, 16, 12, 1, 1, "f32"),
+    Workload("ragged_L2", 2, 3, 13, 11, 5, 2, "f32"),
 ]
 
 

@@ -111,6 +111,12 @@ EDGE = [
     Workload("rows_L0_k5_batched", 5, 4, 8, 64, 5, 0, "f32"),
     Workload("rows_L0_k3_reuse", 6, 1000, 8, 64, 3, 0, "f32"),
     Workload("rows_L0_k1", 2, 3, 12, 64, 1, 0, "f32"),
+    # sides not multiples of 2^L (zero-padded copies, cropped results)
+    Workload("ragged_13x11_L2", 2, 3, 13, 11, 5, 2, "f32"),
+    Workload("ragged_7x9_L3_bf16", 1, 2, 7, 9, 3, 3, "bf16"),
+    Workload("ragged_55x54_L3", 2, 3, 55, 54, 5, 3, "f32"),
+    Workload("ragged_bands_250_L2", 1, 2, 250, 246, 5, 2, "bf16"),
+    Workload("ragged_3x3_L3_k1", 2, 2, 3, 3, 1, 3, "f32"),
 ]
 
 
@@ -167,8 +173,9 @@ def test_weight_gradients_deterministic(cuda_ok):
         assert torch.equal(a[k], b[k]), k
 
 
-def test_fused_backward_matches_separate_calls(cuda_ok):
-    wl = Workload("fused", 3, 4, 32, 32, 5, 2, "f32")
+@pytest.mark.parametrize("wl", [Workload("fused", 3, 4, 32, 32, 5, 2, "f32"),
+                                Workload("fused_ragged", 2, 3, 29, 27, 5, 2, "f32")], ids=["even", "ragged"])
+def test_fused_backward_matches_separate_calls(cuda_ok, wl):
     d = _dev(make_inputs(wl, 2), wl.io)
     sep = run_gpu(d)
     dx, g = wt.backward(d["X"], d["dY"], d["W0"], d["b0"], d["s0"], d["Wl"], d["sl"])
@@ -212,8 +219,9 @@ def test_stream_argument_and_preallocated_outputs(cuda_ok):
 
 
 @pytest.mark.parametrize("wl", [Workload("status_whole", 2, 3, 32, 32, 5, 3, "f32"),
-                                Workload("status_bands", 1, 2, 256, 128, 5, 3, "bf16")],
-                         ids=["whole_planes", "row_bands"])
+                                Workload("status_bands", 1, 2, 256, 128, 5, 3, "bf16"),
+                                Workload("status_ragged", 2, 3, 30, 27, 3, 2, "f32")],
+                         ids=["whole_planes", "row_bands", "ragged"])
 def test_status_word_stays_clear(cuda_ok, wl):
     """The workspace header's status word is set only when a bounded wait for
     an asynchronous copy runs out; after ordinary calls of every entry point
