@@ -168,7 +168,7 @@ __global__ void __launch_bounds__(BW_NT, 2) wtconv_bwdw_kernel(const __grid_cons
   // this thread's branch (fixed for the whole CTA)
   int b = 0;
   while (b + 1 < P.nbr && tid >= P.br[b + 1].first) ++b;
-  const BwBranch& B = P.br[b];
+  const BwBranch B = P.br[b];  // by value: registers, not per-use constant loads
   const int lt = tid - B.first;
   const bool busy = tid < P.br[P.nbr - 1].first + P.br[P.nbr - 1].nthr;
   float G[KK];
