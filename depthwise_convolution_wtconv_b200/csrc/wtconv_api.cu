@@ -157,6 +157,8 @@ bool build_main_plan(MainPlan& M, const wtconv_desc* d, int max_smem) {
   M.io_bytes = io_bytes(d);
   M.vec_in = (d->W % 4) == 0;
   M.vec_out = (d->W % 4) == 0;
+  M.oH = d->H;
+  M.oW = d->W;
   M.wblk = main_wblk(d);
   M.bulk_t = d->L >= 2 && (M.W1 % 4) == 0;
   // level-0 fp32 rows of at least 256 bytes go straight to the padded row
@@ -317,7 +319,8 @@ wtconv_status check_desc(const wtconv_desc* d) {
 }
 
 // Sides not multiples of 2^L: the passes run on zero-padded copies of the
-// planes (the padded descriptor) in the workspace, and outputs are cropped.
+// input planes (the padded descriptor) in the workspace; the output kernel
+// stores only the image part of each output plane.
 bool ragged(const wtconv_desc* d) {
   const int m = 1 << d->L;
   return (d->H % m) != 0 || (d->W % m) != 0;
@@ -335,29 +338,20 @@ size_t act_bytes(const wtconv_desc* p) {
   return rup16((size_t)p->N * p->C * p->H * p->W * (p->io == WTCONV_BF16 ? 2 : 4));
 }
 
-wtconv_status launch_pad_crop(const wtconv_desc* d, const wtconv_desc* p, const void* src, void* dst, bool pad,
-                              cudaStream_t st) {
+// Copies the planes of `src` (d's sides) zero-padded into `dst` (p's sides).
+wtconv_status launch_pad(const wtconv_desc* d, const wtconv_desc* p, const void* src, void* dst, cudaStream_t st) {
   const long long planes = (long long)d->N * d->C;
-  const int per = pad ? p->H * p->W : d->H * d->W;
+  const int per = p->H * p->W;
   const int cpp = (per + PADC - 1) / PADC;
   const int grid = (int)std::min<long long>(planes * cpp, 148LL * 8);
-  const FDiv f = make_fdiv(pad ? p->W : d->W);
-  if (d->io == WTCONV_F32) {
-    if (pad)
-      wtconv_pad_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float*>(src), static_cast<float*>(dst), d->H,
-                                                     d->W, p->H, p->W, f, planes, cpp);
-    else
-      wtconv_crop_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float*>(src), static_cast<float*>(dst), d->H,
-                                                      d->W, p->H, p->W, f, planes, cpp);
-  } else {
-    using B = __nv_bfloat16;
-    if (pad)
-      wtconv_pad_kernel<B><<<grid, 256, 0, st>>>(static_cast<const B*>(src), static_cast<B*>(dst), d->H, d->W, p->H,
-                                                 p->W, f, planes, cpp);
-    else
-      wtconv_crop_kernel<B><<<grid, 256, 0, st>>>(static_cast<const B*>(src), static_cast<B*>(dst), d->H, d->W, p->H,
-                                                  p->W, f, planes, cpp);
-  }
+  const FDiv f = make_fdiv(p->W);
+  if (d->io == WTCONV_F32)
+    wtconv_pad_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float*>(src), static_cast<float*>(dst), d->H,
+                                                   d->W, p->H, p->W, f, planes, cpp);
+  else
+    wtconv_pad_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(src),
+                                                           static_cast<__nv_bfloat16*>(dst), d->H, d->W, p->H, p->W,
+                                                           f, planes, cpp);
   return cudaGetLastError() == cudaSuccess ? WTCONV_OK : WTCONV_ERR_CUDA;
 }
 
@@ -462,9 +456,14 @@ wtconv_status launch_fold(const wtconv_desc* d, const Device& dev, const float* 
 // weights `wfold`.
 template <int K, typename IO>
 wtconv_status launch_forward_t(const wtconv_desc* d, const Device& dev, const void* x, const float* wfold, void* y,
-                               int* status, float* t1, cudaStream_t st) {
+                               int* status, float* t1, const wtconv_desc* out, cudaStream_t st) {
   MainPlan M;
   if (!build_main_plan(M, d, dev.max_smem)) return WTCONV_ERR_UNSUPPORTED;
+  if (out) {  // y is the image inside the padded planes x holds
+    M.oH = out->H;
+    M.oW = out->W;
+    M.vec_out = (out->W % 4) == 0;
+  }
   if (d->L >= 2 && !M.fused) {
     DeepPlan D;
     if (!build_deep_plan(D, d, dev.max_smem)) return WTCONV_ERR_UNSUPPORTED;
@@ -504,9 +503,9 @@ wtconv_status launch_forward_t(const wtconv_desc* d, const Device& dev, const vo
 
 template <int K>
 wtconv_status launch_forward_k(const wtconv_desc* d, const Device& dev, const void* x, const float* wfold, void* y,
-                               int* status, float* t1, cudaStream_t st) {
-  if (d->io == WTCONV_F32) return launch_forward_t<K, float>(d, dev, x, wfold, y, status, t1, st);
-  return launch_forward_t<K, __nv_bfloat16>(d, dev, x, wfold, y, status, t1, st);
+                               int* status, float* t1, const wtconv_desc* out, cudaStream_t st) {
+  if (d->io == WTCONV_F32) return launch_forward_t<K, float>(d, dev, x, wfold, y, status, t1, out, st);
+  return launch_forward_t<K, __nv_bfloat16>(d, dev, x, wfold, y, status, t1, out, st);
 }
 
 // Folds the weights into `wfold` (flip = 1: the adjoint's block).
@@ -524,29 +523,32 @@ wtconv_status run_fold(const wtconv_desc* d, const float* w0, const float* b0, c
 }
 
 // The data pass over a folded block.  ws: 16-byte header (status word)
-// followed by t1 when L >= 2.
-wtconv_status run_folded(const wtconv_desc* d, const void* x, const float* wfold, void* y, void* ws, cudaStream_t st) {
+// followed by t1 when L >= 2.  With `out`, x holds zero-padded planes and y
+// receives only the out->H x out->W image of each.
+wtconv_status run_folded(const wtconv_desc* d, const void* x, const float* wfold, void* y, void* ws, cudaStream_t st,
+                         const wtconv_desc* out = nullptr) {
   Device dev;
   wtconv_status e = query_device(dev);
   if (e != WTCONV_OK) return e;
   int* status = static_cast<int*>(ws);
   float* t1 = reinterpret_cast<float*>(static_cast<char*>(ws) + 16);
   switch (d->k) {
-    case 1: return launch_forward_k<1>(d, dev, x, wfold, y, status, t1, st);
-    case 3: return launch_forward_k<3>(d, dev, x, wfold, y, status, t1, st);
-    case 5: return launch_forward_k<5>(d, dev, x, wfold, y, status, t1, st);
-    default: return launch_forward_k<7>(d, dev, x, wfold, y, status, t1, st);
+    case 1: return launch_forward_k<1>(d, dev, x, wfold, y, status, t1, out, st);
+    case 3: return launch_forward_k<3>(d, dev, x, wfold, y, status, t1, out, st);
+    case 5: return launch_forward_k<5>(d, dev, x, wfold, y, status, t1, out, st);
+    default: return launch_forward_k<7>(d, dev, x, wfold, y, status, t1, out, st);
   }
 }
 
 // Forward (flip = 0) or backward-data (flip = 1): the weights are folded into
 // the workspace after t1, then the data pass runs over them.
 wtconv_status run_forward(const wtconv_desc* d, const void* x, const float* w0, const float* b0, const float* s0,
-                          const float* wl, const float* sl, void* y, int flip, void* ws, cudaStream_t st) {
+                          const float* wl, const float* sl, void* y, int flip, void* ws, cudaStream_t st,
+                          const wtconv_desc* out = nullptr) {
   float* wfold = reinterpret_cast<float*>(static_cast<char*>(ws) + 16 + t1_bytes(d));
   wtconv_status e = run_fold(d, w0, b0, s0, wl, sl, flip, wfold, st);
   if (e != WTCONV_OK) return e;
-  return run_folded(d, x, wfold, y, ws, st);
+  return run_folded(d, x, wfold, y, ws, st, out);
 }
 
 // Workspace: a 16-byte header whose first int is the device status word,
@@ -1045,9 +1047,10 @@ size_t op_ws(const wtconv_desc* desc, int op) {
   }
 }
 
-// padded activation tensors a ragged call of `op` keeps in its workspace:
-// input and output (both backward passes: x, dy and dx)
-int op_acts(int op) { return op == WTCONV_OP_BACKWARD ? 3 : 2; }
+// padded input planes a ragged call of `op` keeps in its workspace (x or
+// dy; both for the weight gradients and the fused backward); outputs are
+// written straight into the caller's unpadded tensors
+int op_acts(int op) { return (op == WTCONV_OP_BACKWARD || op == WTCONV_OP_BACKWARD_WEIGHT) ? 2 : 1; }
 
 // Ragged shapes: the workspace of the padded shape, then the padded
 // activations, each 16-byte aligned.  Returns the i-th one.
@@ -1095,10 +1098,8 @@ wtconv_status wtconv_forward_folded(const wtconv_desc* desc, const void* x, cons
   if (!ragged(desc)) return run_folded(desc, x, wf, y, ws, st);
   const wtconv_desc p = padded(desc);
   void* xp = act_slot(&p, WTCONV_OP_FORWARD_FOLDED, ws, 0);
-  void* yp = act_slot(&p, WTCONV_OP_FORWARD_FOLDED, ws, 1);
-  if ((e = launch_pad_crop(desc, &p, x, xp, true, st)) != WTCONV_OK) return e;
-  if ((e = run_folded(&p, xp, wf, yp, ws, st)) != WTCONV_OK) return e;
-  return launch_pad_crop(desc, &p, yp, y, false, st);
+  if ((e = launch_pad(desc, &p, x, xp, st)) != WTCONV_OK) return e;
+  return run_folded(&p, xp, wf, y, ws, st, desc);
 }
 
 wtconv_status wtconv_forward(const wtconv_desc* desc, const void* x, const float* w0, const float* b0,
@@ -1114,10 +1115,8 @@ wtconv_status wtconv_forward(const wtconv_desc* desc, const void* x, const float
   if (!ragged(desc)) return run_forward(desc, x, w0, b0, s0, wl, sl, y, 0, ws, st);
   const wtconv_desc p = padded(desc);
   void* xp = act_slot(&p, WTCONV_OP_FORWARD, ws, 0);
-  void* yp = act_slot(&p, WTCONV_OP_FORWARD, ws, 1);
-  if ((e = launch_pad_crop(desc, &p, x, xp, true, st)) != WTCONV_OK) return e;
-  if ((e = run_forward(&p, xp, w0, b0, s0, wl, sl, yp, 0, ws, st)) != WTCONV_OK) return e;
-  return launch_pad_crop(desc, &p, yp, y, false, st);
+  if ((e = launch_pad(desc, &p, x, xp, st)) != WTCONV_OK) return e;
+  return run_forward(&p, xp, w0, b0, s0, wl, sl, y, 0, ws, st, desc);
 }
 
 wtconv_status wtconv_backward_data(const wtconv_desc* desc, const void* dy, const float* w0, const float* s0,
@@ -1133,10 +1132,8 @@ wtconv_status wtconv_backward_data(const wtconv_desc* desc, const void* dy, cons
   if (!ragged(desc)) return run_forward(desc, dy, w0, nullptr, s0, wl, sl, dx, 1, ws, st);
   const wtconv_desc p = padded(desc);
   void* dyp = act_slot(&p, WTCONV_OP_BACKWARD_DATA, ws, 0);
-  void* dxp = act_slot(&p, WTCONV_OP_BACKWARD_DATA, ws, 1);
-  if ((e = launch_pad_crop(desc, &p, dy, dyp, true, st)) != WTCONV_OK) return e;
-  if ((e = run_forward(&p, dyp, w0, nullptr, s0, wl, sl, dxp, 1, ws, st)) != WTCONV_OK) return e;
-  return launch_pad_crop(desc, &p, dxp, dx, false, st);
+  if ((e = launch_pad(desc, &p, dy, dyp, st)) != WTCONV_OK) return e;
+  return run_forward(&p, dyp, w0, nullptr, s0, wl, sl, dx, 1, ws, st, desc);
 }
 
 wtconv_status wtconv_backward_weight(const wtconv_desc* desc, const void* x, const void* dy, const float* w0,
@@ -1155,8 +1152,8 @@ wtconv_status wtconv_backward_weight(const wtconv_desc* desc, const void* x, con
   const wtconv_desc p = padded(desc);
   void* xp = act_slot(&p, WTCONV_OP_BACKWARD_WEIGHT, ws, 0);
   void* dyp = act_slot(&p, WTCONV_OP_BACKWARD_WEIGHT, ws, 1);
-  if ((e = launch_pad_crop(desc, &p, x, xp, true, st)) != WTCONV_OK) return e;
-  if ((e = launch_pad_crop(desc, &p, dy, dyp, true, st)) != WTCONV_OK) return e;
+  if ((e = launch_pad(desc, &p, x, xp, st)) != WTCONV_OK) return e;
+  if ((e = launch_pad(desc, &p, dy, dyp, st)) != WTCONV_OK) return e;
   return run_bwdw(&p, xp, dyp, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, ws, st);
 }
 
@@ -1180,11 +1177,9 @@ wtconv_status wtconv_backward(const wtconv_desc* desc, const void* x, const void
   const wtconv_desc p = padded(desc);
   void* xp = act_slot(&p, WTCONV_OP_BACKWARD, ws, 0);
   void* dyp = act_slot(&p, WTCONV_OP_BACKWARD, ws, 1);
-  void* dxp = act_slot(&p, WTCONV_OP_BACKWARD, ws, 2);
-  if ((e = launch_pad_crop(desc, &p, dy, dyp, true, st)) != WTCONV_OK) return e;
-  if ((e = run_forward(&p, dyp, w0, nullptr, s0, wl, sl, dxp, 1, ws, st)) != WTCONV_OK) return e;
-  if ((e = launch_pad_crop(desc, &p, dxp, dx, false, st)) != WTCONV_OK) return e;
-  if ((e = launch_pad_crop(desc, &p, x, xp, true, st)) != WTCONV_OK) return e;
+  if ((e = launch_pad(desc, &p, dy, dyp, st)) != WTCONV_OK) return e;
+  if ((e = run_forward(&p, dyp, w0, nullptr, s0, wl, sl, dx, 1, ws, st, desc)) != WTCONV_OK) return e;
+  if ((e = launch_pad(desc, &p, x, xp, st)) != WTCONV_OK) return e;
   return run_bwdw(&p, xp, dyp, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, ws, st);
 }
 
@@ -1264,7 +1259,7 @@ int wtconv_kernel_launches(const wtconv_desc* desc, int op) {
     const wtconv_desc p = padded(desc);
     const int inner = wtconv_kernel_launches(&p, op);
     if (inner == 0 || op == WTCONV_OP_FOLD) return inner;
-    return inner + (op == WTCONV_OP_BACKWARD ? 3 : 2);  // pads of the inputs, crop of the output
+    return inner + op_acts(op);  // the pads of the inputs
   }
   MainPlan M;
   const bool main_ok = build_main_plan(M, desc, PLAN_SMEM);

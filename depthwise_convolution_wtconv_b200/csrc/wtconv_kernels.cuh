@@ -133,14 +133,13 @@ __global__ void wtconv_bwdw_finalize(const FinalizeArgs P, const float* __restri
 
 // Planes whose sides are not multiples of 2^L run on zero-padded copies:
 // zero rows at the bottom and zero columns at the right of every plane up to
-// Hp x Wp (multiples of 2^L), and the result cropped back.  Padding each
+// Hp x Wp (multiples of 2^L); the output kernel then stores only the image.  Padding each
 // level's plane to even sides and cropping each level's synthesis, the
 // reading the layer follows for such sides, gives the same outputs on the
 // image and the same gradients: the extra rows and columns of every level
 // hold zeros or feed only outputs outside the image.
-// Both kernels walk chunks of PADC elements of one plane (the padded plane
-// for the pad, the cropped one for the crop); each thread takes PADC / 256
-// elements of a chunk, issuing its loads before its stores.
+// The pad walks chunks of PADC elements of one padded plane; each thread
+// takes PADC / 256 elements of a chunk, issuing its loads before its stores.
 constexpr int PADC = 1024;
 
 template <typename IO>
@@ -162,32 +161,6 @@ __global__ void __launch_bounds__(256) wtconv_pad_kernel(const IO* __restrict__ 
       if (e < per) {
         const int y = fWp.div(e), x = e - y * Wp;
         if (y < H && x < W) v[k] = s[y * W + x];
-      }
-    }
-#pragma unroll
-    for (int k = 0; k < PADC / 256; ++k)
-      if (c0 + k * 256 < per) d[c0 + k * 256] = v[k];
-  }
-}
-
-template <typename IO>
-__global__ void __launch_bounds__(256) wtconv_crop_kernel(const IO* __restrict__ src, IO* __restrict__ dst, int H,
-                                                          int W, int Hp, int Wp, FDiv fW, long long planes,
-                                                          int cpp) {
-  const int per = H * W;
-  const long long units = planes * cpp;
-  for (long long u = blockIdx.x; u < units; u += gridDim.x) {
-    const long long p = u / cpp;
-    const int c0 = (int)(u - p * cpp) * PADC + threadIdx.x;
-    const IO* s = src + (size_t)p * Hp * Wp;
-    IO* d = dst + (size_t)p * per;
-    IO v[PADC / 256];
-#pragma unroll
-    for (int k = 0; k < PADC / 256; ++k) {
-      const int e = c0 + k * 256;
-      if (e < per) {
-        const int y = fW.div(e), x = e - y * W;
-        v[k] = s[y * Wp + x];
       }
     }
 #pragma unroll

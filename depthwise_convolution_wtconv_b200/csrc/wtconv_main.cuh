@@ -381,12 +381,15 @@ __device__ __forceinline__ void main_out_tile(const MainPlan& P, const float* sl
   } else {
     conv_tile<K, R3, 4>(slot + P.xf.off + j * P.xf.ps + yy0 * P.xf.ld + xx0, P.xf.ld, sw, acc);
   }
-  const int n = P.W - xx0 < 4 ? P.W - xx0 : 4;
-  IO* yp = y + plane_index(P, g, j) * P.H * P.W;
+  // y holds oH x oW planes: the image, or its top-left corner when the
+  // planes were zero-padded to multiples of 2^L
+  const int n = P.oW - xx0 < 4 ? P.oW - xx0 : 4;
+  if (n <= 0) return;
+  IO* yp = y + plane_index(P, g, j) * P.oH * P.oW;
 #pragma unroll
   for (int a = 0; a < R3; ++a) {
     const int yr = g.y0 + yy0 + a;
-    if (yy0 + a < P.TH && yr < P.H) store4(yp + (size_t)yr * P.W + xx0, acc[a], n, P.vec_out != 0);
+    if (yy0 + a < P.TH && yr < P.oH) store4(yp + (size_t)yr * P.oW + xx0, acc[a], n, P.vec_out != 0);
   }
 }
 

@@ -64,6 +64,7 @@ struct MainPlan {
   int R3, tiles, tiles_pp;   // output tile rows (8 or 4; tiles are 4 wide), tiles per unit, per plane
   int bulk_x, bulk_t;        // TMA bulk copies usable for x rows / t1 rows
   int vec_in, vec_out;
+  int oH, oW;                // planes of y: H x W, or the image inside zero-padded planes
   int st_row0, st_rows, st_q, stage_pp;  // staged rows per plane (band), items per plane
   int slot0, slot_floats;    // slot offset (after the header) and size
   int wblk;                  // floats of one channel's folded weights

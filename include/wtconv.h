@@ -24,8 +24,9 @@
  *   is the library's reading): at every level an odd side of the plane
  *   entering the analysis gets one zero row (bottom) or column (right), and
  *   that level's synthesis output is cropped back to the plane's size.  The
- *   library computes this on copies of the planes zero-padded to multiples
- *   of 2^L, which gives the same outputs and gradients, and crops.
+ *   library computes this on copies of the input planes zero-padded to
+ *   multiples of 2^L, which gives the same outputs and gradients, and
+ *   stores only the image part of each output plane.
  *
  * Layouts (all contiguous, row-major):
  *   x, y, dy, dx : [N][C][H][W] in the I/O dtype (fp32 or bf16)
@@ -48,9 +49,8 @@
  *     channel and, for L >= 2, the synthesis of levels >= 2 at level-1
  *     resolution (fp32, N*C*(H/2)*(W/2)); the weight-gradient passes keep
  *     their per-CTA partial sums.  For sides that are not multiples of 2^L
- *     it also holds the zero-padded copies of the call's input and output
- *     planes (two, or three for wtconv_backward).  The workspace is
- *     required.
+ *     it also holds zero-padded copies of the call's input planes (x or dy;
+ *     both for the weight-gradient passes).  The workspace is required.
  *   - Arithmetic is fp32 throughout; bf16 I/O is rounded to nearest even on
  *     output.  Results are deterministic run to run (fixed reduction order).
  *   - Gradients are overwritten, not accumulated.
@@ -229,7 +229,8 @@ wtconv_status wtconv_fold_weights(const wtconv_desc* desc, const float* w0,
  * output).  Given an adjoint block and dy in place of x, it computes the
  * backward-data pass dx.  x, y: NCHW device memory, 16-byte aligned; the
  * block is only read.  Needs wtconv_workspace_size(desc, 4) bytes of ws
- * (the status header and, for L >= 2, the level >= 2 synthesis). */
+ * (the status header, for L >= 2 the level >= 2 synthesis, and for sides
+ * not multiples of 2^L the padded copy of x). */
 wtconv_status wtconv_forward_folded(const wtconv_desc* desc, const void* x,
                                     const void* folded, void* y, void* ws,
                                     size_t ws_bytes, void* stream);

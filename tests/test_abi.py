@@ -92,8 +92,9 @@ def test_kernel_launch_counts(lib):
 
 def test_workspace_of_ragged_sides(lib):
     """Sides not multiples of 2^L: the workspace of the padded shape (H and W
-    rounded up to multiples of 2^L), then the padded input and output planes
-    (x, dy and dx for both backward passes), each rounded to 16 bytes."""
+    rounded up to multiples of 2^L), then the padded input planes (x or dy;
+    both for the weight-gradient passes), each rounded to 16 bytes; outputs
+    go straight to the caller's tensors."""
     d = _desc(H=18, W=13, L=2)                       # padded to 20 x 16
     t1 = 2 * 3 * 10 * 8 * 4
     folded = 3 * ((1 + 4 * 2) * 28 + 4) * 4
@@ -101,21 +102,21 @@ def test_workspace_of_ragged_sides(lib):
     V = 25 * (1 + 4 * 2) + 1
     fwd = 16 + t1 + folded                           # 5008, a multiple of 16
     bw = 16 + 2 * 3 * V * 4
-    assert lib.wtconv_workspace_size(ctypes.byref(d), 0) == fwd + 2 * act
-    assert lib.wtconv_workspace_size(ctypes.byref(d), 1) == fwd + 2 * act
+    assert lib.wtconv_workspace_size(ctypes.byref(d), 0) == fwd + act
+    assert lib.wtconv_workspace_size(ctypes.byref(d), 1) == fwd + act
     assert lib.wtconv_workspace_size(ctypes.byref(d), 2) == bw + 2 * act
-    assert lib.wtconv_workspace_size(ctypes.byref(d), 3) == (max(bw, fwd) + 15) // 16 * 16 + 3 * act
-    assert lib.wtconv_workspace_size(ctypes.byref(d), 4) == 16 + t1 + 2 * act
+    assert lib.wtconv_workspace_size(ctypes.byref(d), 3) == (max(bw, fwd) + 15) // 16 * 16 + 2 * act
+    assert lib.wtconv_workspace_size(ctypes.byref(d), 4) == 16 + t1 + act
     bf = _desc(H=7, W=5, L=1, io=1)                  # 8 x 6 bf16: 2*3*8*6*2 = 576 bytes
-    assert lib.wtconv_workspace_size(ctypes.byref(bf), 0) == 16 + 3 * (5 * 28 + 4) * 4 + 2 * 576
+    assert lib.wtconv_workspace_size(ctypes.byref(bf), 0) == 16 + 3 * (5 * 28 + 4) * 4 + 576
 
 
 def test_ragged_launch_counts_and_noalloc(lib):
-    """Ragged sides add the pads of the inputs and the crop of the output;
-    the no-allocation weight gradients refuse them (no room for the copies)."""
+    """Ragged sides add one pad launch per input; the no-allocation weight
+    gradients refuse them (no room for the copies)."""
     n = lambda d, op: lib.wtconv_kernel_launches(ctypes.byref(d), op)
     d = _lib.WTConvDesc(32, 96, 55, 54, 5, 3, 0)      # padded to 56 x 56
-    assert [n(d, op) for op in range(6)] == [4, 4, 4, 7, 3, 1]
+    assert [n(d, op) for op in range(6)] == [3, 3, 4, 6, 2, 1]
     args = [FAKE] * 12
     assert lib.wtconv_backward_weight_noalloc(ctypes.byref(d), *args, None) == SHAPE
 
