@@ -598,7 +598,8 @@ def run_reference(args, wl, world, rank):
         "impl": "reference", "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 / value, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": wl.name, **{k: v for k, v in wl.as_dict().items() if k != "name"}},
+        "config": {"workload": wl.name, **{k: v for k, v in wl.as_dict().items() if k != "name"},
+                   "global_batch": wl.N, "parallelism": "host (rank 0 only, one core)"},
         "cpu_baseline": {"value": value, "unit": "steps/s", "cores": 1, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
