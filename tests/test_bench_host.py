@@ -1,0 +1,52 @@
+"""Host-side pieces of the benchmark that need no GPU: the algorithmic counts
+behind the roofline, the launch count it reports, and the source hash that
+decides whether the committed DRAM traffic still describes the kernels."""
+import json
+import os
+
+import pytest
+
+import bench
+import depthwise_convolution_wtconv_b200 as wt
+from depthwise_convolution_wtconv_b200.configs import WORKLOADS
+
+
+def test_algorithmic_counts_of_the_stage1_workload():
+    """32x96x56x56, k = 5, L = 3, fp32: per pixel and pass
+    k^2 (1 + (4/3)(1 - 4^-3)) = 25 * 1 + 25 * (4/3) * (63/64) = 57.8125 FMAs;
+    forward bytes = read x + write y = 8 per pixel (plus the parameters)."""
+    wl = WORKLOADS["stage1_f32_k5_L3"]
+    c = bench.algorithmic_counts(wl)
+    P = 32 * 96 * 56 * 56
+    assert c["fwd"]["fma"] == pytest.approx(P * 57.8125, rel=1e-12)
+    params = 4 * (96 * 25 + 2 * 96 + 3 * 96 * 4 * 26)
+    assert c["fwd"]["bytes"] == 8 * P + params
+    assert c["bwd_weight"]["bytes"] == 8 * P + 2 * params
+    # level 0: the plain depthwise conv, k^2 FMAs per pixel
+    c0 = bench.algorithmic_counts(WORKLOADS["dw_k3_112_f32"])
+    assert c0["fwd"]["fma"] == 64 * 32 * 112 * 112 * 9
+
+
+def test_launches_per_step_of_the_stage1_workload():
+    """fold + output kernel for each data pass, weight-gradient kernel +
+    finalize: six library kernels per step."""
+    wl = WORKLOADS["stage1_f32_k5_L3"]
+    desc = wt.make_desc(wl.N, wl.C, wl.H, wl.W, wl.k, wl.L, wl.io)
+    assert bench.launches_per_step(wt, desc) == 6
+
+
+def test_source_hash_ignores_comments_and_layout_only():
+    a = "int f(int x) {  // doubles\n  return 2 * x;  /* no overflow check */\n}\n"
+    b = "int f(int x) {\n    return 2 * x;\n}\n"
+    c = "int f(int x) {\n  return 3 * x;\n}\n"
+    assert bench._code_only(a) == bench._code_only(b)
+    assert bench._code_only(a) != bench._code_only(c)
+
+
+def test_committed_traffic_is_used_only_while_the_sources_match(monkeypatch):
+    rec = json.load(open(os.path.join(bench.ROOT, "profiles", "traffic.json")))
+    wl = "stage1_f32_k5_L3"
+    monkeypatch.setattr(bench, "sources_sha256", lambda: rec["sources_sha256"])
+    assert bench.load_traffic("fwd", wl) == rec[wl]["fwd"]
+    monkeypatch.setattr(bench, "sources_sha256", lambda: "0" * 64)
+    assert bench.load_traffic("fwd", wl) is None
