@@ -296,14 +296,65 @@ bool build_deep_plan(DeepPlan& D, const wtconv_desc* d, int max_smem) {
   return true;
 }
 
+// Plan constants of sm_100a (B200): opt-in shared memory per CTA and SM
+// count.  The weight-gradient path, the way the data passes get their deep
+// levels, and the workspaces of both depend on the shape only, through
+// these, so wtconv_workspace_size needs no device query.
+constexpr int PLAN_SMEM = 232448;
+constexpr int PLAN_SMS = 148;
+
 size_t t1_bytes(const wtconv_desc* d) {
   return d->L >= 2 ? (((size_t)d->N * d->C * (d->H / 2) * (d->W / 2) * sizeof(float) + 15) / 16) * 16 : 0;
 }
 
-// Forward / backward-data workspace: 16-byte header (status word), t1 of
-// every plane (levels >= 2), then the folded weights of every channel.
-size_t fwd_ws_bytes(const wtconv_desc* d) {
-  return 16 + t1_bytes(d) + (size_t)d->C * main_wblk(d) * sizeof(float);
+// Row-band planes with L >= 2 whose level-2 planes exceed the deep kernel's
+// shared memory compute their levels >= 2 as a smaller layer: L - 1 levels on
+// the level-1 LL planes (H/2 x W/2, fp32), no base branch.  Its output is the
+// synthesis of levels >= 2 at level-1 resolution, i.e. t1.
+bool deep_by_recursion(const wtconv_desc* d) {
+  if (d->L < 2) return false;
+  MainPlan M;
+  if (!build_main_plan(M, d, PLAN_SMEM) || M.fused) return false;
+  DeepPlan D;
+  return !build_deep_plan(D, d, PLAN_SMEM);
+}
+wtconv_desc half_layer(const wtconv_desc* d) {
+  wtconv_desc h = *d;
+  h.H = d->H / 2;
+  h.W = d->W / 2;
+  h.L = d->L - 1;
+  h.io = WTCONV_F32;
+  return h;
+}
+size_t fold_bytes(const wtconv_desc* d) { return (size_t)d->C * main_wblk(d) * sizeof(float); }
+
+// Workspace of the data pass over a folded block (run_folded): 16-byte
+// header (status word), t1 of every plane (levels >= 2), and for the
+// recursion the LL planes, the smaller layer's folded block and its own
+// data-pass workspace.
+size_t pass_ws_bytes(const wtconv_desc* d) {
+  size_t b = 16 + t1_bytes(d);
+  if (deep_by_recursion(d)) {
+    const wtconv_desc h = half_layer(d);
+    b += t1_bytes(d) + (fold_bytes(&h) + 15) / 16 * 16 + pass_ws_bytes(&h);
+  }
+  return b;
+}
+
+// Forward / backward-data workspace: the data pass's, then the folded
+// weights of every channel.
+size_t fwd_ws_bytes(const wtconv_desc* d) { return pass_ws_bytes(d) + fold_bytes(d); }
+
+// Kernels one data pass over a folded block launches: [the LL planes, the
+// smaller layer's block and its own pass], [deep kernel], output kernel.
+int pass_launches(const wtconv_desc* d) {
+  MainPlan M;
+  if (!build_main_plan(M, d, PLAN_SMEM)) return 0;
+  if (d->L < 2 || M.fused) return 1;
+  if (!deep_by_recursion(d)) return 2;
+  const wtconv_desc h = half_layer(d);
+  const int inner = pass_launches(&h);
+  return inner ? 3 + inner : 0;
 }
 
 wtconv_status check_desc(const wtconv_desc* d) {
@@ -464,9 +515,8 @@ wtconv_status launch_forward_t(const wtconv_desc* d, const Device& dev, const vo
     M.oW = out->W;
     M.vec_out = (out->W % 4) == 0;
   }
-  if (d->L >= 2 && !M.fused) {
-    DeepPlan D;
-    if (!build_deep_plan(D, d, dev.max_smem)) return WTCONV_ERR_UNSUPPORTED;
+  DeepPlan D;
+  if (d->L >= 2 && !M.fused && build_deep_plan(D, d, dev.max_smem)) {  // else t1 came from the smaller layer
     auto kd = wtconv_deep_kernel<K, IO>;
     const size_t smem = (size_t)D.smem_floats * 4;
     int occ = 0;
@@ -526,12 +576,36 @@ wtconv_status run_fold(const wtconv_desc* d, const float* w0, const float* b0, c
 // followed by t1 when L >= 2.  With `out`, x holds zero-padded planes and y
 // receives only the out->H x out->W image of each.
 wtconv_status run_folded(const wtconv_desc* d, const void* x, const float* wfold, void* y, void* ws, cudaStream_t st,
-                         const wtconv_desc* out = nullptr) {
+                         const wtconv_desc* out = nullptr, int* status_word = nullptr) {
   Device dev;
   wtconv_status e = query_device(dev);
   if (e != WTCONV_OK) return e;
-  int* status = static_cast<int*>(ws);
+  // the workspace layout (deep kernel or recursion) is planned for sm_100a's
+  // shared memory per CTA
+  if (dev.max_smem < PLAN_SMEM) return WTCONV_ERR_UNSUPPORTED;
+  // the smaller layer's kernels report to the caller's status word
+  int* status = status_word ? status_word : static_cast<int*>(ws);
   float* t1 = reinterpret_cast<float*>(static_cast<char*>(ws) + 16);
+  if (deep_by_recursion(d)) {
+    // t1 = the smaller layer (levels 2..L as 1..L-1) on the LL planes
+    const wtconv_desc h = half_layer(d);
+    char* extra = static_cast<char*>(ws) + 16 + t1_bytes(d);
+    float* ll = reinterpret_cast<float*>(extra);
+    float* wf1 = reinterpret_cast<float*>(extra + t1_bytes(d));
+    void* ws1 = extra + t1_bytes(d) + (fold_bytes(&h) + 15) / 16 * 16;
+    const long long n = (long long)d->N * d->C * h.H * h.W;
+    const int grid = (int)std::min<long long>((n + 255) / 256, (long long)dev.sms * 8);
+    if (d->io == WTCONV_F32)
+      wtconv_ll_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float*>(x), ll, d->H, d->W, n);
+    else
+      wtconv_ll_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(x), ll, d->H, d->W,
+                                                             n);
+    const int kk4 = rup(d->k * d->k, 4), nw = d->C * main_wblk(&h);
+    wtconv_shift_fold_kernel<<<std::min((nw + 255) / 256, dev.sms * 4), 256, 0, st>>>(
+        wfold, wf1, d->C, kk4, main_wblk(d), main_wblk(&h), h.L);
+    if (cudaGetLastError() != cudaSuccess) return WTCONV_ERR_CUDA;
+    if ((e = run_folded(&h, ll, wf1, t1, ws1, st, nullptr, status)) != WTCONV_OK) return e;
+  }
   switch (d->k) {
     case 1: return launch_forward_k<1>(d, dev, x, wfold, y, status, t1, out, st);
     case 3: return launch_forward_k<3>(d, dev, x, wfold, y, status, t1, out, st);
@@ -545,7 +619,7 @@ wtconv_status run_folded(const wtconv_desc* d, const void* x, const float* wfold
 wtconv_status run_forward(const wtconv_desc* d, const void* x, const float* w0, const float* b0, const float* s0,
                           const float* wl, const float* sl, void* y, int flip, void* ws, cudaStream_t st,
                           const wtconv_desc* out = nullptr) {
-  float* wfold = reinterpret_cast<float*>(static_cast<char*>(ws) + 16 + t1_bytes(d));
+  float* wfold = reinterpret_cast<float*>(static_cast<char*>(ws) + pass_ws_bytes(d));
   wtconv_status e = run_fold(d, w0, b0, s0, wl, sl, flip, wfold, st);
   if (e != WTCONV_OK) return e;
   return run_folded(d, x, wfold, y, ws, st, out);
@@ -555,11 +629,7 @@ wtconv_status run_forward(const wtconv_desc* d, const void* x, const float* w0, 
 // then (weight gradients) the per-CTA partial sums.
 constexpr size_t WS_HEADER = 16;
 
-// Plan constants of sm_100a (B200): opt-in shared memory per CTA and SM
-// count.  The weight-gradient path and its workspace depend on the shape
-// only, through these, so wtconv_workspace_size needs no device query.
-constexpr int PLAN_SMEM = 232448;
-constexpr int PLAN_SMS = 148;
+
 
 // ---- whole-plane weight-gradient plan
 
@@ -1041,7 +1111,7 @@ size_t op_ws(const wtconv_desc* desc, int op) {
     case WTCONV_OP_BACKWARD:
       return std::max(bwdw_ws_bytes(desc), fwd_ws_bytes(desc));
     case WTCONV_OP_FORWARD_FOLDED:
-      return 16 + t1_bytes(desc);
+      return pass_ws_bytes(desc);
     default:
       return 0;
   }
@@ -1261,10 +1331,8 @@ int wtconv_kernel_launches(const wtconv_desc* desc, int op) {
     if (inner == 0 || op == WTCONV_OP_FOLD) return inner;
     return inner + op_acts(op);  // the pads of the inputs
   }
-  MainPlan M;
-  const bool main_ok = build_main_plan(M, desc, PLAN_SMEM);
-  const int pass = main_ok ? 1 + ((desc->L >= 2 && !M.fused) ? 1 : 0) : 0;  // [deep], output
-  const int data = main_ok ? 1 + pass : 0;                                  // fold first
+  const int pass = pass_launches(desc);
+  const int data = pass ? 1 + pass : 0;  // fold first
   const int weight = bwdw_whole_plane(desc) ? 2 : (desc->L == 0 ? 1 : desc->L) + 1;  // kernel(s), finalize
   switch (op) {
     case WTCONV_OP_FORWARD:

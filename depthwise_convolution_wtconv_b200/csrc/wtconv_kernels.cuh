@@ -169,4 +169,40 @@ __global__ void __launch_bounds__(256) wtconv_pad_kernel(const IO* __restrict__ 
   }
 }
 
+// Planes too large for the deep kernel compute their levels >= 2 as a layer
+// of one level fewer on the level-1 LL planes (the raw LL band that goes one
+// level deeper); these two kernels prepare its input and its weights.
+//
+// LL band of the level-1 Haar analysis: (a+b+c+d)/2 of every 2x2 block.
+template <typename IO>
+__global__ void wtconv_ll_kernel(const IO* __restrict__ x, float* __restrict__ ll, int H, int W, long long n) {
+  const int W1 = W / 2, H1 = H / 2;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+    const long long row = i / W1;  // row of the LL plane stack
+    const int j = (int)(i - row * W1);
+    const long long p = row / H1;
+    const int r = (int)(row - p * H1);
+    const IO* a = x + ((size_t)p * H + 2 * r) * W + 2 * j;
+    using T = io_traits<IO>;
+    ll[i] = 0.5f * ((T::to_f(a[0]) + T::to_f(a[1])) + (T::to_f(a[W]) + T::to_f(a[W + 1])));
+  }
+}
+
+// Folded block of that smaller layer from the layer's own block: base
+// kernel and bias zero (the smaller layer has no base branch), level l' =
+// level l' + 1 of the original.  The original's 2^-(l'+1) s W equals the
+// smaller layer's 2^-l' (s/2) W: the extra 1/2 is the level-1 synthesis
+// factor that its output carries into the original layer.
+__global__ void wtconv_shift_fold_kernel(const float* __restrict__ wf, float* __restrict__ wf1, int C, int kk4,
+                                         int wblk, int wblk1, int L1) {
+  // level l' starts at kk4 + 4 + 4 (l' - 1) kk4 in both layouts, so the
+  // original's level l' + 1 sits 4 kk4 floats further on
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < C * wblk1; i += gridDim.x * blockDim.x) {
+    const int c = i / wblk1, e = i - c * wblk1;
+    float v = 0.f;
+    if (e >= kk4 + 4 && e < kk4 + 4 + 4 * L1 * kk4) v = wf[(size_t)c * wblk + e + 4 * kk4];
+    wf1[i] = v;
+  }
+}
+
 }  // namespace wt

@@ -121,6 +121,25 @@ def test_ragged_launch_counts_and_noalloc(lib):
     assert lib.wtconv_backward_weight_noalloc(ctypes.byref(d), *args, None) == SHAPE
 
 
+def test_large_planes_take_their_deep_levels_from_a_smaller_layer(lib):
+    """512x512 planes with L = 2 do not fit the deep kernel: the levels >= 2
+    run as a layer of L - 1 levels on the 256x256 LL planes.  Workspace:
+    header, t1, the LL planes (as large as t1), the smaller layer's folded
+    block and its own data-pass workspace (header only at L = 1), then this
+    layer's folded block; launches: fold, LL planes, shifted block, the
+    smaller layer's output kernel, this layer's output kernel."""
+    d = _lib.WTConvDesc(2, 3, 512, 512, 5, 2, 0)
+    t1 = 2 * 3 * 256 * 256 * 4
+    fold_half = 3 * (5 * 28 + 4) * 4                 # L = 1 block of the smaller layer
+    fold = 3 * (9 * 28 + 4) * 4
+    assert lib.wtconv_workspace_size(ctypes.byref(d), 0) == 16 + t1 + t1 + fold_half + 16 + fold
+    assert lib.wtconv_workspace_size(ctypes.byref(d), 4) == 16 + t1 + t1 + fold_half + 16
+    n = lambda d, op: lib.wtconv_kernel_launches(ctypes.byref(d), op)
+    assert n(d, 0) == 5 and n(d, 4) == 4
+    # 1024x1024 with L = 3 recurses twice (512x512 L = 2, then 256x256 L = 1)
+    assert n(_lib.WTConvDesc(1, 1, 1024, 1024, 3, 3, 0), 0) == 8
+
+
 def test_folded_block_size_and_launches(lib):
     """The folded block: per channel k*k padded to 4, then the bias slot (4
     floats), then 4 padded kernels per level.  forward_folded launches the

@@ -23,6 +23,7 @@ CASES = [
     Workload("small_L0_k5", 4, 5, 14, 14, 5, 0, "f32"),
     Workload("L1_k1", 2, 3, 16, 12, 1, 1, "f32"),
     Workload("ragged_L2", 2, 3, 13, 11, 5, 2, "f32"),
+    Workload("recursive_512_L2", 1, 2, 512, 512, 3, 2, "f32"),
 ]
 
 

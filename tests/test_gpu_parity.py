@@ -117,6 +117,10 @@ EDGE = [
     Workload("ragged_55x54_L3", 2, 3, 55, 54, 5, 3, "f32"),
     Workload("ragged_bands_250_L2", 1, 2, 250, 246, 5, 2, "bf16"),
     Workload("ragged_3x3_L3_k1", 2, 2, 3, 3, 1, 3, "f32"),
+    # planes too large for the deep kernel: levels >= 2 as a smaller layer on
+    # the level-1 LL planes (twice for 1024x1024)
+    Workload("recursive_512_L2", 1, 2, 512, 512, 5, 2, "f32"),
+    Workload("recursive_640x384_L3_bf16", 1, 2, 640, 384, 3, 3, "bf16"),
 ]
 
 
@@ -162,6 +166,24 @@ def test_parity_deep_full_size_sampled(cuda_ok):
         assert _rel(_np(dx[n:n + 1]), ref["dX"]) <= TOL["bf16"]
     sub = dataclasses.replace(wl, N=2)
     check_all(sub)
+
+
+def test_data_passes_recurse_twice_for_1024x1024(cuda_ok):
+    """1024x1024 planes with L = 3: the levels >= 2 run as a 512x512 layer
+    with L = 2, whose own levels >= 2 run as a 256x256 layer with L = 1.
+    Forward and backward-data against the oracle (the row-band weight
+    gradients do not reach planes this wide with k = 7)."""
+    wl = Workload("recursive_twice", 1, 1, 1024, 1024, 7, 3, "f32")
+    inp = make_inputs(wl, 4)
+    d = _dev(inp, wl.io)
+    y = wt.forward(d["X"], d["W0"], d["b0"], d["s0"], d["Wl"], d["sl"])
+    dx = wt.backward_data(d["dY"], d["W0"], d["s0"], d["Wl"], d["sl"])
+    torch.cuda.synchronize()
+    p = as_float64(inp)
+    Y = oracle.forward(p["X"], p["W0"], p["b0"], p["s0"], p["Wl"], p["sl"])
+    dX = oracle.backward(p["X"], p["dY"], p["W0"], p["b0"], p["s0"], p["Wl"], p["sl"])["dX"]
+    assert _rel(_np(y), Y) <= TOL["f32"]
+    assert _rel(_np(dx), dX) <= TOL["f32"]
 
 
 def test_weight_gradients_deterministic(cuda_ok):
