@@ -140,6 +140,15 @@ def test_large_planes_take_their_deep_levels_from_a_smaller_layer(lib):
     assert n(_lib.WTConvDesc(1, 1, 1024, 1024, 3, 3, 0), 0) == 8
 
 
+def test_planes_wider_than_the_row_bands_hold_are_not_planned(lib):
+    """Row bands keep whole rows on chip: with L >= 1 and k = 5 the data
+    passes plan widths up to 1280 and no wider (0 launches = refused)."""
+    n = lambda d, op: lib.wtconv_kernel_launches(ctypes.byref(d), op)
+    assert n(_lib.WTConvDesc(1, 1, 64, 1280, 5, 2, 0), 0) > 0
+    assert n(_lib.WTConvDesc(1, 1, 64, 1536, 5, 2, 0), 0) == 0
+    assert n(_lib.WTConvDesc(1, 1, 4096, 64, 5, 2, 0), 0) > 0   # tall planes are fine
+
+
 def test_folded_block_size_and_launches(lib):
     """The folded block: per channel k*k padded to 4, then the bias slot (4
     floats), then 4 padded kernels per level.  forward_folded launches the
