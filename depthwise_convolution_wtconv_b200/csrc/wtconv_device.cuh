@@ -55,35 +55,9 @@ __device__ __forceinline__ float4 load4(const __nv_bfloat16* __restrict__ p, int
   return t;
 }
 
-// Stores n (<= 8) consecutive values of one output row.  `vec` says the
-// row start p is 16-byte aligned for the full 8-element vector form.
-__device__ __forceinline__ void store8(float* __restrict__ p, const float (&v)[8], int n, bool vec) {
-  if (vec && n == 8) {
-    reinterpret_cast<float4*>(p)[0] = make_float4(v[0], v[1], v[2], v[3]);
-    reinterpret_cast<float4*>(p)[1] = make_float4(v[4], v[5], v[6], v[7]);
-    return;
-  }
-#pragma unroll
-  for (int e = 0; e < 8; ++e)
-    if (e < n) p[e] = v[e];
-}
 __device__ __forceinline__ unsigned pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 t = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<unsigned*>(&t);
-}
-__device__ __forceinline__ void store8(__nv_bfloat16* __restrict__ p, const float (&v)[8], int n, bool vec) {
-  if (vec && n == 8) {
-    uint4 t;
-    t.x = pack_bf16x2(v[0], v[1]);
-    t.y = pack_bf16x2(v[2], v[3]);
-    t.z = pack_bf16x2(v[4], v[5]);
-    t.w = pack_bf16x2(v[6], v[7]);
-    *reinterpret_cast<uint4*>(p) = t;
-    return;
-  }
-#pragma unroll
-  for (int e = 0; e < 8; ++e)
-    if (e < n) p[e] = __float2bfloat16_rn(v[e]);
 }
 
 // Stores n (<= 4) consecutive values of one output row.  `vec` says the row
