@@ -408,6 +408,9 @@ def run_ours(args, wl, world, rank, local):
                    "l2": "flushed before every timed step (256 MiB write)"},
         "roofline": {"bound": bound, "kernel": f"{dom} pass: {PASS_KERNELS[dom]}", "achieved": achieved,
                      "peak": peak, "unit": unit, "frac": achieved / peak, "traffic": traffic,
+                     "traffic_source": ("profiles/traffic.json (ncu dram__bytes_read.sum + dram__bytes_write.sum "
+                                        "per launch, same sources)" if traffic is not None else
+                                        "none: no ncu capture of the current sources"),
                      "peak_source": peak_source},
         "hbm": {"achieved_gbs": hbm_gbs, "peak_gbs": hbm_peak, "frac": hbm_gbs / hbm_peak,
                 "algorithmic_bytes_per_step": step_bytes, "peak_source": peak_src},
