@@ -137,7 +137,14 @@ def test_large_planes_take_their_deep_levels_from_a_smaller_layer(lib):
     n = lambda d, op: lib.wtconv_kernel_launches(ctypes.byref(d), op)
     assert n(d, 0) == 5 and n(d, 4) == 4
     # 1024x1024 with L = 3 recurses twice (512x512 L = 2, then 256x256 L = 1)
-    assert n(_lib.WTConvDesc(1, 1, 1024, 1024, 3, 3, 0), 0) == 8
+    big = _lib.WTConvDesc(1, 1, 1024, 1024, 3, 3, 0)
+    assert n(big, 0) == 8
+    fold = lambda L: (((1 + 4 * L) * 12 + 4 + 3) // 4 * 4) * 4    # k = 3: k*k padded to 12
+    t1_512, t1_1024 = 256 * 256 * 4, 512 * 512 * 4
+    inner = 16 + t1_512 + t1_512 + fold(1) + 16                     # the 512x512 L = 2 layer's pass
+    outer = 16 + t1_1024 + t1_1024 + fold(2) + inner
+    assert lib.wtconv_workspace_size(ctypes.byref(big), 4) == outer
+    assert lib.wtconv_workspace_size(ctypes.byref(big), 0) == outer + fold(3)
 
 
 def test_planes_wider_than_the_row_bands_hold_are_not_planned(lib):
