@@ -36,9 +36,10 @@
  *
  * Conventions shared by every entry point:
  *   - Every tensor pointer is caller-owned DEVICE memory; the library never
- *     allocates, frees or keeps state between calls.  Calls are asynchronous
- *     on `stream` (a cudaStream_t; NULL = legacy default stream) and never
- *     synchronise.
+ *     allocates, frees or keeps state between calls (one exception:
+ *     wtconv_backward_weight_noalloc's own device array, below).  Calls are
+ *     asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and never synchronise.
  *   - Workspace (`ws`, `ws_bytes`): device memory of at least
  *     wtconv_workspace_size(desc, op) bytes, 16-byte aligned.  Its first 16
  *     bytes are a header whose first int is a device status word: a kernel
@@ -192,7 +193,9 @@ wtconv_status wtconv_backward(const wtconv_desc* desc, const void* x,
  * allocating library routine).  Every call on a device shares the one array,
  * which keeps the last call's contents (each call overwrites every partial it
  * reads): calls that overlap on the GPU, e.g. on two streams, race and must
- * be serialised by the caller. */
+ * be serialised by the caller.  There is no device status word here: a
+ * bounded in-kernel wait that runs out still ends the kernel, but nothing
+ * tells the caller; callers that check for it use wtconv_backward_weight. */
 wtconv_status wtconv_backward_weight_noalloc(const wtconv_desc* desc,
                                              const void* x, const void* dy,
                                              const float* w0, const float* b0,
