@@ -162,6 +162,83 @@ def test_delta_kernels_reproduce_scaled_block_means(L):
     np.testing.assert_allclose(Y, ref, rtol=0, atol=1e-12)
 
 
+# Signs of the four Haar bands over a 2x2 block, indexed [row bit][col bit]:
+# LL (a+b+c+d)/2, LH (a+b-c-d)/2, HL (a-b+c-d)/2, HH (a-b-c+d)/2.
+_SIGMA = {0: ((1, 1), (1, 1)), 1: ((1, 1), (-1, -1)), 2: ((1, -1), (1, -1)), 3: ((1, -1), (-1, 1))}
+
+
+def _single_band_delta_error(level, band):
+    """Max |oracle - hand-worked value| for one shifted delta kernel on one
+    band of one level, everything else 0.
+
+    Worked by hand from the layer's definition (Haar analysis, depthwise
+    conv with scale, inverse cascade): the LL chain gives
+    LL_m(p, q) = 2^-m * (sum of the aligned 2^m x 2^m block of X), so band s
+    at level l is B(P, Q) = 1/2 sum_{a,b} sigma_s(a, b) LL_{l-1}(2P+a, 2Q+b);
+    a delta at tap (r+du, r+dv) reads B(P+du, Q+dv) (zero outside); the level-l
+    synthesis spreads c*B/2 with the band's signs over bit l-1 of the output
+    coordinates, and every coarser-to-finer step after it halves it again:
+        Y(i, j) = 2^-l * c * sigma_s(bit_{l-1} i, bit_{l-1} j) * B(i>>l + du, j>>l + dv).
+    Computed here with plain loops, independent of the oracle's code."""
+    N, C, H, W, k = 1, 2, 32, 32, 5
+    r = k // 2
+    du, dv = 1, -2
+    L = level
+    X = rng.standard_normal((N, C, H, W))
+    c = np.array([0.75, 1.25])
+    Wl = np.zeros((L, C, 4, k, k))
+    Wl[level - 1, :, band, r + du, r + dv] = 1.0
+    sl = rng.uniform(0.5, 1.5, (L, C, 4))
+    sl[level - 1, :, band] = c
+    Y = oracle.forward(X, np.zeros((C, k, k)), np.zeros(C), rng.uniform(0.5, 1.5, C), Wl, sl)
+
+    m = level - 1
+    hb, wb = H >> level, W >> level
+    sig = _SIGMA[band]
+    ref = np.zeros_like(X)
+    for ch in range(C):
+        x = X[0, ch]
+        llm = np.zeros((H >> m, W >> m))
+        for p in range(H >> m):
+            for q in range(W >> m):
+                llm[p, q] = x[p << m:(p + 1) << m, q << m:(q + 1) << m].sum() / 2 ** m
+        B = np.zeros((hb, wb))
+        for P in range(hb):
+            for Q in range(wb):
+                B[P, Q] = 0.5 * sum(sig[a][b] * llm[2 * P + a, 2 * Q + b] for a in (0, 1) for b in (0, 1))
+        for i in range(H):
+            for j in range(W):
+                P, Q = (i >> level) + du, (j >> level) + dv
+                if 0 <= P < hb and 0 <= Q < wb:
+                    s_ij = sig[(i >> m) & 1][(j >> m) & 1]
+                    ref[0, ch, i, j] = 2.0 ** -level * c[ch] * s_ij * B[P, Q]
+    assert np.max(np.abs(ref)) > 0.1  # the shifted taps reach the band
+    return float(np.max(np.abs(Y - ref)))
+
+
+@pytest.mark.parametrize("level,band", [(2, 1), (2, 2), (2, 3), (3, 3), (3, 1), (1, 2)])
+def test_single_band_shifted_delta_by_hand(level, band):
+    assert _single_band_delta_error(level, band) < 1e-12
+
+
+def test_single_band_pin_catches_swapped_bands_and_transposed_kernel(monkeypatch):
+    """The pin above fails on an oracle with LH and HL swapped in its
+    analysis, or with its depthwise kernels transposed."""
+    good_analysis = oracle.wtconv_oracle.haar_analysis
+
+    def swapped(A):
+        S = good_analysis(A)
+        return S[..., [0, 2, 1, 3], :, :]
+    monkeypatch.setattr(oracle.wtconv_oracle, "haar_analysis", swapped)
+    assert _single_band_delta_error(2, 1) > 1e-3
+    monkeypatch.setattr(oracle.wtconv_oracle, "haar_analysis", good_analysis)
+    assert _single_band_delta_error(2, 1) < 1e-12
+
+    good_conv = oracle.wtconv_oracle.dwconv
+    monkeypatch.setattr(oracle.wtconv_oracle, "dwconv", lambda A, Wt: good_conv(A, np.swapaxes(Wt, -1, -2)))
+    assert _single_band_delta_error(3, 3) > 1e-3
+
+
 def test_delta_unit_scales_level1_doubles_input():
     X = rng.standard_normal((1, 2, 8, 8))
     W0 = np.zeros((2, 3, 3)); W0[:, 1, 1] = 1
