@@ -167,9 +167,10 @@ def test_delta_kernels_reproduce_scaled_block_means(L):
 _SIGMA = {0: ((1, 1), (1, 1)), 1: ((1, 1), (-1, -1)), 2: ((1, -1), (1, -1)), 3: ((1, -1), (-1, 1))}
 
 
-def _single_band_delta_error(level, band):
-    """Max |oracle - hand-worked value| for one shifted delta kernel on one
-    band of one level, everything else 0.
+def _single_band_delta_errors(level, band):
+    """Max |oracle - hand-worked value| of Y, of the band's weight gradient
+    and of its scale gradient, for one shifted delta kernel on one band of
+    one level, everything else 0.
 
     Worked by hand from the layer's definition (Haar analysis, depthwise
     conv with scale, inverse cascade): the LL chain gives
@@ -179,23 +180,30 @@ def _single_band_delta_error(level, band):
     synthesis spreads c*B/2 with the band's signs over bit l-1 of the output
     coordinates, and every coarser-to-finer step after it halves it again:
         Y(i, j) = 2^-l * c * sigma_s(bit_{l-1} i, bit_{l-1} j) * B(i>>l + du, j>>l + dv).
-    Computed here with plain loops, independent of the oracle's code."""
+    Y is linear in each tap, so the gradient of <Y, dY> in tap (u, v) is
+        dW(u, v) = c * sum_{i,j} dY(i, j) 2^-l sigma_s(bits) B(i>>l + u-r, j>>l + v-r),
+    and in the scale c it is dW(r+du, r+dv) / c.  Computed here with plain
+    loops, independent of the oracle's code."""
     N, C, H, W, k = 1, 2, 32, 32, 5
     r = k // 2
     du, dv = 1, -2
     L = level
     X = rng.standard_normal((N, C, H, W))
+    dY = rng.standard_normal((N, C, H, W))
     c = np.array([0.75, 1.25])
     Wl = np.zeros((L, C, 4, k, k))
     Wl[level - 1, :, band, r + du, r + dv] = 1.0
     sl = rng.uniform(0.5, 1.5, (L, C, 4))
     sl[level - 1, :, band] = c
-    Y = oracle.forward(X, np.zeros((C, k, k)), np.zeros(C), rng.uniform(0.5, 1.5, C), Wl, sl)
+    W0, b0, s0 = np.zeros((C, k, k)), np.zeros(C), rng.uniform(0.5, 1.5, C)
+    Y = oracle.forward(X, W0, b0, s0, Wl, sl)
+    g = oracle.backward(X, dY, W0, b0, s0, Wl, sl)
 
     m = level - 1
     hb, wb = H >> level, W >> level
     sig = _SIGMA[band]
     ref = np.zeros_like(X)
+    dw = np.zeros((C, k, k))
     for ch in range(C):
         x = X[0, ch]
         llm = np.zeros((H >> m, W >> m))
@@ -206,37 +214,59 @@ def _single_band_delta_error(level, band):
         for P in range(hb):
             for Q in range(wb):
                 B[P, Q] = 0.5 * sum(sig[a][b] * llm[2 * P + a, 2 * Q + b] for a in (0, 1) for b in (0, 1))
+        # D(P, Q): dY times the synthesis weight, summed over each level-l block
+        D = np.zeros((hb, wb))
         for i in range(H):
             for j in range(W):
+                s_ij = sig[(i >> m) & 1][(j >> m) & 1]
+                D[i >> level, j >> level] += 2.0 ** -level * s_ij * dY[0, ch, i, j]
                 P, Q = (i >> level) + du, (j >> level) + dv
                 if 0 <= P < hb and 0 <= Q < wb:
-                    s_ij = sig[(i >> m) & 1][(j >> m) & 1]
                     ref[0, ch, i, j] = 2.0 ** -level * c[ch] * s_ij * B[P, Q]
+        for u in range(k):
+            for v in range(k):
+                for P in range(hb):
+                    for Q in range(wb):
+                        if 0 <= P + u - r < hb and 0 <= Q + v - r < wb:
+                            dw[ch, u, v] += c[ch] * D[P, Q] * B[P + u - r, Q + v - r]
     assert np.max(np.abs(ref)) > 0.1  # the shifted taps reach the band
-    return float(np.max(np.abs(Y - ref)))
+    ds = dw[:, r + du, r + dv] / c
+    return (float(np.max(np.abs(Y - ref))),
+            float(np.max(np.abs(g["dWl"][level - 1, :, band] - dw))),
+            float(np.max(np.abs(g["dsl"][level - 1, :, band] - ds))))
 
 
 @pytest.mark.parametrize("level,band", [(2, 1), (2, 2), (2, 3), (3, 3), (3, 1), (1, 2)])
 def test_single_band_shifted_delta_by_hand(level, band):
-    assert _single_band_delta_error(level, band) < 1e-12
+    ey, ew, es = _single_band_delta_errors(level, band)
+    assert ey < 1e-12 and ew < 1e-11 and es < 1e-11, (ey, ew, es)
 
 
 def test_single_band_pin_catches_swapped_bands_and_transposed_kernel(monkeypatch):
     """The pin above fails on an oracle with LH and HL swapped in its
-    analysis, or with its depthwise kernels transposed."""
+    analysis, with its depthwise kernels transposed, or with its
+    weight-gradient correlation transposed."""
     good_analysis = oracle.wtconv_oracle.haar_analysis
 
     def swapped(A):
         S = good_analysis(A)
         return S[..., [0, 2, 1, 3], :, :]
     monkeypatch.setattr(oracle.wtconv_oracle, "haar_analysis", swapped)
-    assert _single_band_delta_error(2, 1) > 1e-3
+    assert _single_band_delta_errors(2, 1)[0] > 1e-3
     monkeypatch.setattr(oracle.wtconv_oracle, "haar_analysis", good_analysis)
-    assert _single_band_delta_error(2, 1) < 1e-12
+    assert _single_band_delta_errors(2, 1)[0] < 1e-12
 
     good_conv = oracle.wtconv_oracle.dwconv
     monkeypatch.setattr(oracle.wtconv_oracle, "dwconv", lambda A, Wt: good_conv(A, np.swapaxes(Wt, -1, -2)))
-    assert _single_band_delta_error(3, 3) > 1e-3
+    assert _single_band_delta_errors(3, 3)[0] > 1e-3
+    monkeypatch.setattr(oracle.wtconv_oracle, "dwconv", good_conv)
+
+    good_corr = oracle.wtconv_oracle.dwcorr_weight
+    monkeypatch.setattr(oracle.wtconv_oracle, "dwcorr_weight",
+                        lambda A, G, k: np.swapaxes(good_corr(A, G, k), -1, -2))
+    ey, ew, es = _single_band_delta_errors(2, 3)
+    # the oracle's scale gradient does not go through the tap correlation
+    assert ey < 1e-12 and ew > 1e-3 and es < 1e-11
 
 
 def test_delta_unit_scales_level1_doubles_input():
