@@ -196,7 +196,10 @@ def backward_weight(x, dy, w0, b0, s0, wl=None, sl=None, grads=None, ws=None, st
 def backward_weight_noalloc(x, dy, w0, b0, s0, wl=None, sl=None, grads=None, stream=None):
     """Parameter gradients without a workspace: the library keeps its partial
     sums in its own fixed device array (for callers that cannot allocate
-    device memory where they call it).  Same outputs as backward_weight."""
+    device memory where they call it).  Same outputs as backward_weight.
+    The C call allocates nothing; this wrapper allocates the gradient tensors
+    only when `grads` is not given, so pass `grads` to keep the call
+    allocation-free."""
     lib = load()
     _cuda(x, "x")
     _cuda(dy, "dy", x.dtype)
