@@ -268,3 +268,25 @@ def test_python_binding_refuses_cpu_tensors():
     w = torch.zeros(1, 3, 3)
     with pytest.raises(TypeError):
         wt.forward(x, w, torch.zeros(1), torch.ones(1))
+
+
+_CPU = dict(x=torch.zeros(1, 2, 8, 8), w0=torch.zeros(2, 3, 3), b0=torch.zeros(2), s0=torch.ones(2),
+            wl=torch.zeros(1, 2, 4, 3, 3), sl=torch.ones(1, 2, 4))
+_CALLS = {
+    "forward": lambda t: wt.forward(t["x"], t["w0"], t["b0"], t["s0"], t["wl"], t["sl"]),
+    "backward_data": lambda t: wt.backward_data(t["x"], t["w0"], t["s0"], t["wl"], t["sl"]),
+    "backward_weight": lambda t: wt.backward_weight(t["x"], t["x"], t["w0"], t["b0"], t["s0"], t["wl"], t["sl"]),
+    "backward_weight_noalloc": lambda t: wt.backward_weight_noalloc(t["x"], t["x"], t["w0"], t["b0"], t["s0"],
+                                                                    t["wl"], t["sl"]),
+    "backward": lambda t: wt.backward(t["x"], t["x"], t["w0"], t["b0"], t["s0"], t["wl"], t["sl"]),
+    "fold_weights": lambda t: wt.fold_weights(t["w0"], t["b0"], t["s0"], t["wl"], t["sl"]),
+    "forward_folded": lambda t: wt.forward_folded(t["x"], torch.zeros(4096, dtype=torch.uint8), 3, 1),
+}
+
+
+@pytest.mark.parametrize("name", sorted(_CALLS))
+def test_every_binding_refuses_cpu_tensors(name):
+    """No entry point has a CPU path: host tensors are refused before any
+    library call, on a machine with or without a GPU."""
+    with pytest.raises(TypeError, match="CUDA tensor"):
+        _CALLS[name](_CPU)
