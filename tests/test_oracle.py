@@ -167,7 +167,7 @@ def test_delta_kernels_reproduce_scaled_block_means(L):
 _SIGMA = {0: ((1, 1), (1, 1)), 1: ((1, 1), (-1, -1)), 2: ((1, -1), (1, -1)), 3: ((1, -1), (-1, 1))}
 
 
-def _single_band_delta_errors(level, band):
+def _single_band_delta_errors(level, band, H=32, W=32):
     """Max |oracle - hand-worked value| of Y, of the band's weight gradient
     and of its scale gradient, for one shifted delta kernel on one band of
     one level, everything else 0.
@@ -182,9 +182,11 @@ def _single_band_delta_errors(level, band):
         Y(i, j) = 2^-l * c * sigma_s(bit_{l-1} i, bit_{l-1} j) * B(i>>l + du, j>>l + dv).
     Y is linear in each tap, so the gradient of <Y, dY> in tap (u, v) is
         dW(u, v) = c * sum_{i,j} dY(i, j) 2^-l sigma_s(bits) B(i>>l + u-r, j>>l + v-r),
-    and in the scale c it is dW(r+du, r+dv) / c.  Computed here with plain
-    loops, independent of the oracle's code."""
-    N, C, H, W, k = 1, 2, 32, 32, 5
+    and in the scale c it is dW(r+du, r+dv) / c.  Sides that are not
+    multiples of 2^l take the zero-padded image in the block sums (the
+    layer's reading for such sides) and only outputs inside the image.
+    Computed here with plain loops, independent of the oracle's code."""
+    N, C, k = 1, 2, 5
     r = k // 2
     du, dv = 1, -2
     L = level
@@ -200,15 +202,18 @@ def _single_band_delta_errors(level, band):
     g = oracle.backward(X, dY, W0, b0, s0, Wl, sl)
 
     m = level - 1
-    hb, wb = H >> level, W >> level
+    b = 1 << level
+    Hp, Wp = -(-H // b) * b, -(-W // b) * b  # sides padded with zeros
+    hb, wb = Hp >> level, Wp >> level
     sig = _SIGMA[band]
     ref = np.zeros_like(X)
     dw = np.zeros((C, k, k))
     for ch in range(C):
-        x = X[0, ch]
-        llm = np.zeros((H >> m, W >> m))
-        for p in range(H >> m):
-            for q in range(W >> m):
+        x = np.zeros((Hp, Wp))
+        x[:H, :W] = X[0, ch]
+        llm = np.zeros((Hp >> m, Wp >> m))
+        for p in range(Hp >> m):
+            for q in range(Wp >> m):
                 llm[p, q] = x[p << m:(p + 1) << m, q << m:(q + 1) << m].sum() / 2 ** m
         B = np.zeros((hb, wb))
         for P in range(hb):
@@ -239,6 +244,12 @@ def _single_band_delta_errors(level, band):
 @pytest.mark.parametrize("level,band", [(2, 1), (2, 2), (2, 3), (3, 3), (3, 1), (1, 2)])
 def test_single_band_shifted_delta_by_hand(level, band):
     ey, ew, es = _single_band_delta_errors(level, band)
+    assert ey < 1e-12 and ew < 1e-11 and es < 1e-11, (ey, ew, es)
+
+
+@pytest.mark.parametrize("level,band,H,W", [(2, 3, 30, 22), (3, 1, 28, 28), (3, 2, 27, 21), (1, 3, 17, 9)])
+def test_single_band_shifted_delta_by_hand_ragged_sides(level, band, H, W):
+    ey, ew, es = _single_band_delta_errors(level, band, H, W)
     assert ey < 1e-12 and ew < 1e-11 and es < 1e-11, (ey, ew, es)
 
 
