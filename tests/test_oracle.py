@@ -182,7 +182,10 @@ def _single_band_delta_errors(level, band, H=32, W=32):
         Y(i, j) = 2^-l * c * sigma_s(bit_{l-1} i, bit_{l-1} j) * B(i>>l + du, j>>l + dv).
     Y is linear in each tap, so the gradient of <Y, dY> in tap (u, v) is
         dW(u, v) = c * sum_{i,j} dY(i, j) 2^-l sigma_s(bits) B(i>>l + u-r, j>>l + v-r),
-    and in the scale c it is dW(r+du, r+dv) / c.  Sides that are not
+    and in the scale c it is dW(r+du, r+dv) / c; the input gradient is
+        dX(i, j) = 2^-l * c * sigma_s(bits) * D(i>>l - du, j>>l - dv),
+    D(P, Q) = sum over the level-l block (P, Q) of 2^-l sigma_s(bits) dY.
+    Sides that are not
     multiples of 2^l take the zero-padded image in the block sums (the
     layer's reading for such sides) and only outputs inside the image.
     Computed here with plain loops, independent of the oracle's code."""
@@ -207,6 +210,7 @@ def _single_band_delta_errors(level, band, H=32, W=32):
     hb, wb = Hp >> level, Wp >> level
     sig = _SIGMA[band]
     ref = np.zeros_like(X)
+    dx = np.zeros_like(X)
     dw = np.zeros((C, k, k))
     for ch in range(C):
         x = np.zeros((Hp, Wp))
@@ -228,29 +232,35 @@ def _single_band_delta_errors(level, band, H=32, W=32):
                 P, Q = (i >> level) + du, (j >> level) + dv
                 if 0 <= P < hb and 0 <= Q < wb:
                     ref[0, ch, i, j] = 2.0 ** -level * c[ch] * s_ij * B[P, Q]
+        for i in range(H):
+            for j in range(W):
+                P, Q = (i >> level) - du, (j >> level) - dv
+                if 0 <= P < hb and 0 <= Q < wb:
+                    dx[0, ch, i, j] = 2.0 ** -level * c[ch] * sig[(i >> m) & 1][(j >> m) & 1] * D[P, Q]
         for u in range(k):
             for v in range(k):
                 for P in range(hb):
                     for Q in range(wb):
                         if 0 <= P + u - r < hb and 0 <= Q + v - r < wb:
                             dw[ch, u, v] += c[ch] * D[P, Q] * B[P + u - r, Q + v - r]
-    assert np.max(np.abs(ref)) > 0.1  # the shifted taps reach the band
+    assert np.max(np.abs(ref)) > 0.1 and np.max(np.abs(dx)) > 0.01  # the shifted taps reach the band
     ds = dw[:, r + du, r + dv] / c
     return (float(np.max(np.abs(Y - ref))),
             float(np.max(np.abs(g["dWl"][level - 1, :, band] - dw))),
-            float(np.max(np.abs(g["dsl"][level - 1, :, band] - ds))))
+            float(np.max(np.abs(g["dsl"][level - 1, :, band] - ds))),
+            float(np.max(np.abs(g["dX"] - dx))))
 
 
 @pytest.mark.parametrize("level,band", [(2, 1), (2, 2), (2, 3), (3, 3), (3, 1), (1, 2)])
 def test_single_band_shifted_delta_by_hand(level, band):
-    ey, ew, es = _single_band_delta_errors(level, band)
-    assert ey < 1e-12 and ew < 1e-11 and es < 1e-11, (ey, ew, es)
+    ey, ew, es, ex = _single_band_delta_errors(level, band)
+    assert ey < 1e-12 and ew < 1e-11 and es < 1e-11 and ex < 1e-12, (ey, ew, es, ex)
 
 
 @pytest.mark.parametrize("level,band,H,W", [(2, 3, 30, 22), (3, 1, 28, 28), (3, 2, 27, 21), (1, 3, 17, 9)])
 def test_single_band_shifted_delta_by_hand_ragged_sides(level, band, H, W):
-    ey, ew, es = _single_band_delta_errors(level, band, H, W)
-    assert ey < 1e-12 and ew < 1e-11 and es < 1e-11, (ey, ew, es)
+    ey, ew, es, ex = _single_band_delta_errors(level, band, H, W)
+    assert ey < 1e-12 and ew < 1e-11 and es < 1e-11 and ex < 1e-12, (ey, ew, es, ex)
 
 
 def test_single_band_pin_catches_swapped_bands_and_transposed_kernel(monkeypatch):
@@ -269,13 +279,14 @@ def test_single_band_pin_catches_swapped_bands_and_transposed_kernel(monkeypatch
 
     good_conv = oracle.wtconv_oracle.dwconv
     monkeypatch.setattr(oracle.wtconv_oracle, "dwconv", lambda A, Wt: good_conv(A, np.swapaxes(Wt, -1, -2)))
-    assert _single_band_delta_errors(3, 3)[0] > 1e-3
+    ey, _, _, ex = _single_band_delta_errors(3, 3)
+    assert ey > 1e-3 and ex > 1e-3
     monkeypatch.setattr(oracle.wtconv_oracle, "dwconv", good_conv)
 
     good_corr = oracle.wtconv_oracle.dwcorr_weight
     monkeypatch.setattr(oracle.wtconv_oracle, "dwcorr_weight",
                         lambda A, G, k: np.swapaxes(good_corr(A, G, k), -1, -2))
-    ey, ew, es = _single_band_delta_errors(2, 3)
+    ey, ew, es, _ = _single_band_delta_errors(2, 3)
     # the oracle's scale gradient does not go through the tap correlation
     assert ey < 1e-12 and ew > 1e-3 and es < 1e-11
 
