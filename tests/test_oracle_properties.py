@@ -74,3 +74,32 @@ def test_euler_identity_catches_a_planted_adjoint_mistake(monkeypatch):
     err = _euler_errors((1, 2, 11, 9, 5, 2, 7))
     assert err["W0"] > 1e-3 and err["Wl"] > 1e-3
     assert err["X"] <= 1e-11 and err["b0"] <= 1e-11
+
+
+@settings(max_examples=60, deadline=None, derandomize=True)
+@given(layer_case())
+def test_forward_and_gradients_equal_torch_composition_on_random_shapes(case):
+    """The oracle against the layer composed from library routines (per-level
+    F.pad, grouped conv2d, conv_transpose2d, cropping; autograd for the
+    gradients) on the same random shape and values."""
+    import torch
+    from test_oracle import torch_wtconv_ragged
+
+    N, C, H, W, k, L, seed = case
+    g = np.random.default_rng(seed)
+    p = dict(X=g.standard_normal((N, C, H, W)), W0=g.standard_normal((C, k, k)) / k,
+             b0=g.standard_normal(C) * 0.1, s0=g.uniform(0.5, 1.5, C),
+             Wl=g.standard_normal((L, C, 4, k, k)) / k if L else None,
+             sl=g.uniform(0.5, 1.5, (L, C, 4)) if L else None)
+    dY = g.standard_normal((N, C, H, W))
+    t = {key: (None if v is None else torch.tensor(v, requires_grad=True)) for key, v in p.items()}
+    Yt = torch_wtconv_ragged(t["X"], t["W0"], t["b0"], t["s0"], t["Wl"], t["sl"])
+    Yt.backward(torch.tensor(dY))
+    Y = oracle.forward(p["X"], p["W0"], p["b0"], p["s0"], p["Wl"], p["sl"])
+    np.testing.assert_allclose(Y, Yt.detach().numpy(), rtol=0, atol=1e-12 * (1 + np.abs(Y).max()))
+    gr = oracle.backward(p["X"], dY, p["W0"], p["b0"], p["s0"], p["Wl"], p["sl"])
+    for name, gname in (("X", "dX"), ("W0", "dW0"), ("b0", "db0"), ("s0", "ds0"), ("Wl", "dWl"), ("sl", "dsl")):
+        if t[name] is None:
+            continue
+        want = t[name].grad.numpy()
+        np.testing.assert_allclose(gr[gname], want, rtol=0, atol=1e-11 * (1 + np.abs(want).max()), err_msg=gname)
