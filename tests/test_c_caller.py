@@ -52,3 +52,16 @@ def test_c_caller_gets_host_side_errors(c_results):
     assert int(c_results["noalloc_huge_c"]) == 7        # WTCONV_ERR_SCRATCH_LIMIT
     assert c_results["status_string_ok"] == "set"
     assert c_results["status_string_limit"] == "set"
+
+
+def test_same_caller_as_cxx_links_through_extern_c(c_results, tmp_path):
+    """C++ callers get the unmangled symbols through the header's extern "C"
+    block: the caller built as C++17 prints the same results."""
+    if shutil.which("g++") is None:
+        pytest.skip("no C++ compiler")
+    exe = str(tmp_path / "cxx_abi_caller")
+    subprocess.run(["g++", "-x", "c++", "-std=c++17", "-Wall", "-Wextra", "-Werror",
+                    "-I" + os.path.join(ROOT, "include"), os.path.join(ROOT, "tests", "c_abi_caller.c"),
+                    "-L" + PKG, "-lwtconv", "-Wl,-rpath," + PKG, "-o", exe], check=True)
+    out = subprocess.run([exe], check=True, capture_output=True, text=True).stdout
+    assert dict(line.split(" ", 1) for line in out.strip().splitlines()) == c_results
