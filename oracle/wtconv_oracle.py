@@ -229,11 +229,6 @@ def backward(X, dY, W0, b0, s0, Wl, sl):
     return dict(dX=dX, dW0=dW0, db0=db0, ds0=ds0, dWl=dWl, dsl=dsl)
 
 
-def block_bits_sign(s, py, px):
-    """SIGN[s] at integer arrays of bits py, px."""
-    return SIGN[s][py, px]
-
-
 def analysis_closed_form(X, l):
     """Level-l subbands straight from X (reformulation (1) of arXiv:2608.10805).
 
@@ -277,12 +272,13 @@ def synthesis_closed_form(Zs, H, W):
 
 
 def level_outputs(X, Wl, sl):
-    """Z_l for every level (scaled level-conv outputs), for closed-form checks."""
-    L = Wl.shape[0]
-    Zs = []
-    cur = X
-    for l in range(L):
-        sub = haar_analysis(cur)
-        Zs.append(sl[l][None, :, :, None, None] * dwconv(sub, Wl[l][None]))
-        cur = sub[:, :, 0]
-    return Zs
+    """Z_l for every level (scaled level-conv outputs), for closed-form checks.
+
+    Taken from `forward`'s own intermediates (the level-conv outputs before
+    their scale), so the closed form is checked against exactly what the
+    cascade computed, on any plane size.
+    """
+    C, k = X.shape[1], Wl.shape[-1]
+    zero = np.zeros(C)
+    _, inter = forward(X, np.zeros((C, k, k)), zero, zero, Wl, sl, return_intermediates=True)
+    return [sl[l][None, :, :, None, None] * conv for l, conv in enumerate(inter["convs"])]
