@@ -46,4 +46,7 @@ WORKLOADS = {
     "deep_bf16_k5_L5": Workload("deep_bf16_k5_L5", 16, 64, 256, 256, 5, 5, "bf16"),
 }
 
-BENCH_WORKLOAD = "stage1_f32_k5_L3"
+# the headline workload (the largest single-GPU shape) and the other
+# full-size workloads the benchmark reports beside it
+BENCH_WORKLOAD = "deep_bf16_k5_L5"
+OTHER_WORKLOADS = ("stage1_f32_k5_L3", "stage2_bf16_k5_L2", "dw_k3_112_f32", "dw_k5_14_f32")

@@ -18,13 +18,43 @@ def test_algorithmic_counts_of_the_stage1_workload():
     wl = WORKLOADS["stage1_f32_k5_L3"]
     c = bench.algorithmic_counts(wl)
     P = 32 * 96 * 56 * 56
-    assert c["fwd"]["fma"] == pytest.approx(P * 57.8125, rel=1e-12)
+    assert c["passes"]["fwd"]["fma"] == pytest.approx(P * 57.8125, rel=1e-12)
     params = 4 * (96 * 25 + 2 * 96 + 3 * 96 * 4 * 26)
-    assert c["fwd"]["bytes"] == 8 * P + params
-    assert c["bwd_weight"]["bytes"] == 8 * P + 2 * params
+    assert bench.param_bytes(wl) == params
+    assert c["passes"]["fwd"]["bytes"] == 8 * P + params
+    assert c["passes"]["bwd_weight"]["bytes"] == 8 * P + 2 * params
+    # a step must read x, write y, read x and dy, write dx: 5 activations
+    assert c["step"]["bytes"] == 5 * 4 * P + 2 * params
+    assert c["step"]["design_bytes"] == 6 * 4 * P + 4 * params
+    assert c["step"]["fma"] == pytest.approx(3 * P * 57.8125, rel=1e-12)
     # level 0: the plain depthwise conv, k^2 FMAs per pixel
     c0 = bench.algorithmic_counts(WORKLOADS["dw_k3_112_f32"])
-    assert c0["fwd"]["fma"] == 64 * 32 * 112 * 112 * 9
+    assert c0["passes"]["fwd"]["fma"] == 64 * 32 * 112 * 112 * 9
+
+
+def test_algorithmic_bytes_of_the_deep_bf16_workload():
+    """16x64x256x256 bf16: S = 134.2 MB; 5S + 2 params = 671.4 MB a step."""
+    wl = WORKLOADS["deep_bf16_k5_L5"]
+    c = bench.algorithmic_counts(wl)
+    S = 16 * 64 * 256 * 256 * 2
+    assert S == 134217728
+    assert c["step"]["bytes"] == 5 * S + 2 * bench.param_bytes(wl)
+    assert c["step"]["bytes"] == pytest.approx(671.4e6, rel=1e-3)
+
+
+def test_step_and_pass_rooflines_pick_the_slower_bound():
+    wl = WORKLOADS["dw_k3_112_f32"]
+    c = bench.algorithmic_counts(wl)
+    peaks = {"hbm_gbs": 6528.7, "hbm_source": "m", "fp32_tflops": 74.45, "fp32_source": "n"}
+    kernels = {"fwd": 0.05, "bwd_data": 0.05, "bwd_weight": 0.1}
+    r = bench.pass_roofline(c, kernels, peaks)
+    assert r["pass_name"] == "bwd_weight" and r["bound"] == "hbm"
+    assert r["frac"] == pytest.approx(c["passes"]["bwd_weight"]["bytes"] / 0.1e-3 / 1e9 / 6528.7)
+    s = bench.step_bound(c, 0.2, peaks)
+    assert s["bound"] == "hbm"
+    assert s["frac"] == pytest.approx(c["step"]["bytes"] / 6528.7e9 / 0.2e-3)
+    wl3 = WORKLOADS["stage1_f32_k5_L3"]
+    assert bench.step_bound(bench.algorithmic_counts(wl3), 0.2, peaks)["bound"] == "alu"
 
 
 def test_launches_per_step_of_the_stage1_workload():
