@@ -19,12 +19,12 @@ OP_FORWARD_FOLDED, OP_FOLD = 4, 5
 STATUS_NAMES = {0: "WTCONV_OK", 1: "WTCONV_ERR_ARG", 2: "WTCONV_ERR_SHAPE", 3: "WTCONV_ERR_ALIGN",
                 4: "WTCONV_ERR_WORKSPACE", 5: "WTCONV_ERR_CUDA", 6: "WTCONV_ERR_UNSUPPORTED",
                 7: "WTCONV_ERR_SCRATCH_LIMIT"}
-NOALLOC_SCRATCH_BYTES = 8 << 20
 
 # every symbol include/wtconv.h declares
 EXPORTS = ("wtconv_workspace_size", "wtconv_forward", "wtconv_backward_data", "wtconv_backward_weight",
            "wtconv_backward", "wtconv_backward_weight_noalloc", "wtconv_folded_size", "wtconv_fold_weights",
-           "wtconv_forward_folded", "wtconv_kernel_launches", "wtconv_status_string")
+           "wtconv_forward_folded", "wtconv_kernel_launches", "wtconv_status_string",
+           "wtconv_noalloc_scratch_bytes")
 
 
 class WTConvDesc(ctypes.Structure):
@@ -73,8 +73,16 @@ def load(path=LIB_PATH):
     lib.wtconv_forward_folded.restype = ctypes.c_int
     lib.wtconv_kernel_launches.argtypes = [dp, ctypes.c_int]
     lib.wtconv_kernel_launches.restype = ctypes.c_int
+    lib.wtconv_noalloc_scratch_bytes.argtypes = []
+    lib.wtconv_noalloc_scratch_bytes.restype = sz
     _lib = lib
     return lib
+
+
+def noalloc_scratch_bytes():
+    """Size of the device array the no-allocation weight-gradient call uses,
+    as the loaded library was built with."""
+    return int(load().wtconv_noalloc_scratch_bytes())
 
 
 def make_desc(N, C, H, W, k, L, io):

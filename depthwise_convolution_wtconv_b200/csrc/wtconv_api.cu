@@ -1095,10 +1095,6 @@ wtconv_status check_grad_outputs(const wtconv_desc* d, const float* dw0, const f
 
 using namespace wt;
 
-extern "C" {
-
-}  // extern "C"
-
 namespace {
 // workspace of `op` for sides that are multiples of 2^L
 size_t op_ws(const wtconv_desc* desc, int op) {
@@ -1253,6 +1249,8 @@ wtconv_status wtconv_backward(const wtconv_desc* desc, const void* x, const void
   return run_bwdw(&p, xp, dyp, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, ws, st);
 }
 
+}  // extern "C"
+
 // ------------------------------------------------------------------------
 // Weight gradients for callers that cannot allocate device memory.
 //
@@ -1269,25 +1267,70 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[WTCONV_NOALLOC_
 namespace {
 constexpr int MAX_DEVICES = 64;
 std::mutex g_scratch_mutex;
-void* g_scratch_addr[MAX_DEVICES] = {};
+struct ScratchAddr {
+  unsigned long long ctx_id;  // id of the CUDA context the address belongs to
+  void* addr;
+};
+ScratchAddr g_scratch_addr[MAX_DEVICES] = {};
 
-// Device address of g_noalloc_scratch on the current device.  In host code
+// Id of the CUDA context current on this thread (0 when none is current
+// yet).  Ids are unique for the life of the process, so a context created
+// again after cudaDeviceReset never matches a cached entry.  The two driver
+// calls are fetched through the runtime, so the library links no driver
+// library of its own.  Called with g_scratch_mutex held.
+typedef int (*CtxGetCurrentFn)(void**);
+typedef int (*CtxGetIdFn)(void*, unsigned long long*);
+wtconv_status current_context_id(unsigned long long* id) {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  if (!get_current || !get_id) {
+    void* f1 = nullptr;
+    void* f2 = nullptr;
+    cudaDriverEntryPointQueryResult q1, q2;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f1, cudaEnableDefault, &q1) != cudaSuccess ||
+        q1 != cudaDriverEntryPointSuccess || !f1)
+      return WTCONV_ERR_CUDA;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &f2, cudaEnableDefault, &q2) != cudaSuccess ||
+        q2 != cudaDriverEntryPointSuccess || !f2)
+      return WTCONV_ERR_CUDA;
+    get_current = reinterpret_cast<CtxGetCurrentFn>(f1);
+    get_id = reinterpret_cast<CtxGetIdFn>(f2);
+  }
+  void* ctx = nullptr;
+  if (get_current(&ctx) != 0) return WTCONV_ERR_CUDA;
+  *id = 0;
+  if (ctx && get_id(ctx, id) != 0) return WTCONV_ERR_CUDA;
+  return WTCONV_OK;
+}
+
+// Device address of g_noalloc_scratch in the current context.  In host code
 // the array's name is only a host-side stand-in, so the address is looked up
-// once per device (with that device current) and cached.
+// with the device current, once per context, and cached with the context's
+// id: after cudaDeviceReset the module is loaded again (the array may move),
+// and the new context's id forces a fresh lookup.
 wtconv_status noalloc_scratch(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return WTCONV_ERR_CUDA;
   if (dev < 0 || dev >= MAX_DEVICES) return WTCONV_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_scratch_mutex);
-  if (!g_scratch_addr[dev]) {
+  unsigned long long id = 0;
+  wtconv_status e = current_context_id(&id);
+  if (e != WTCONV_OK) return e;
+  if (id == 0 || !g_scratch_addr[dev].addr || g_scratch_addr[dev].ctx_id != id) {
     void* p = nullptr;
+    // also makes the device's primary context current when none was
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return WTCONV_ERR_CUDA;
-    g_scratch_addr[dev] = p;
+    if ((e = current_context_id(&id)) != WTCONV_OK) return e;
+    g_scratch_addr[dev] = ScratchAddr{id, p};
   }
-  *out = g_scratch_addr[dev];
+  *out = g_scratch_addr[dev].addr;
   return WTCONV_OK;
 }
 }  // namespace
+
+extern "C" {
+
+size_t wtconv_noalloc_scratch_bytes(void) { return WTCONV_NOALLOC_SCRATCH_BYTES; }
 
 wtconv_status wtconv_backward_weight_noalloc(const wtconv_desc* desc, const void* x, const void* dy,
                                              const float* w0, const float* b0, const float* s0, const float* wl,

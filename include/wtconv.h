@@ -144,7 +144,10 @@ wtconv_status wtconv_backward_data(const wtconv_desc* desc, const void* dy,
                                    void* ws, size_t ws_bytes, void* stream);
 
 /* Backward weight pass: gradients of <y, dy> with respect to every
- * parameter, with G_0[c,u,v] = sum_{n,i,j} dy[n,c,i,j] x[n,c,i+u-r,j+v-r]
+ * parameter (arXiv:2608.10805, abstract: the layer is trained, so its
+ * learned weights and per-channel scales need gradients; the Haar pyramids
+ * of x and dy are recomputed on chip, reformulation (1)), with
+ * G_0[c,u,v] = sum_{n,i,j} dy[n,c,i,j] x[n,c,i+u-r,j+v-r]
  * and G_l[c,s,u,v] = sum dZ_l[c,s](i,j) sub_l[c,s](i+u-r,j+v-r), where
  * dZ_l = Haar pyramid of dy and sub_l = Haar pyramid of x:
  *   dw0 = s0 G_0   db0 = s0 sum(dy)   ds0 = sum_uv w0 G_0 + b0 sum(dy)
@@ -159,10 +162,10 @@ wtconv_status wtconv_backward_weight(const wtconv_desc* desc, const void* x,
                                      float* dwl, float* dsl, void* ws,
                                      size_t ws_bytes, void* stream);
 
-/* Both backward passes in one call (dx and every parameter gradient), as
- * wtconv_backward_data followed by wtconv_backward_weight but sharing the
- * reads of x and dy where the shape allows.  Needs
- * wtconv_workspace_size(desc, 3) bytes of ws. */
+/* Both backward passes in one call (dx and every parameter gradient):
+ * wtconv_backward_data, then wtconv_backward_weight, launched in that order
+ * on `stream` with one workspace; the results equal those of the two calls.
+ * Needs wtconv_workspace_size(desc, 3) bytes of ws. */
 wtconv_status wtconv_backward(const wtconv_desc* desc, const void* x,
                               const void* dy, const float* w0, const float* b0,
                               const float* s0, const float* wl, const float* sl,
@@ -184,12 +187,17 @@ wtconv_status wtconv_backward(const wtconv_desc* desc, const void* x,
  *
  * The per-CTA partial sums go to a file-scope device array of
  * WTCONV_NOALLOC_SCRATCH_BYTES instead; the library then uses fewer CTAs per
- * channel if needed so they fit.  Shapes whose partial sums for one CTA per
- * channel, C * (k*k*(1+4L)+1) floats plus a 16-byte header, exceed that size
- * are rejected with WTCONV_ERR_SCRATCH_LIMIT before anything touches the GPU.
- * The first call on each device looks up the array's device address (with
- * that device current) and caches it; make that first call before any stream
- * capture.  The call allocates nothing (no cudaMalloc, no cudaFree, no
+ * channel if needed so they fit.  Planes too large for one SM (the row-band
+ * path) also keep there the raw LL planes that each level hands to the next:
+ * 2 * N * C * (H/2^l) * (W/2^l) floats for every level l = 1 .. L-1.  Shapes
+ * whose LL planes plus the partial sums of one CTA per channel,
+ * C * (k*k*(1+4L)+1) floats, plus a 16-byte header and 16 bytes of
+ * alignment, exceed the array are rejected with WTCONV_ERR_SCRATCH_LIMIT
+ * before anything touches the GPU.
+ * The first call in each CUDA context of a device looks up the array's
+ * device address (with that device current) and caches it with the
+ * context's id, so a context created again after cudaDeviceReset gets a
+ * fresh lookup; make the first call in a context before any stream capture.  The call allocates nothing (no cudaMalloc, no cudaFree, no
  * allocating library routine).  Every call on a device shares the one array,
  * which keeps the last call's contents (each call overwrites every partial it
  * reads): calls that overlap on the GPU, e.g. on two streams, race and must
@@ -203,6 +211,11 @@ wtconv_status wtconv_backward_weight_noalloc(const wtconv_desc* desc,
                                              const float* sl, float* dw0,
                                              float* db0, float* ds0, float* dwl,
                                              float* dsl, void* stream);
+
+/* WTCONV_NOALLOC_SCRATCH_BYTES as this build of the library has it (for
+ * callers that load the library at run time and want the limit from the
+ * binary itself).  No counterpart in the paper. */
+size_t wtconv_noalloc_scratch_bytes(void);
 
 /* Bytes of the folded-weight block of `desc` (0 when desc is invalid): per
  * channel, s0*w0 and s0*b0, then 2^-l s_l[s] w_l[s] for every level l and

@@ -43,6 +43,8 @@ int main(void) {
          (int)wtconv_backward_weight_noalloc(&ragged, FAKE, FAKE, fp, fp, fp, fp, fp, op, op, op, op, op, NULL));
   printf("noalloc_huge_c %d\n",
          (int)wtconv_backward_weight_noalloc(&huge_c, FAKE, FAKE, fp, fp, fp, fp, fp, op, op, op, op, op, NULL));
+  printf("scratch_bytes %zu\n", wtconv_noalloc_scratch_bytes());
+  printf("scratch_macro %zu\n", (size_t)WTCONV_NOALLOC_SCRATCH_BYTES);
   printf("status_string_ok %s\n", wtconv_status_string(WTCONV_OK) ? "set" : "null");
   printf("status_string_limit %s\n", wtconv_status_string(WTCONV_ERR_SCRATCH_LIMIT) ? "set" : "null");
   return 0;

@@ -51,6 +51,8 @@ def test_c_caller_gets_host_side_errors(c_results):
     assert int(c_results["noalloc_ragged"]) == 2        # WTCONV_ERR_SHAPE
     assert int(c_results["noalloc_huge_c"]) == 7        # WTCONV_ERR_SCRATCH_LIMIT
     assert c_results["status_string_ok"] == "set"
+    # the array size the header promises is the one the library was built with
+    assert int(c_results["scratch_bytes"]) == int(c_results["scratch_macro"]) == _lib.noalloc_scratch_bytes()
     assert c_results["status_string_limit"] == "set"
 
 

@@ -48,6 +48,10 @@ CASES = [
     Workload("bf16_L0", 6, 64, 28, 28, 3, 0, "bf16"),
     # planes too large for one SM: the row-band path, LL planes in the array too
     Workload("band_path_L2", 1, 2, 192, 192, 5, 2, "f32"),
+    # row-band path whose LL planes (7.9 MB) leave room for 10 groups of
+    # partial sums where the workspace entry point would use 24: the array
+    # forces fewer CTAs per channel on the row-band path
+    Workload("band_fewer_groups", 2, 14, 384, 384, 5, 2, "f32"),
 ]
 
 
@@ -74,7 +78,7 @@ def test_noalloc_refuses_shapes_beyond_its_array():
     (no GPU is touched, so this runs anywhere)."""
     lib = wt.load()
     V = 25 * (1 + 4 * 2) + 1
-    C = (_lib.NOALLOC_SCRATCH_BYTES // (V * 4)) + 1
+    C = (_lib.noalloc_scratch_bytes() // (V * 4)) + 1
     d = _lib.WTConvDesc(1, C, 16, 16, 5, 2, 0)
     st = lib.wtconv_backward_weight_noalloc(ctypes.byref(d), *([FAKE] * 12), None)
     assert st == SCRATCH_LIMIT
