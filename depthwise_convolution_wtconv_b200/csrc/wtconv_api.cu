@@ -517,6 +517,9 @@ wtconv_status launch_forward_t(const wtconv_desc* d, const Device& dev, const vo
   }
   DeepPlan D;
   if (d->L >= 2 && !M.fused && build_deep_plan(D, d, dev.max_smem)) {  // else t1 came from the smaller layer
+    // the deep kernel reads x with unchecked 4-wide loads: W is a multiple
+    // of 2^L >= 4 for every descriptor that reaches here
+    if (d->W % 4) return WTCONV_ERR_UNSUPPORTED;
     auto kd = wtconv_deep_kernel<K, IO>;
     const size_t smem = (size_t)D.smem_floats * 4;
     int occ = 0;
@@ -903,7 +906,7 @@ wtconv_status launch_finalize(const wtconv_desc* d, int groups, const float* par
                               const float* s0, const float* wl, const float* sl, float* dw0, float* db0, float* ds0,
                               float* dwl, float* dsl, cudaStream_t st) {
   const FinalizeArgs F{d->C, d->L, d->k * d->k * (1 + 4 * d->L) + 1, groups};
-  const size_t fsmem = (size_t)F.V * sizeof(float);
+  const size_t fsmem = ((size_t)F.V + (size_t)(1 + 4 * d->L) * d->k * d->k) * sizeof(float);
   auto fin = wtconv_bwdw_finalize<K>;
   int occ = 0;
   if (fsmem > 48 * 1024) {

@@ -30,13 +30,14 @@
 namespace wt {
 
 // Stages `rows` rows of a plane (row y0 first; rows outside [0, h) are
-// written as zeros) into shared memory at dst + i*ld + col0, converting to
+// written as zeros) into shared memory at dst + i*ld + COL0, converting to
 // fp32.  The rows come from the plane in global memory, or (SMEM) from a
 // raw copy in shared memory holding row i of the window at raw + i*w.
-// Returns this thread's sum of the staged in-image values when SUM.
-template <typename IN, bool SUM, bool SMEM>
+// Returns this thread's sum of the staged in-image values when SUM.  Full
+// 4-element groups are stored with the widest aligned stores COL0 allows.
+template <typename IN, bool SUM, bool SMEM, int COL0>
 __device__ __forceinline__ float stage_band_rows(const IN* __restrict__ src, const IN* raw, int h, int w, int y0,
-                                                 int rows, float* __restrict__ dst, int ld, int col0, bool vec) {
+                                                 int rows, float* __restrict__ dst, int ld, bool vec) {
   float sum = 0.f;
   const int q4 = (w + 3) >> 2;
   for (int it = threadIdx.x; it < rows * q4; it += NT) {
@@ -49,11 +50,14 @@ __device__ __forceinline__ float stage_band_rows(const IN* __restrict__ src, con
       else
         v = load4(src + (size_t)y * w + x, x, w, vec);
     }
-    float* o = dst + i * ld + col0 + x;
-    o[0] = v.x;
-    if (x + 1 < w) o[1] = v.y;
-    if (x + 2 < w) o[2] = v.z;
-    if (x + 3 < w) o[3] = v.w;
+    float* o = dst + i * ld + COL0 + x;
+    if (x + 3 < w) {
+      sts4<COL0>(o, v);
+    } else {
+      o[0] = v.x;
+      if (x + 1 < w) o[1] = v.y;
+      if (x + 2 < w) o[2] = v.z;
+    }
     if (SUM) sum += (v.x + v.y) + (v.z + v.w);
   }
   return sum;
@@ -126,11 +130,11 @@ __global__ void __launch_bounds__(NT, 2) wtconv_bwband_kernel(const BandPlan P, 
     float sdy;
     if (P.bulk) {
       mb_wait(full, k & 1, abort_flag);
-      stage_band_rows<IN, false, true>(a, rawa, P.H, P.W, y0 - P.ha, P.FR + 2 * P.ha, sa, P.a_ld, r, P.vec);
-      sdy = stage_band_rows<IN, true, true>(bb, rawb, P.H, P.W, y0, P.FR, sb, P.b_ld, 0, P.vec);
+      stage_band_rows<IN, false, true, r>(a, rawa, P.H, P.W, y0 - P.ha, P.FR + 2 * P.ha, sa, P.a_ld, P.vec);
+      sdy = stage_band_rows<IN, true, true, 0>(bb, rawb, P.H, P.W, y0, P.FR, sb, P.b_ld, P.vec);
     } else {
-      stage_band_rows<IN, false, false>(a, nullptr, P.H, P.W, y0 - P.ha, P.FR + 2 * P.ha, sa, P.a_ld, r, P.vec);
-      sdy = stage_band_rows<IN, true, false>(bb, nullptr, P.H, P.W, y0, P.FR, sb, P.b_ld, 0, P.vec);
+      stage_band_rows<IN, false, false, r>(a, nullptr, P.H, P.W, y0 - P.ha, P.FR + 2 * P.ha, sa, P.a_ld, P.vec);
+      sdy = stage_band_rows<IN, true, false, 0>(bb, nullptr, P.H, P.W, y0, P.FR, sb, P.b_ld, P.vec);
     }
     if (P.lvl <= 1) sumdy += sdy;
     __syncthreads();
@@ -149,7 +153,13 @@ __global__ void __launch_bounds__(NT, 2) wtconv_bwband_kernel(const BandPlan P, 
         const float* src = isx ? sa + 2 * q * P.a_ld + r + 2 * jj : sb + 2 * q * P.b_ld + 2 * jj;
         const int ld = isx ? P.a_ld : P.b_ld;
         float ll, lh, hl, hh;
-        haar4(src[0], src[1], src[ld], src[ld + 1], ll, lh, hl, hh);
+        if constexpr (r % 2 == 0) {  // 8-byte aligned pairs: one load per row of the block
+          const float2 top = *reinterpret_cast<const float2*>(src);
+          const float2 bot = *reinterpret_cast<const float2*>(src + ld);
+          haar4(top.x, top.y, bot.x, bot.y, ll, lh, hl, hh);
+        } else {
+          haar4(src[0], src[1], src[ld], src[ld + 1], ll, lh, hl, hh);
+        }
         if (isx) {
           float* o = ss + q * P.s_ld + r + jj;
           o[0] = ll;

@@ -90,6 +90,9 @@ __device__ __forceinline__ void zero_taps(float (&G)[K * K]) {
 
 // Sums the per-CTA partials of channel c = blockIdx.x over its groups in a
 // fixed order and applies the chain rule through the scales and the bias.
+// The channel's base and level kernels are first copied to shared memory by
+// all threads at once, so the per-branch dot products below read no global
+// memory.
 struct FinalizeArgs {
   int C, L, V, ngroups;
 };
@@ -100,10 +103,21 @@ __global__ void wtconv_bwdw_finalize(const FinalizeArgs P, const float* __restri
                                      float* __restrict__ dw0, float* __restrict__ db0, float* __restrict__ ds0,
                                      float* __restrict__ dwl, float* __restrict__ dsl) {
   constexpr int KK = K * K;
-  extern __shared__ float gsum[];
+  extern __shared__ float gsum[];  // V sums, then the channel's kernels: w0 (KK), wl (4L x KK)
+  float* wsm = gsum + P.V;
   const int c = blockIdx.x;
+  for (int e = threadIdx.x; e < (1 + 4 * P.L) * KK; e += blockDim.x) {
+    if (e < KK) {
+      wsm[e] = w0[(size_t)c * KK + e];
+    } else {
+      const int br = (e - KK) / KK, t = (e - KK) - br * KK;
+      const size_t base = ((size_t)(br >> 2) * P.C + c) * 4 + (br & 3);
+      wsm[e] = wl[base * KK + t];
+    }
+  }
   for (int e = threadIdx.x; e < P.V; e += blockDim.x) {
     float a = 0.f;
+#pragma unroll 4
     for (int g = 0; g < P.ngroups; ++g) a += part[((size_t)g * P.C + c) * P.V + e];
     gsum[e] = a;
   }
@@ -112,7 +126,7 @@ __global__ void wtconv_bwdw_finalize(const FinalizeArgs P, const float* __restri
   for (int t = threadIdx.x; t < KK; t += blockDim.x) dw0[(size_t)c * KK + t] = s0[c] * gsum[t];
   if (threadIdx.x == 0) {
     float a = 0.f;
-    for (int t = 0; t < KK; ++t) a = fmaf(w0[(size_t)c * KK + t], gsum[t], a);
+    for (int t = 0; t < KK; ++t) a = fmaf(wsm[t], gsum[t], a);
     ds0[c] = a + b0[c] * sdy;
     db0[c] = s0[c] * sdy;
   }
@@ -126,7 +140,7 @@ __global__ void wtconv_bwdw_finalize(const FinalizeArgs P, const float* __restri
     const int l = br >> 2, s = br & 3;
     const size_t base = ((size_t)l * P.C + c) * 4 + s;
     float a = 0.f;
-    for (int t = 0; t < KK; ++t) a = fmaf(wl[base * KK + t], gsum[KK + br * KK + t], a);
+    for (int t = 0; t < KK; ++t) a = fmaf(wsm[KK + br * KK + t], gsum[KK + br * KK + t], a);
     dsl[base] = a;
   }
 }

@@ -641,7 +641,7 @@ __global__ void __launch_bounds__(DEEP_NT) wtconv_deep_kernel(const DeepPlan P, 
             const int x0 = (rem - by * bw) << 2;
             const IO* src = x + ((size_t)(nb0 + pb) * P.C + c) * plane + (size_t)(by << 2) * P.W + x0;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) v[q][i] = load4(src + (size_t)i * P.W, x0, P.W, true);
+            for (int i = 0; i < 4; ++i) v[q][i] = load4v(src + (size_t)i * P.W);  // W % 4 == 0 here
           }
         }
 #pragma unroll

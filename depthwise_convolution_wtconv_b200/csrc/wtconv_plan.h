@@ -21,7 +21,7 @@ constexpr int MAXL = WTCONV_MAX_LEVELS;
 
 // register-tile shapes (rows x cols of outputs per thread)
 constexpr int DP_R = 2, DP_CW = 4;  // deep-level kernel
-constexpr int BW_R = 4, BW_CW = 8;  // row-band weight gradients, full resolution
+constexpr int BW_R = 8, BW_CW = 4;  // row-band weight gradients, full resolution (4 wide: lanes read consecutive 16-byte words)
 constexpr int B1_R = 4, B1_CW = 4;  // row-band weight gradients, level grid
 
 // Division by a runtime divisor d >= 1 without an integer divide:
