@@ -214,6 +214,8 @@ bool build_main_plan(MainPlan& M, const wtconv_desc* d, int max_smem) {
   const int atx = cdiv_h(M.W1, 4), aty = cdiv_h(TH / 2, 4);
   M.a_pp = d->L >= 1 ? 4 * aty * atx : 0;
   M.f_app = make_fdiv(std::max(1, M.a_pp));
+  M.f_t1q = make_fdiv((M.W1 + 3) / 4);
+  M.f_t1pp = make_fdiv(std::max(1, (TH / 2) * ((M.W1 + 3) / 4)));
   M.f_abt = make_fdiv(aty * atx);
   M.f_atx = make_fdiv(atx);
   int first = 0;
@@ -278,18 +280,12 @@ bool build_deep_plan(DeepPlan& D, const wtconv_desc* d, int max_smem) {
   const int bw = D.W >> 2;
   D.f_stage_per = make_fdiv((D.H >> 2) * bw);
   D.f_stage_x = make_fdiv(bw);
-  int first = 0;
-  for (int l = 0; l <= MAXL + 1; ++l) D.deep_first[l] = 0;
   for (int l = 2; l <= D.L; ++l) {
     const int tx = cdiv_h(D.W >> l, DP_CW), tiles = cdiv_h(D.H >> l, DP_R) * tx;
     D.f_l_tiles[l] = make_fdiv(tiles);
     D.f_l_tx[l] = make_fdiv(tx);
-    D.deep_first[l] = first;
-    first += 4 * tiles;
+    D.f_l_per[l] = make_fdiv(4 * tiles);
   }
-  D.deep_items = first;
-  D.deep_first[D.L + 1] = first;
-  D.f_deep_per = make_fdiv(first);
   const int tq = cdiv_h(D.W1, 4);
   D.f_t1_x = make_fdiv(tq);
   D.f_t1_per = make_fdiv(D.H1 * tq);
@@ -830,6 +826,8 @@ void band_layout(BandPlan& B, int TB) {
   const int sx = bands ? cdiv_h(B.Wl, B1_CW) : 1;
   B.f_sx = make_fdiv(sx);
   B.f_sper = make_fdiv(bands ? cdiv_h(TB, B1_R) * sx : 1);
+  B.f_q4 = make_fdiv(cdiv_h(B.W, 4));
+  B.f_wl = make_fdiv(B.Wl);
 }
 
 // Plan of the launch for level lvl (0 only when L = 0): the largest band
@@ -910,10 +908,10 @@ wtconv_status launch_finalize(const wtconv_desc* d, int groups, const float* par
   auto fin = wtconv_bwdw_finalize<K>;
   int occ = 0;
   if (fsmem > 48 * 1024) {
-    const wtconv_status e = prepare(fin, fsmem, occ, 128);
+    const wtconv_status e = prepare(fin, fsmem, occ, 256);
     if (e != WTCONV_OK) return e;
   }
-  fin<<<F.C, 128, fsmem, st>>>(F, part, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl);
+  fin<<<F.C, 256, fsmem, st>>>(F, part, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl);
   return cudaGetLastError() == cudaSuccess ? WTCONV_OK : WTCONV_ERR_CUDA;
 }
 

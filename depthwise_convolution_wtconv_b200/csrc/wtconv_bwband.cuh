@@ -35,13 +35,26 @@ namespace wt {
 // raw copy in shared memory holding row i of the window at raw + i*w.
 // Returns this thread's sum of the staged in-image values when SUM.  Full
 // 4-element groups are stored with the widest aligned stores COL0 allows.
+// Haar analysis of the 2x2 block at src (rows ld apart): one 8-byte load per
+// row when the block starts on an 8-byte boundary (ALIGNED), else scalars.
+template <bool ALIGNED>
+__device__ __forceinline__ void haar_pair(const float* src, int ld, float& ll, float& lh, float& hl, float& hh) {
+  if constexpr (ALIGNED) {
+    const float2 top = *reinterpret_cast<const float2*>(src);
+    const float2 bot = *reinterpret_cast<const float2*>(src + ld);
+    haar4(top.x, top.y, bot.x, bot.y, ll, lh, hl, hh);
+  } else {
+    haar4(src[0], src[1], src[ld], src[ld + 1], ll, lh, hl, hh);
+  }
+}
+
 template <typename IN, bool SUM, bool SMEM, int COL0>
 __device__ __forceinline__ float stage_band_rows(const IN* __restrict__ src, const IN* raw, int h, int w, int y0,
-                                                 int rows, float* __restrict__ dst, int ld, bool vec) {
+                                                 int rows, float* __restrict__ dst, int ld, bool vec, FDiv fq4) {
   float sum = 0.f;
-  const int q4 = (w + 3) >> 2;
+  const int q4 = fq4.d;  // (w + 3) / 4
   for (int it = threadIdx.x; it < rows * q4; it += NT) {
-    const int i = it / q4, q = it - i * q4;
+    const int i = fq4.div(it), q = it - i * q4;
     const int y = y0 + i, x = 4 * q;
     float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
     if (y >= 0 && y < h) {
@@ -130,11 +143,11 @@ __global__ void __launch_bounds__(NT, 2) wtconv_bwband_kernel(const BandPlan P, 
     float sdy;
     if (P.bulk) {
       mb_wait(full, k & 1, abort_flag);
-      stage_band_rows<IN, false, true, r>(a, rawa, P.H, P.W, y0 - P.ha, P.FR + 2 * P.ha, sa, P.a_ld, P.vec);
-      sdy = stage_band_rows<IN, true, true, 0>(bb, rawb, P.H, P.W, y0, P.FR, sb, P.b_ld, P.vec);
+      stage_band_rows<IN, false, true, r>(a, rawa, P.H, P.W, y0 - P.ha, P.FR + 2 * P.ha, sa, P.a_ld, P.vec, P.f_q4);
+      sdy = stage_band_rows<IN, true, true, 0>(bb, rawb, P.H, P.W, y0, P.FR, sb, P.b_ld, P.vec, P.f_q4);
     } else {
-      stage_band_rows<IN, false, false, r>(a, nullptr, P.H, P.W, y0 - P.ha, P.FR + 2 * P.ha, sa, P.a_ld, P.vec);
-      sdy = stage_band_rows<IN, true, false, 0>(bb, nullptr, P.H, P.W, y0, P.FR, sb, P.b_ld, P.vec);
+      stage_band_rows<IN, false, false, r>(a, nullptr, P.H, P.W, y0 - P.ha, P.FR + 2 * P.ha, sa, P.a_ld, P.vec, P.f_q4);
+      sdy = stage_band_rows<IN, true, false, 0>(bb, nullptr, P.H, P.W, y0, P.FR, sb, P.b_ld, P.vec, P.f_q4);
     }
     if (P.lvl <= 1) sumdy += sdy;
     __syncthreads();
@@ -146,37 +159,30 @@ __global__ void __launch_bounds__(NT, 2) wtconv_bwband_kernel(const BandPlan P, 
       // the TB band rows; raw LL of the band rows to the next level
       const int wl = P.Wl;
       const int nsub = (P.TB + 2 * r) * wl;
-      for (int it = threadIdx.x; it < nsub + P.TB * wl; it += NT) {
-        const bool isx = it < nsub;
-        const int k = isx ? it : it - nsub;
-        const int q = k / wl, jj = k - q * wl;
-        const float* src = isx ? sa + 2 * q * P.a_ld + r + 2 * jj : sb + 2 * q * P.b_ld + 2 * jj;
-        const int ld = isx ? P.a_ld : P.b_ld;
+      const size_t ll0 = ((size_t)n * P.C + c) * P.Hl * wl + (size_t)i0 * wl;
+      for (int it = threadIdx.x; it < nsub; it += NT) {
+        const int q = P.f_wl.div(it), jj = it - q * wl;
+        const float* src = sa + 2 * q * P.a_ld + r + 2 * jj;
         float ll, lh, hl, hh;
-        if constexpr (r % 2 == 0) {  // 8-byte aligned pairs: one load per row of the block
-          const float2 top = *reinterpret_cast<const float2*>(src);
-          const float2 bot = *reinterpret_cast<const float2*>(src + ld);
-          haar4(top.x, top.y, bot.x, bot.y, ll, lh, hl, hh);
-        } else {
-          haar4(src[0], src[1], src[ld], src[ld + 1], ll, lh, hl, hh);
-        }
-        if (isx) {
-          float* o = ss + q * P.s_ld + r + jj;
-          o[0] = ll;
-          o[s_band] = lh;
-          o[2 * s_band] = hl;
-          o[3 * s_band] = hh;
-          const int qi = q - r;
-          if (P.write_ll && qi >= 0 && qi < P.TB)
-            llx[((size_t)n * P.C + c) * P.Hl * wl + (size_t)(i0 + qi) * wl + jj] = ll;
-        } else {
-          float* o = sd + q * P.d_ld + jj;
-          o[0] = ll;
-          o[d_band] = lh;
-          o[2 * d_band] = hl;
-          o[3 * d_band] = hh;
-          if (P.write_ll) lld[((size_t)n * P.C + c) * P.Hl * wl + (size_t)(i0 + q) * wl + jj] = ll;
-        }
+        haar_pair<r % 2 == 0>(src, P.a_ld, ll, lh, hl, hh);
+        float* o = ss + q * P.s_ld + r + jj;
+        o[0] = ll;
+        o[s_band] = lh;
+        o[2 * s_band] = hl;
+        o[3 * s_band] = hh;
+        const int qi = q - r;
+        if (P.write_ll && qi >= 0 && qi < P.TB) llx[ll0 + (size_t)qi * wl + jj] = ll;
+      }
+      for (int it = threadIdx.x; it < P.TB * wl; it += NT) {
+        const int q = P.f_wl.div(it), jj = it - q * wl;
+        float ll, lh, hl, hh;
+        haar_pair<true>(sb + 2 * q * P.b_ld + 2 * jj, P.b_ld, ll, lh, hl, hh);
+        float* o = sd + q * P.d_ld + jj;
+        o[0] = ll;
+        o[d_band] = lh;
+        o[2 * d_band] = hl;
+        o[3 * d_band] = hh;
+        if (P.write_ll) lld[ll0 + (size_t)q * wl + jj] = ll;
       }
       __syncthreads();
     }

@@ -115,10 +115,20 @@ __global__ void wtconv_bwdw_finalize(const FinalizeArgs P, const float* __restri
       wsm[e] = wl[base * KK + t];
     }
   }
+  // groups summed in index order; their loads issued eight at a time
+  const size_t gstride = (size_t)P.C * P.V;
   for (int e = threadIdx.x; e < P.V; e += blockDim.x) {
+    const float* src = part + (size_t)c * P.V + e;
     float a = 0.f;
-#pragma unroll 4
-    for (int g = 0; g < P.ngroups; ++g) a += part[((size_t)g * P.C + c) * P.V + e];
+    int g = 0;
+    for (; g + 8 <= P.ngroups; g += 8) {
+      float v[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) v[q] = __ldg(src + (size_t)(g + q) * gstride);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) a += v[q];
+    }
+    for (; g < P.ngroups; ++g) a += __ldg(src + (size_t)g * gstride);
     gsum[e] = a;
   }
   __syncthreads();

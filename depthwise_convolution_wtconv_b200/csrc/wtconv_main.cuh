@@ -546,10 +546,10 @@ __global__ void __launch_bounds__(MAIN_NT, 4)
     for (int i = tid; i < (P.wblk >> 2); i += MAIN_NT)
       reinterpret_cast<float4*>(slot + P.w_off)[i] = reinterpret_cast<const float4*>(slot + P.wraw_off)[i];
     if (!FUSED && P.L >= 2) {
-      const int rows = P.TH >> 1, q4 = (P.W1 + 3) >> 2;
-      for (int it = tid; it < g.npb * rows * q4; it += MAIN_NT) {
-        const int j = it / (rows * q4), rem = it - j * rows * q4;
-        const int rr = rem / q4, x0 = (rem - rr * q4) << 2;
+      const int q4 = P.f_t1q.d, per = P.f_t1pp.d;  // (W1 + 3) / 4, TH/2 rows of them
+      for (int it = tid; it < g.npb * per; it += MAIN_NT) {
+        const int j = P.f_t1pp.div(it), rem = it - j * per;
+        const int rr = P.f_t1q.div(rem), x0 = (rem - rr * q4) << 2;
         float4 v;
         if (P.bulk_t) {
           v = *reinterpret_cast<const float4*>(slot + P.rawt_off + j * P.rawt_pp + rr * P.W1 + x0);
@@ -629,10 +629,10 @@ __global__ void __launch_bounds__(DEEP_NT) wtconv_deep_kernel(const DeepPlan P, 
       const int bw = P.W >> 2, per = (P.H >> 2) * bw, n = npb * per;
       const BufDesc& d = P.sd[2];
       const int bs = d.ld * d.rows;
-      for (int it0 = threadIdx.x; it0 < n; it0 += 2 * DEEP_NT) {
-        float4 v[2][4];
+      for (int it0 = threadIdx.x; it0 < n; it0 += 4 * DEEP_NT) {
+        float4 v[4][4];
 #pragma unroll
-        for (int q = 0; q < 2; ++q) {
+        for (int q = 0; q < 4; ++q) {
           const int it = it0 + q * DEEP_NT;
           if (it < n) {
             const int pb = P.f_stage_per.div(it);
@@ -645,7 +645,7 @@ __global__ void __launch_bounds__(DEEP_NT) wtconv_deep_kernel(const DeepPlan P, 
           }
         }
 #pragma unroll
-        for (int q = 0; q < 2; ++q) {
+        for (int q = 0; q < 4; ++q) {
           const int it = it0 + q * DEEP_NT;
           if (it < n) {
             const int pb = P.f_stage_per.div(it);
@@ -680,31 +680,33 @@ __global__ void __launch_bounds__(DEEP_NT) wtconv_deep_kernel(const DeepPlan P, 
                     d.ld, d.ld * d.rows, d.ps);
       __syncthreads();
     }
-    const int per = P.deep_items;
-    for (int it = threadIdx.x; it < npb * per; it += DEEP_NT) {
-      const int pb = P.f_deep_per.div(it);
-      int rem = it - pb * per;
-      int l = 2;
-      while (rem >= P.deep_first[l + 1]) ++l;
-      rem -= P.deep_first[l];
-      const int tpb = P.f_l_tiles[l].d;
-      const int s = P.f_l_tiles[l].div(rem);
-      rem -= s * tpb;
-      const int ti = P.f_l_tx[l].div(rem);
-      const int tj = rem - ti * P.f_l_tx[l].d;
-      const BufDesc& d = P.sd[l];
-      const BufDesc& z = P.zd[l];
-      float acc[DP_R][DP_CW];
+    // every level's band convs (no barrier between levels: each reads its own
+    // subbands and writes its own Z planes); the per-level plan entries are
+    // read once per level, outside the tile loop
+    for (int l = 2; l <= P.L; ++l) {
+      const BufDesc d = P.sd[l];
+      const BufDesc z = P.zd[l];
+      const FDiv ft = P.f_l_tiles[l], fx = P.f_l_tx[l], fp = P.f_l_per[l];
+      const float* wlv = sw + (l - 2) * 4 * kk4;
+      for (int it = threadIdx.x; it < npb * fp.d; it += DEEP_NT) {
+        const int pb = fp.div(it);
+        int rem = it - pb * fp.d;
+        const int s = ft.div(rem);
+        rem -= s * ft.d;
+        const int ti = fx.div(rem);
+        const int tj = rem - ti * fx.d;
+        float acc[DP_R][DP_CW];
 #pragma unroll
-      for (int a = 0; a < DP_R; ++a)
+        for (int a = 0; a < DP_R; ++a)
 #pragma unroll
-        for (int b = 0; b < DP_CW; ++b) acc[a][b] = 0.f;
-      conv_tile<K, DP_R, DP_CW>(sm + d.off + pb * d.ps + s * d.ld * d.rows + ti * DP_R * d.ld + tj * DP_CW, d.ld,
-                                sw + ((l - 2) * 4 + s) * kk4, acc);
-      float* o = sm + z.off + pb * z.ps + s * z.ld * z.rows + ti * DP_R * z.ld + tj * DP_CW;
+          for (int b = 0; b < DP_CW; ++b) acc[a][b] = 0.f;
+        conv_tile<K, DP_R, DP_CW>(sm + d.off + pb * d.ps + s * d.ld * d.rows + ti * DP_R * d.ld + tj * DP_CW, d.ld,
+                                  wlv + s * kk4, acc);
+        float* o = sm + z.off + pb * z.ps + s * z.ld * z.rows + ti * DP_R * z.ld + tj * DP_CW;
 #pragma unroll
-      for (int a = 0; a < DP_R; ++a)
-        reinterpret_cast<float4*>(o + a * z.ld)[0] = make_float4(acc[a][0], acc[a][1], acc[a][2], acc[a][3]);
+        for (int a = 0; a < DP_R; ++a)
+          reinterpret_cast<float4*>(o + a * z.ld)[0] = make_float4(acc[a][0], acc[a][1], acc[a][2], acc[a][3]);
+      }
     }
     __syncthreads();
     {

@@ -80,6 +80,7 @@ struct MainPlan {
   FDiv f_bpp, f_bx4;         // fused: 4x4 staging blocks per plane, per block row
   FDiv f_tiles, f_tpp, f_tx, f_stq, f_spp, f_bands, f_C;
   FDiv f_app, f_abt, f_atx;  // phase-A decomposition: per plane, per band, per tile row
+  FDiv f_t1pp, f_t1q;        // t1 rows of a unit: 4-float groups per plane, per row
   int smem_floats;
 };
 
@@ -92,9 +93,8 @@ struct DeepPlan {
   int wblk, wdeep;           // floats per channel of the folded block; offset of its level-2 kernels
   int w_off;                 // folded weights of levels 2..L
   BufDesc sd[MAXL + 1], zd[MAXL + 1];
-  FDiv f_stage_per, f_stage_x, f_deep_per, f_t1_per, f_t1_x;
-  FDiv f_l_tiles[MAXL + 1], f_l_tx[MAXL + 1];
-  int deep_items, deep_first[MAXL + 2];
+  FDiv f_stage_per, f_stage_x, f_t1_per, f_t1_x;
+  FDiv f_l_tiles[MAXL + 1], f_l_tx[MAXL + 1], f_l_per[MAXL + 1];  // per level: tiles per band, per row, per plane
   int smem_floats;
 };
 
@@ -122,6 +122,7 @@ struct BandPlan {
   int smem_floats;
   int vec, write_ll, seg;
   FDiv f_nb, f_bx, f_bper, f_sx, f_sper;
+  FDiv f_q4, f_wl;           // 4-element groups per input row; level-grid width
 };
 
 // One correlation branch of the whole-plane weight-gradient kernel: the
