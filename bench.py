@@ -69,14 +69,24 @@ def algorithmic_counts(wl):
     prm = param_bytes(wl)
     passes = dict(fwd=dict(fma=fma, bytes=2 * S + prm),
                   bwd_data=dict(fma=fma, bytes=2 * S + prm),
-                  bwd_weight=dict(fma=fma, bytes=2 * S + 2 * prm))
+                  bwd_weight=dict(fma=fma, bytes=2 * S + 2 * prm),
+                  bwd=dict(fma=2 * fma, bytes=3 * S + 2 * prm))  # both backward passes in one
     step = dict(fma=3 * fma, bytes=5 * S + 2 * prm, design_bytes=6 * S + 4 * prm)
     return dict(passes=passes, step=step)
 
 
+def fused_backward(wt, desc):
+    """True when the library runs both backward passes of the shape as one
+    fused pass (fewer launches for op 3 than for ops 1 and 2)."""
+    return wt.kernel_launches(desc, 3) < wt.kernel_launches(desc, 1) + wt.kernel_launches(desc, 2)
+
+
 def launches_per_step(wt, desc):
-    """Kernels of this library launched per step (forward, backward-data,
-    backward-weight), as the library reports them for the shape."""
+    """Kernels of this library launched per step (forward, then the fused
+    backward or backward-data and backward-weight), as the library reports
+    them for the shape."""
+    if fused_backward(wt, desc):
+        return wt.kernel_launches(desc, 0) + wt.kernel_launches(desc, 3)
     return sum(wt.kernel_launches(desc, op) for op in (0, 1, 2))
 
 
@@ -84,6 +94,7 @@ PASS_KERNELS = {
     "fwd": "wtconv_fold_kernel + wtconv_main_kernel (+ wtconv_deep_kernel for row-band planes)",
     "bwd_data": "wtconv_fold_kernel + wtconv_main_kernel, flipped (+ wtconv_deep_kernel for row-band planes)",
     "bwd_weight": "wtconv_bwdw_kernel + wtconv_bwdw_finalize (row-band planes: wtconv_bwband_kernel per level)",
+    "bwd": "wtconv_fold_kernel + wtconv_bwd_fused_kernel + wtconv_bwdw_finalize (both backward passes)",
 }
 
 
@@ -233,6 +244,9 @@ class Layer:
         self.ws2 = torch.empty(max(16, wt.workspace_size(self.desc, 2)), dtype=torch.uint8, device=device)
         self.graphs = {}
         self.step_graph = None
+        self.fused = fused_backward(wt, self.desc)
+        self.passes = PASSES + (("bwd",) if self.fused else ())
+        self.step_backward = "two streams"
 
     def fwd(self, st, x=None, y=None):
         p = self.p
@@ -250,38 +264,75 @@ class Layer:
                                 p["s0"], self.Wl, self.sl, grads=self.grads, ws=self.ws if ws is None else ws,
                                 stream=st)
 
+    def bwd(self, st, x=None, dy=None, dx=None):
+        p = self.p
+        self.wt.backward(self.X if x is None else x, self.dY if dy is None else dy, p["W0"], p["b0"], p["s0"],
+                         self.Wl, self.sl, dx=self.dX if dx is None else dx, grads=self.grads, ws=self.ws,
+                         stream=st)
+
     def eager_step(self, st, x=None, dy=None, y=None, dx=None):
         self.fwd(st, x, y)
-        self.bwd_data(st, dy, dx)
-        self.bwd_weight(st, x, dy)
+        if self.step_backward == "fused":
+            self.bwd(st, x, dy, dx)
+        else:
+            self.bwd_data(st, dy, dx)
+            self.bwd_weight(st, x, dy)
 
     def capture(self, stream, warmup, flush):
         """Each pass as a CUDA graph of its own, and the whole step as one
-        graph: the forward, then backward-data and the weight gradients,
-        which are independent, on two streams (a workspace each)."""
+        graph: the forward, then the fused backward where the library fuses
+        the shape's backward passes, else backward-data and the weight
+        gradients, which are independent, on two streams (a workspace
+        each)."""
         cap = torch.cuda.Stream(self.device)
         cap2 = torch.cuda.Stream(self.device)
         cap.wait_stream(stream)
-        for name in PASSES:
+        for name in self.passes:
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=cap):
                 getattr(self, name)(cap)
             self.graphs[name] = g
-        self.step_graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(self.step_graph, stream=cap):
+        steps = {}
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=cap):
             self.fwd(cap)
             cap2.wait_stream(cap)
             self.bwd_weight(cap2, ws=self.ws2)
             self.bwd_data(cap)
             cap.wait_stream(cap2)
+        steps["two streams"] = g
+        if self.fused:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=cap):
+                self.fwd(cap)
+                self.bwd(cap)
+            steps["fused"] = g
         stream.wait_stream(cap)
         for _ in range(warmup):
             flush.fill_(0.0)
-            for name in PASSES:
+            for name in self.passes:
                 self.graphs[name].replay()
-            flush.fill_(0.0)
-            self.step_graph.replay()
+            for g in steps.values():
+                flush.fill_(0.0)
+                g.replay()
         torch.cuda.synchronize(self.device)
+        # the step runs the faster of the two backward forms, timed here on
+        # warm-up replays (L2 flushed before each)
+        best = None
+        for name, g in steps.items():
+            t = 0.0
+            for _ in range(max(3, warmup)):
+                flush.fill_(0.0)
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                g.replay()
+                e1.record(stream)
+                torch.cuda.synchronize(self.device)
+                t += e0.elapsed_time(e1)
+            if best is None or t < best[1]:
+                best = (name, t)
+        self.step_backward = best[0]
+        self.step_graph = steps[best[0]]
 
 
 def timed_steps(steps, run, flush, device, world, nev):
@@ -338,8 +389,10 @@ def measure(layer, args, world, flush, stream, peaks):
     torch.cuda.synchronize(device)
     layer.capture(stream, args.warmup, flush)
 
+    names = layer.passes
+
     def per_pass_flushed(ev):
-        for i, name in enumerate(PASSES):
+        for i, name in enumerate(names):
             if i:
                 flush.fill_(0.0)
             ev[2 * i].record(stream)
@@ -348,7 +401,7 @@ def measure(layer, args, world, flush, stream, peaks):
 
     def per_pass_warm(ev):
         ev[0].record(stream)
-        for i, name in enumerate(PASSES):
+        for i, name in enumerate(names):
             layer.graphs[name].replay()
             ev[i + 1].record(stream)
 
@@ -365,12 +418,12 @@ def measure(layer, args, world, flush, stream, peaks):
         ev[1].record(stream)
 
     K = args.steps
-    evs = timed_steps(K, per_pass_flushed, flush, device, world, 6)
+    evs = timed_steps(K, per_pass_flushed, flush, device, world, 2 * len(names))
     kernels = {n: max_over_ranks(sum(e[2 * i].elapsed_time(e[2 * i + 1]) for e in evs) / K, world, device)
-               for i, n in enumerate(PASSES)}
-    evs = timed_steps(K, per_pass_warm, flush, device, world, 4)
+               for i, n in enumerate(names)}
+    evs = timed_steps(K, per_pass_warm, flush, device, world, len(names) + 1)
     warm = {n: max_over_ranks(sum(e[i].elapsed_time(e[i + 1]) for e in evs) / K, world, device)
-            for i, n in enumerate(PASSES)}
+            for i, n in enumerate(names)}
     evs = timed_steps(K, eager, flush, device, world, 2)
     eager_ms = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in evs), world, device) / K
     t_wall = time.perf_counter()
@@ -379,18 +432,22 @@ def measure(layer, args, world, flush, stream, peaks):
     ms_per_step = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in evs), world, device) / K
 
     counts = algorithmic_counts(wl)
-    roof = pass_roofline(counts, kernels, peaks)
+    # the roofline of the slowest pass the step runs
+    step_passes = ("fwd", "bwd") if layer.step_backward == "fused" else PASSES
+    roof = pass_roofline(counts, {n: kernels[n] for n in step_passes}, peaks)
     hbm_gbs = counts["step"]["bytes"] / (ms_per_step * 1e-3) / 1e9
     return dict(
         workload=wl.name, ms_per_step=ms_per_step, value=world * 1000.0 / ms_per_step, unit="steps/s",
-        kernels_ms=kernels, kernels_ms_warm=warm,
+        kernels_ms=kernels, kernels_ms_warm=warm, fused_backward=layer.fused,
+        step_backward=layer.step_backward,
         roofline=roof,
         step_roofline=step_bound(counts, ms_per_step, peaks),
         hbm={"achieved_gbs": hbm_gbs, "peak_gbs": peaks["hbm_gbs"], "frac": hbm_gbs / peaks["hbm_gbs"],
              "algorithmic_bytes_per_step": counts["step"]["bytes"],
              "design_bytes_per_step": counts["step"]["design_bytes"], "peak_source": peaks["hbm_source"]},
         eager={"ms_per_step": eager_ms, "value": world * 1000.0 / eager_ms, "unit": "steps/s"},
-        gpu_launches_per_step=launches_per_step(layer.wt, layer.desc),
+        gpu_launches_per_step=(launches_per_step(layer.wt, layer.desc) if layer.step_backward == "fused" else
+                               sum(layer.wt.kernel_launches(layer.desc, op) for op in (0, 1, 2))),
         wall_s_timed_region=t_wall,
     )
 
@@ -519,9 +576,14 @@ def run_ours(args, wl, world, rank, local):
         "fma_per_step": counts["step"]["fma"],
         "kernels_ms": m["kernels_ms"],
         "kernels_ms_warm": m["kernels_ms_warm"],
-        "timing": ("the whole step one CUDA graph replay (forward, then backward-data and weight gradients on "
-                   "two streams with a workspace each); kernels_ms: one graph per pass, L2 flushed before each "
-                   "pass; kernels_ms_warm: the pass graphs back to back; CUDA events on the launching stream"),
+        "fused_backward": m["fused_backward"],
+        "step_backward": m["step_backward"],
+        "timing": ("the whole step one CUDA graph replay: the forward, then the backward as step_backward "
+                   "says (\"fused\": one wtconv_backward call; \"two streams\": backward-data and weight "
+                   "gradients on two streams with a workspace each; where the library fuses the shape's "
+                   "backward, the faster of the two on warm-up replays); kernels_ms: one graph per pass (bwd: "
+                   "wtconv_backward), L2 flushed before each pass; kernels_ms_warm: the pass graphs back to "
+                   "back; CUDA events on the launching stream"),
         "eager": m["eager"],
         "e2e": e2e,
         "gpu_launches": m["gpu_launches_per_step"] * args.steps,

@@ -5,6 +5,7 @@
 
 #include <algorithm>
 #include <cstdint>
+#include <cstring>
 #include <initializer_list>
 #include <mutex>
 #include <type_traits>
@@ -130,6 +131,10 @@ int main_slot(MainPlan& M, int TH, int PB) {
     for (int l = 2; l <= M.L; ++l) M.zd[l] = make_plain(pcur, M.H >> l, M.W >> l, {{4, 4}}, 4);
   }
   const int pstride = rup(pcur, 4);
+  // level-0 rows arrive by one tensor copy per unit: its destination starts
+  // on a 128-byte boundary (the slot itself starts MAIN_HEADER floats into
+  // shared memory)
+  if (M.direct) cur = rup(cur + MAIN_HEADER, 32) - MAIN_HEADER;
   for (BufDesc* bd : {&M.xf, &M.s1, &M.t1, &M.zb}) {
     bd->off += cur;
     bd->ps = pstride;
@@ -139,10 +144,11 @@ int main_slot(MainPlan& M, int TH, int PB) {
       bd->off += cur;
       bd->ps = pstride;
     }
-  cur += PB * pstride;
   M.xbuf = 0;
   if (M.direct) {
-    M.xbuf = PB * pstride;
+    M.xbuf = rup(PB * pstride, 32);  // the second buffer, also 128-byte aligned
+    cur += 2 * M.xbuf;
+  } else {
     cur += PB * pstride;
   }
   return rup(cur, 4);
@@ -161,9 +167,10 @@ bool build_main_plan(MainPlan& M, const wtconv_desc* d, int max_smem) {
   M.oW = d->W;
   M.wblk = main_wblk(d);
   M.bulk_t = d->L >= 2 && (M.W1 % 4) == 0;
-  // level-0 fp32 rows of at least 256 bytes go straight to the padded row
-  // buffers (shorter rows: many small copies cost more than staging saves)
-  M.direct = d->L == 0 && d->io == WTCONV_F32 && (d->W % 4) == 0 && d->W >= 64;
+  // level-0 fp32 planes whose rows are 16-byte multiples go straight to the
+  // padded row buffers by one tensor copy per unit (box inner extent W + 8,
+  // at most 256 elements)
+  M.direct = d->L == 0 && d->io == WTCONV_F32 && (d->W % 4) == 0 && d->W + 8 <= 256;
   const int tx = cdiv_h(d->W, 4);
   // Whole planes when at least three CTAs fit per SM (no halo rows staged
   // twice); else the most CTAs per SM (four, then three, two, one) with the
@@ -176,6 +183,7 @@ bool build_main_plan(MainPlan& M, const wtconv_desc* d, int max_smem) {
     const size_t budget = std::min((size_t)max_smem, (size_t)SM_SMEM / occ - 1024);
     for (int cand = d->H; cand >= (pass == 0 ? d->H : 2) && TH < 0; --cand) {
       if (d->H % cand || (cand != d->H && (cand & 1))) continue;
+      if (M.direct && rup(cand, main_r3(d->H, d->L, cand)) + 2 * M.r > 256) continue;  // tensor box rows
       const int tpp = cdiv_h(cand, main_r3(d->H, d->L, cand)) * tx;
       int pb = cand == d->H ? std::max(1, std::min(d->N, MAIN_NT / tpp)) : 1;
       for (; pb >= 1 && TH < 0; --pb) {
@@ -455,6 +463,40 @@ wtconv_status query_device(Device& dev) {
   return WTCONV_OK;
 }
 
+// Tensor maps for the TMA tensor copies.  The encoder is a driver call,
+// fetched once through the runtime (the library links no driver library).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_tiled_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+  });
+  return fn;
+}
+
+// Map of an fp32 activation tensor viewed as [N][C][H][W] (innermost last)
+// whose box is `box` = {columns, rows, channels, batch entries}; elements
+// outside the tensor read as zeros.  Needs W % 4 == 0 (16-byte row stride)
+// and a 16-byte aligned base.
+bool encode_act_map(CUtensorMap* map, const void* base, const wtconv_desc* d, const cuuint32_t (&box)[4]) {
+  EncodeTiledFn enc = encode_tiled_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[4] = {(cuuint64_t)d->W, (cuuint64_t)d->H, (cuuint64_t)d->C, (cuuint64_t)d->N};
+  const cuuint64_t strides[3] = {(cuuint64_t)d->W * 4, (cuuint64_t)d->H * d->W * 4,
+                                 (cuuint64_t)d->C * d->H * d->W * 4};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Makes `kern` launchable with `smem` bytes of dynamic shared memory and
 // returns its resident CTAs per SM for `nthreads` threads.
 template <typename F>
@@ -527,13 +569,19 @@ wtconv_status launch_forward_t(const wtconv_desc* d, const Device& dev, const vo
   }
   const size_t smem = (size_t)M.smem_floats * 4;
   int occ = 0;
+  CUtensorMap xmap;
+  std::memset(&xmap, 0, sizeof(xmap));
+  if (M.direct) {
+    const cuuint32_t box[4] = {(cuuint32_t)M.xf.ld, (cuuint32_t)M.xf.rows, 1, (cuuint32_t)M.PB};
+    if (!encode_act_map(&xmap, x, d, box)) return WTCONV_ERR_CUDA;
+  }
 #define WT_MAIN(R3, FUSED, DIRECT)                                                                      \
   {                                                                                                     \
     auto km = wtconv_main_kernel<K, R3, IO, FUSED, DIRECT>;                                             \
     wtconv_status e = prepare(km, smem, occ, MAIN_NT);                                                  \
     if (e != WTCONV_OK) return e;                                                                       \
     km<<<std::min(M.units, dev.sms * occ), MAIN_NT, smem, st>>>(M, static_cast<const IO*>(x), t1, wfold, \
-                                                                static_cast<IO*>(y), status);           \
+                                                                static_cast<IO*>(y), status, xmap);     \
   }
   if (M.fused) {
     if (M.R3 == 8) WT_MAIN(8, true, false) else WT_MAIN(4, true, false)
@@ -636,23 +684,29 @@ constexpr size_t WS_HEADER = 16;
 int bw_slab(BwPlan& B) {
   const int r = B.r;
   int cur = 0;
+  // dy's buffers: plain for the correlations alone, shifted like x's when
+  // the fused backward also convolves them (dys)
+  auto gbuf = [&](int h, int w, int nb) {
+    return B.dys ? make_shifted(cur, h, w, r, {{4, 4}}, nb) : make_plain(cur, h, w, {{4, 4}}, nb);
+  };
   B.xf = make_shifted(cur, B.H, B.W, r, {{4, 4}}, 1);
-  B.gf = make_plain(cur, B.H, B.W, {{4, 4}}, 1);
+  B.gf = gbuf(B.H, B.W, 1);
   B.s1 = B.g1 = BufDesc{0, 0, 0, 0};
   for (int l = 0; l <= MAXL; ++l) B.sd[l] = B.gd[l] = BufDesc{0, 0, 0, 0};
   if (B.L >= 1) {
     B.s1 = make_shifted(cur, B.H1, B.W1, r, {{4, 4}}, 4);
-    B.g1 = make_plain(cur, B.H1, B.W1, {{4, 4}}, 4);
+    B.g1 = gbuf(B.H1, B.W1, 4);
   }
   for (int l = 2; l <= B.L; ++l) {
     B.sd[l] = make_shifted(cur, B.H >> l, B.W >> l, r, {{4, 4}}, 4);
-    B.gd[l] = make_plain(cur, B.H >> l, B.W >> l, {{4, 4}}, 4);
+    B.gd[l] = gbuf(B.H >> l, B.W >> l, 4);
   }
   return rup(cur, 4);
 }
 
-// Layout for PB planes per unit; false when it needs more than max_smem.
-bool bw_layout(BwPlan& B, int PB, int max_smem) {
+// Layout for PB planes per unit (and `wblk` floats of folded weights, for
+// the fused backward); false when it needs more than max_smem.
+bool bw_layout(BwPlan& B, int PB, int max_smem, int wblk = 0) {
   B.PB = PB;
   B.ps = bw_slab(B);
   const size_t plane_bytes = (size_t)B.H * B.W * B.io_bytes;
@@ -663,6 +717,8 @@ bool bw_layout(BwPlan& B, int PB, int max_smem) {
   cur += PB * B.raw_pp;
   B.raw_g = cur;
   cur += PB * B.raw_pp;
+  B.w_off = cur;
+  cur += rup(wblk, 4);
   const int base = cur;
   for (BufDesc* bd : {&B.xf, &B.gf, &B.s1, &B.g1}) bd->off += base;
   for (int l = 2; l <= B.L; ++l) {
@@ -702,7 +758,7 @@ void bw_branches(BwPlan& B) {
     }
     br.a_off = a->off + s * a->ld * a->rows;
     br.a_ld = a->ld;
-    br.g_off = g->off + s * g->ld * g->rows;
+    br.g_off = g->off + s * g->ld * g->rows + (B.dys ? B.r * g->ld + B.r : 0);  // element (0, 0)
     br.g_ld = g->ld;
     br.seg = KK * b;
     const int tx = cdiv_h(w, 4);
@@ -735,7 +791,8 @@ void bw_branches(BwPlan& B) {
 // Whole-plane plan: the most planes per unit (up to two tiles per thread,
 // one at level 0) that fit two CTAs per SM, else one.  False when one plane
 // does not fit; such shapes run on the row-band path.
-bool build_bw_plan(BwPlan& B, const wtconv_desc* d, int max_smem) {
+// Fields of the weight-gradient plan that depend on the shape alone.
+void bw_init(BwPlan& B, const wtconv_desc* d) {
   B = BwPlan{};
   B.N = d->N;
   B.C = d->C;
@@ -751,8 +808,18 @@ bool build_bw_plan(BwPlan& B, const wtconv_desc* d, int max_smem) {
   B.io_bytes = io_bytes(d);
   B.vec_in = (d->W % 4) == 0;
   B.BH = d->L >= 2 ? 4 : (d->L == 1 ? 2 : 1);
+}
+
+// 4x4 tiles of every correlation branch of one plane.
+int bw_tiles_per_plane(const wtconv_desc* d) {
   int per_plane = cdiv_h(d->H, 4) * cdiv_h(d->W, 4);
   for (int l = 1; l <= d->L; ++l) per_plane += 4 * cdiv_h(d->H >> l, 4) * cdiv_h(d->W >> l, 4);
+  return per_plane;
+}
+
+bool build_bw_plan(BwPlan& B, const wtconv_desc* d, int max_smem) {
+  bw_init(B, d);
+  const int per_plane = bw_tiles_per_plane(d);
   // up to two tiles per thread; level 0 (one branch, short units) up to one,
   // which leaves each CTA several units whose copies overlap the compute
   const int tpt = d->L == 0 ? 1 : 2;
@@ -771,10 +838,178 @@ bool build_bw_plan(BwPlan& B, const wtconv_desc* d, int max_smem) {
   return true;
 }
 
-// True when one plane's whole weight-gradient working set fits one SM.
+// Level-0 fp32 weight gradients fed by tensor copies: two buffer sets of PB
+// planes (x zero-padded, dy plain), the most planes per unit up to one tile
+// per thread that fit two CTAs per SM, else one.  False when the shape does
+// not qualify (L > 0, bf16, W % 4 != 0, a box side over 256) or one plane's
+// two buffer sets do not fit.
+bool build_bw_direct_plan(BwDirectPlan& B, const wtconv_desc* d, int max_smem) {
+  B = BwDirectPlan{};
+  if (d->L != 0 || d->io != WTCONV_F32 || (d->W % 4) != 0) return false;
+  B.N = d->N;
+  B.C = d->C;
+  B.H = d->H;
+  B.W = d->W;
+  B.K = d->k;
+  B.r = d->k / 2;
+  B.kk4 = rup(d->k * d->k, 4);
+  B.V = d->k * d->k + 1;
+  B.xld = d->W + 8;
+  B.xrows = rup(d->H, 4) + 2 * B.r;
+  if (B.xld > 256 || B.xrows > 256) return false;
+  B.xps = B.xld * B.xrows;
+  B.gld = d->W;
+  B.grows = rup(d->H, 4);
+  B.gps = B.gld * B.grows;
+  B.tiles_pp = (B.grows / 4) * (d->W / 4);
+  B.f_tiles = make_fdiv(B.tiles_pp);
+  B.f_tx = make_fdiv(d->W / 4);
+  const int pb0 = std::max(1, std::min({d->N, cdiv_h(BW_NT, B.tiles_pp), 256}));
+  for (const int budget : {(int)(SM_SMEM / 2 - 1024), max_smem}) {
+    for (int pb = pb0; pb >= 1; --pb) {
+      // header: two mbarriers and the abort flag; buffers on 128-byte boundaries
+      int cur = 32;
+      for (int b = 0; b < 2; ++b) {
+        B.xoff[b] = cur;
+        cur += rup(pb * B.xps, 32);
+        B.goff[b] = cur;
+        cur += rup(pb * B.gps, 32);
+      }
+      B.red_off = B.xoff[0];
+      const int need = std::max(cur, B.red_off + BW_NT * (B.kk4 + 1) + BW_NT);
+      if ((size_t)rup(need, 4) * 4 <= (size_t)std::min(budget, max_smem)) {
+        B.PB = pb;
+        B.smem_floats = rup(need, 4);
+        return true;
+      }
+    }
+  }
+  return false;
+}
+
+// True when one plane's whole weight-gradient working set fits one SM
+// (either whole-plane kernel; both write one partial vector per CTA).
 bool bwdw_whole_plane(const wtconv_desc* d) {
+  BwDirectPlan D;
+  if (build_bw_direct_plan(D, d, PLAN_SMEM)) return true;
   BwPlan B;
   return build_bw_plan(B, d, PLAN_SMEM);
+}
+
+// ---- fused backward (whole planes)
+
+// Fills the output-kernel plan of the adjoint pass over B's staged dy: its
+// input buffers are dy's (shifted), its Z planes reuse x's buffers (zb over
+// xf, the deep levels' over s1), read only by the correlations that precede
+// the adjoint phases.  False when those Z planes do not fit there.
+bool bwd_adjoint_plan(const BwPlan& B, const wtconv_desc* d, const wtconv_desc* out, int wblk, MainPlan& M) {
+  M = MainPlan{};
+  M.N = d->N; M.C = d->C; M.H = d->H; M.W = d->W; M.K = d->k; M.r = d->k / 2; M.L = d->L;
+  M.H1 = B.H1;
+  M.W1 = B.W1;
+  M.kk4 = B.kk4;
+  M.io_bytes = B.io_bytes;
+  M.TH = d->H;
+  M.nbands = 1;
+  M.PB = B.PB;
+  M.R3 = 4;
+  M.oH = out->H;
+  M.oW = out->W;
+  M.vec_out = (out->W % 4) == 0;
+  M.wblk = wblk;
+  M.w_off = B.w_off;
+  M.units = 0;
+  const int tx = cdiv_h(d->W, 4);
+  M.tiles_pp = cdiv_h(d->H, 4) * tx;
+  M.tiles = M.PB * M.tiles_pp;
+  M.f_tx = make_fdiv(tx);
+  M.f_tpp = make_fdiv(M.tiles_pp);
+  M.f_C = make_fdiv(d->C);
+  // the weight-gradient plan keeps one slab stride (B.ps) for all of a
+  // plane's buffers; the output-kernel functions read each buffer's own
+  M.xf = B.gf;
+  M.xf.ps = B.ps;
+  M.s1 = B.g1;
+  M.s1.ps = B.ps;
+  for (int l = 0; l <= MAXL; ++l) {
+    M.sd[l] = B.gd[l];
+    M.sd[l].ps = B.ps;
+    M.zd[l] = BufDesc{0, 0, 0, 0};
+  }
+  M.t1 = BufDesc{0, 0, 0, 0};
+  M.zb = BufDesc{0, 0, 0, 0};
+  M.fused = d->L >= 2;
+  if (d->L >= 1) {
+    const int zrows = rup(M.H1, 4), zld = rup(M.W1, 4);
+    if (4 * zrows * zld > B.xf.ld * B.xf.rows) return false;
+    M.zb = BufDesc{B.xf.off, zld, zrows, B.ps};
+    const int atx = cdiv_h(M.W1, 4), aty = cdiv_h(M.H1, 4);
+    M.a_pp = 4 * aty * atx;
+    M.f_app = make_fdiv(M.a_pp);
+    M.f_abt = make_fdiv(aty * atx);
+    M.f_atx = make_fdiv(atx);
+  }
+  int zcur = 0, first = 0;
+  for (int l = 0; l <= MAXL + 1; ++l) M.dfirst[l] = 0;
+  for (int l = 2; l <= d->L; ++l) {
+    const int rows = rup(d->H >> l, 4), ld = rup(d->W >> l, 4);
+    M.zd[l] = BufDesc{B.s1.off + zcur, ld, rows, B.ps};
+    zcur += 4 * rows * ld;
+    const int dtx = cdiv_h(d->W >> l, 4), tiles = cdiv_h(d->H >> l, 4) * dtx;
+    M.f_dtiles[l] = make_fdiv(tiles);
+    M.f_dtx[l] = make_fdiv(dtx);
+    M.dfirst[l] = first;
+    first += 4 * tiles;
+  }
+  if (d->L >= 2 && zcur > 4 * B.s1.ld * B.s1.rows) return false;
+  if (d->L >= 2) M.dfirst[d->L + 1] = first;
+  M.f_dper = make_fdiv(std::max(1, first));
+  return true;
+}
+
+// The fused backward's plan: whole planes, two CTAs per SM (with fewer, the
+// separate passes keep more warps busy), up to two correlation tiles per
+// thread per unit.  False when the shape does not fit; wtconv_backward then
+// runs the two passes.
+bool build_bwd_plan(BwdPlan& Q, const wtconv_desc* d, const wtconv_desc* out, int max_smem) {
+  // k = 7: 49 tap sums per thread on top of the conv tiles exceed the 128
+  // registers of two 256-thread CTAs per SM; the separate passes run it
+  if (d->k > 5) return false;
+  BwPlan& B = Q.B;
+  bw_init(B, d);
+  B.dys = 1;
+  const int wblk = main_wblk(d);
+  const int tpt = d->L == 0 ? 1 : 2;
+  const int pb0 = std::max(1, std::min(d->N, cdiv_h(tpt * BW_NT, bw_tiles_per_plane(d))));
+  const int budget = std::min((int)(SM_SMEM / 2 - 1024), max_smem);
+  for (int pb = pb0; pb >= 1; --pb) {
+    if (!bw_layout(B, pb, budget, wblk)) continue;
+    B.f_sx = make_fdiv(cdiv_h(d->W, 4));
+    B.f_spp = make_fdiv((d->H / B.BH) * cdiv_h(d->W, 4));
+    bw_branches(B);
+    if (bwd_adjoint_plan(B, d, out, wblk, Q.M)) {
+      const MainPlan& M = Q.M;
+      Q.za_off = B.xf.off;
+      Q.za_len = d->L >= 1 ? 4 * M.zb.ld * M.zb.rows : 0;
+      Q.zb_off = B.s1.off;
+      Q.zb_len = 0;
+      for (int l = 2; l <= d->L; ++l) Q.zb_len += 4 * M.zd[l].ld * M.zd[l].rows;
+      return true;
+    }
+  }
+  return false;
+}
+
+bool bwd_fused(const wtconv_desc* d) {
+  BwdPlan Q;
+  return build_bwd_plan(Q, d, d, PLAN_SMEM);
+}
+
+// Workspace of the fused backward: header, the per-CTA partial sums (at
+// most one CTA per plane), then the adjoint folded block.
+size_t bwd_fused_ws_bytes(const wtconv_desc* d) {
+  const size_t V = (size_t)d->k * d->k * (1 + 4 * d->L) + 1;
+  return WS_HEADER + rup16((size_t)d->N * d->C * V * sizeof(float)) + fold_bytes(d);
 }
 
 // ---- row-band weight-gradient path
@@ -915,6 +1150,30 @@ wtconv_status launch_finalize(const wtconv_desc* d, int groups, const float* par
   return cudaGetLastError() == cudaSuccess ? WTCONV_OK : WTCONV_ERR_CUDA;
 }
 
+// Planes per CTA for `units_pb` planes per unit on `slots` resident CTAs:
+// fewest sequential units per CTA slot, counting one more unit per CTA for
+// its fixed costs (clearing its shared memory, the first copy that nothing
+// overlaps, the final reduction and partial write); ties broken towards
+// longer CTAs (fewer partial sums).  0 when no choice has at most
+// max_groups CTAs per channel.
+int planes_per_cta(int N, int C, int units_pb, int slots, int max_groups) {
+  long best = -1;
+  int ppc = 0;
+  for (int q = units_pb; q < N + units_pb; q += units_pb) {
+    const int p = std::min(q, N);
+    const int groups = (N + p - 1) / p;
+    if (groups > max_groups) continue;
+    const long ctas = (long)C * groups;
+    const long cost = ((ctas + slots - 1) / slots) * ((p + units_pb - 1) / units_pb + 1);
+    if (best < 0 || cost <= best) {
+      best = cost;
+      ppc = p;
+    }
+    if (p == N) break;
+  }
+  return ppc;
+}
+
 template <int K, int LC, typename IO>
 wtconv_status launch_bwdw_t(BwPlan& B, const Device& dev, const wtconv_desc* d, const void* x, const void* dy,
                             const float* w0, const float* b0, const float* s0, const float* wl, const float* sl,
@@ -925,25 +1184,8 @@ wtconv_status launch_bwdw_t(BwPlan& B, const Device& dev, const wtconv_desc* d, 
   int occ = 0;
   wtconv_status e = prepare(kern, smem, occ, BW_NT);
   if (e != WTCONV_OK) return e;
-  // planes per CTA: fewest sequential units per CTA slot, counting one more
-  // unit per CTA for its fixed costs (clearing its shared memory, the first
-  // copy that nothing overlaps, the final reduction and partial write); ties
-  // broken towards longer CTAs (fewer partial sums)
-  const int slots = dev.sms * occ;
-  long best = -1;
-  for (int ppc = B.PB; ppc < B.N + B.PB; ppc += B.PB) {
-    const int p = std::min(ppc, B.N);
-    const int groups = (B.N + p - 1) / p;
-    if (groups > max_groups) continue;
-    const long ctas = (long)B.C * groups;
-    const long cost = ((ctas + slots - 1) / slots) * ((p + B.PB - 1) / B.PB + 1);
-    if (best < 0 || cost <= best) {
-      best = cost;
-      B.ppc = p;
-    }
-    if (p == B.N) break;
-  }
-  if (best < 0) return WTCONV_ERR_SCRATCH_LIMIT;
+  B.ppc = planes_per_cta(B.N, B.C, B.PB, dev.sms * occ, max_groups);
+  if (B.ppc == 0) return WTCONV_ERR_SCRATCH_LIMIT;
   B.ngroups = (B.N + B.ppc - 1) / B.ppc;
   kern<<<B.C * B.ngroups, BW_NT, smem, st>>>(B, static_cast<const IO*>(x), static_cast<const IO*>(dy), part, status);
   if (cudaGetLastError() != cudaSuccess) return WTCONV_ERR_CUDA;
@@ -963,6 +1205,26 @@ wtconv_status launch_bwdw_k(BwPlan& B, const Device& dev, const wtconv_desc* d, 
 #undef WT_BW
 }
 
+template <int K>
+wtconv_status launch_bw_direct(BwDirectPlan& B, const Device& dev, const wtconv_desc* d, const void* x,
+                               const void* dy, const float* w0, const float* b0, const float* s0, float* dw0,
+                               float* db0, float* ds0, float* part, int* status, cudaStream_t st, int max_groups) {
+  auto kern = wtconv_bwdw_direct_kernel<K>;
+  const size_t smem = (size_t)B.smem_floats * 4;
+  int occ = 0;
+  wtconv_status e = prepare(kern, smem, occ, BW_NT);
+  if (e != WTCONV_OK) return e;
+  B.ppc = planes_per_cta(B.N, B.C, B.PB, dev.sms * occ, max_groups);
+  if (B.ppc == 0) return WTCONV_ERR_SCRATCH_LIMIT;
+  B.ngroups = (B.N + B.ppc - 1) / B.ppc;
+  CUtensorMap xmap;
+  const cuuint32_t box[4] = {(cuuint32_t)B.xld, (cuuint32_t)B.xrows, 1, (cuuint32_t)B.PB};
+  if (!encode_act_map(&xmap, x, d, box)) return WTCONV_ERR_CUDA;
+  kern<<<B.C * B.ngroups, BW_NT, smem, st>>>(B, static_cast<const float*>(dy), part, status, xmap);
+  if (cudaGetLastError() != cudaSuccess) return WTCONV_ERR_CUDA;
+  return launch_finalize<K>(d, B.ngroups, part, w0, b0, s0, nullptr, nullptr, dw0, db0, ds0, nullptr, nullptr, st);
+}
+
 // Runs the whole-plane weight-gradient kernels with the per-CTA partial sums
 // at `part` and at most `max_groups` CTAs per channel (the partials then
 // fill max_groups * C * V floats).
@@ -973,6 +1235,15 @@ wtconv_status run_bwdw_part(const wtconv_desc* d, const void* x, const void* dy,
   wtconv_status e = query_device(dev);
   if (e != WTCONV_OK) return e;
   if (dev.max_smem < PLAN_SMEM) return WTCONV_ERR_UNSUPPORTED;
+  BwDirectPlan D;
+  if (build_bw_direct_plan(D, d, dev.max_smem)) {
+    switch (d->k) {
+      case 1: return launch_bw_direct<1>(D, dev, d, x, dy, w0, b0, s0, dw0, db0, ds0, part, status, st, max_groups);
+      case 3: return launch_bw_direct<3>(D, dev, d, x, dy, w0, b0, s0, dw0, db0, ds0, part, status, st, max_groups);
+      case 5: return launch_bw_direct<5>(D, dev, d, x, dy, w0, b0, s0, dw0, db0, ds0, part, status, st, max_groups);
+      default: return launch_bw_direct<7>(D, dev, d, x, dy, w0, b0, s0, dw0, db0, ds0, part, status, st, max_groups);
+    }
+  }
   BwPlan B;
   if (!build_bw_plan(B, d, dev.max_smem)) return WTCONV_ERR_UNSUPPORTED;
   switch (d->k) {
@@ -989,6 +1260,68 @@ wtconv_status run_bwdw_part(const wtconv_desc* d, const void* x, const void* dy,
       return launch_bwdw_k<7>(B, dev, d, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, part, status, st,
                               max_groups);
   }
+}
+
+template <int K, int LC, typename IO>
+wtconv_status launch_bwd_fused_t(BwdPlan& Q, const Device& dev, const wtconv_desc* d, const void* x, const void* dy,
+                                 const float* wfold, void* dx, const float* w0, const float* b0, const float* s0,
+                                 const float* wl, const float* sl, float* dw0, float* db0, float* ds0, float* dwl,
+                                 float* dsl, float* part, int* status, cudaStream_t st) {
+  auto kern = wtconv_bwd_fused_kernel<K, LC, IO>;
+  const size_t smem = (size_t)Q.B.smem_floats * 4;
+  int occ = 0;
+  wtconv_status e = prepare(kern, smem, occ, BW_NT);
+  if (e != WTCONV_OK) return e;
+  Q.B.ppc = planes_per_cta(Q.B.N, Q.B.C, Q.B.PB, dev.sms * occ, Q.B.N);
+  if (Q.B.ppc == 0) return WTCONV_ERR_UNSUPPORTED;
+  Q.B.ngroups = (Q.B.N + Q.B.ppc - 1) / Q.B.ppc;
+  kern<<<Q.B.C * Q.B.ngroups, BW_NT, smem, st>>>(Q, static_cast<const IO*>(x), static_cast<const IO*>(dy), wfold,
+                                                 static_cast<IO*>(dx), part, status);
+  if (cudaGetLastError() != cudaSuccess) return WTCONV_ERR_CUDA;
+  return launch_finalize<K>(d, Q.B.ngroups, part, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, st);
+}
+
+// Both backward passes as one fused pass over whole planes (the plan must
+// exist: bwd_fused(d)).  ws: header, partial sums, adjoint folded block.
+// With `out`, x and dy hold zero-padded planes and dx receives only the
+// out->H x out->W image of each.
+wtconv_status run_bwd_fused(const wtconv_desc* d, const wtconv_desc* out, const void* x, const void* dy,
+                            const float* w0, const float* b0, const float* s0, const float* wl, const float* sl,
+                            void* dx, float* dw0, float* db0, float* ds0, float* dwl, float* dsl, void* ws,
+                            cudaStream_t st) {
+  Device dev;
+  wtconv_status e = query_device(dev);
+  if (e != WTCONV_OK) return e;
+  if (dev.max_smem < PLAN_SMEM) return WTCONV_ERR_UNSUPPORTED;
+  BwdPlan Q;
+  if (!build_bwd_plan(Q, d, out, dev.max_smem)) return WTCONV_ERR_UNSUPPORTED;
+  const size_t V = (size_t)d->k * d->k * (1 + 4 * d->L) + 1;
+  int* status = static_cast<int*>(ws);
+  float* part = reinterpret_cast<float*>(static_cast<char*>(ws) + WS_HEADER);
+  float* wfold =
+      reinterpret_cast<float*>(static_cast<char*>(ws) + WS_HEADER + rup16((size_t)d->N * d->C * V * sizeof(float)));
+  if ((e = run_fold(d, w0, nullptr, s0, wl, sl, 1, wfold, st)) != WTCONV_OK) return e;
+  const int lc = d->L >= 2 ? 2 : d->L;
+#define WT_BF(KK, LC, IO)                                                                                      \
+  return launch_bwd_fused_t<KK, LC, IO>(Q, dev, d, x, dy, wfold, dx, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, \
+                                        part, status, st)
+#define WT_BF_K(KK)                                                                   \
+  if (d->io == WTCONV_F32) {                                                          \
+    if (lc == 2) WT_BF(KK, 2, float);                                                 \
+    if (lc == 1) WT_BF(KK, 1, float);                                                 \
+    WT_BF(KK, 0, float);                                                              \
+  } else {                                                                            \
+    if (lc == 2) WT_BF(KK, 2, __nv_bfloat16);                                         \
+    if (lc == 1) WT_BF(KK, 1, __nv_bfloat16);                                         \
+    WT_BF(KK, 0, __nv_bfloat16);                                                      \
+  }
+  switch (d->k) {
+    case 1: WT_BF_K(1)
+    case 3: WT_BF_K(3)
+    default: WT_BF_K(5)
+  }
+#undef WT_BF_K
+#undef WT_BF
 }
 
 template <int K, typename IN>
@@ -1106,7 +1439,7 @@ size_t op_ws(const wtconv_desc* desc, int op) {
     case WTCONV_OP_BACKWARD_WEIGHT:
       return bwdw_ws_bytes(desc);
     case WTCONV_OP_BACKWARD:
-      return std::max(bwdw_ws_bytes(desc), fwd_ws_bytes(desc));
+      return std::max({bwdw_ws_bytes(desc), fwd_ws_bytes(desc), bwd_fused(desc) ? bwd_fused_ws_bytes(desc) : 0});
     case WTCONV_OP_FORWARD_FOLDED:
       return pass_ws_bytes(desc);
     default:
@@ -1237,6 +1570,8 @@ wtconv_status wtconv_backward(const wtconv_desc* desc, const void* x, const void
   if ((e = check_ws(ws, ws_bytes, wtconv_workspace_size(desc, WTCONV_OP_BACKWARD))) != WTCONV_OK) return e;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (!ragged(desc)) {
+    if (bwd_fused(desc))
+      return run_bwd_fused(desc, desc, x, dy, w0, b0, s0, wl, sl, dx, dw0, db0, ds0, dwl, dsl, ws, st);
     e = run_forward(desc, dy, w0, nullptr, s0, wl, sl, dx, 1, ws, st);
     if (e != WTCONV_OK) return e;
     return run_bwdw(desc, x, dy, w0, b0, s0, wl, sl, dw0, db0, ds0, dwl, dsl, ws, st);
@@ -1244,6 +1579,11 @@ wtconv_status wtconv_backward(const wtconv_desc* desc, const void* x, const void
   const wtconv_desc p = padded(desc);
   void* xp = act_slot(&p, WTCONV_OP_BACKWARD, ws, 0);
   void* dyp = act_slot(&p, WTCONV_OP_BACKWARD, ws, 1);
+  if (bwd_fused(&p)) {
+    if ((e = launch_pad(desc, &p, x, xp, st)) != WTCONV_OK) return e;
+    if ((e = launch_pad(desc, &p, dy, dyp, st)) != WTCONV_OK) return e;
+    return run_bwd_fused(&p, desc, xp, dyp, w0, b0, s0, wl, sl, dx, dw0, db0, ds0, dwl, dsl, ws, st);
+  }
   if ((e = launch_pad(desc, &p, dy, dyp, st)) != WTCONV_OK) return e;
   if ((e = run_forward(&p, dyp, w0, nullptr, s0, wl, sl, dx, 1, ws, st, desc)) != WTCONV_OK) return e;
   if ((e = launch_pad(desc, &p, x, xp, st)) != WTCONV_OK) return e;
@@ -1385,7 +1725,7 @@ int wtconv_kernel_launches(const wtconv_desc* desc, int op) {
     case WTCONV_OP_BACKWARD_WEIGHT:
       return weight;
     case WTCONV_OP_BACKWARD:
-      return data + weight;
+      return bwd_fused(desc) ? 3 : data + weight;  // fused: fold, fused pass, finalize
     case WTCONV_OP_FORWARD_FOLDED:
       return pass;
     case WTCONV_OP_FOLD:

@@ -6,6 +6,7 @@
 // wavelet convolution), abstract.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -150,24 +151,50 @@ __device__ __forceinline__ void conv_tile(const float* __restrict__ in, int ld,
 // ------------------------------------------- register-tiled correlation
 // G[u*K+v] += sum_{i<R, j<CW} g[i*ldg + j] * a[(i+u)*lda + (j+v)]
 // a points at (y0-r, x0-r) of the shifted operand, g at (y0, x0) of the
-// gradient operand; both 16-byte aligned, lda/ldg multiples of 4.
-template <int K, int R, int CW>
+// gradient operand; both 16-byte aligned, lda/ldg multiples of 4.  With
+// OFF > 0, a points OFF elements before (y0-r, x0-r) (an aligned window
+// start when the row layout's column padding is not r).  With SUMG, the
+// tile's g values are also added to *gsum.  GV is the width of the g loads
+// (4, 2 or 1 floats): g need only be aligned to GV floats.
+template <int K, int R, int CW, int OFF = 0, bool SUMG = false, int GV = 4>
 __device__ __forceinline__ void corr_tile(const float* __restrict__ a, int lda,
-                                          const float* __restrict__ g, int ldg, float (&G)[K * K]) {
-  constexpr int NIN = CW + K - 1;
+                                          const float* __restrict__ g, int ldg, float (&G)[K * K],
+                                          float* gsum = nullptr) {
+  constexpr int NIN = CW + K - 1 + OFF;
   constexpr int NV = (NIN + 3) / 4;
   float gr[R][CW];
 #pragma unroll
   for (int i = 0; i < R; ++i) {
-    const float4* src = reinterpret_cast<const float4*>(g + i * ldg);
+    if constexpr (GV == 4) {
+      const float4* src = reinterpret_cast<const float4*>(g + i * ldg);
 #pragma unroll
-    for (int q = 0; q < CW / 4; ++q) {
-      const float4 t = src[q];
-      gr[i][4 * q + 0] = t.x;
-      gr[i][4 * q + 1] = t.y;
-      gr[i][4 * q + 2] = t.z;
-      gr[i][4 * q + 3] = t.w;
+      for (int q = 0; q < CW / 4; ++q) {
+        const float4 t = src[q];
+        gr[i][4 * q + 0] = t.x;
+        gr[i][4 * q + 1] = t.y;
+        gr[i][4 * q + 2] = t.z;
+        gr[i][4 * q + 3] = t.w;
+      }
+    } else if constexpr (GV == 2) {
+      const float2* src = reinterpret_cast<const float2*>(g + i * ldg);
+#pragma unroll
+      for (int q = 0; q < CW / 2; ++q) {
+        const float2 t = src[q];
+        gr[i][2 * q + 0] = t.x;
+        gr[i][2 * q + 1] = t.y;
+      }
+    } else {
+#pragma unroll
+      for (int q = 0; q < CW; ++q) gr[i][q] = g[i * ldg + q];
     }
+  }
+  if constexpr (SUMG) {
+    float s = 0.f;
+#pragma unroll
+    for (int i = 0; i < R; ++i)
+#pragma unroll
+      for (int j = 0; j < CW; ++j) s += gr[i][j];
+    *gsum += s;
   }
 #pragma unroll
   for (int row = 0; row < R + K - 1; ++row) {
@@ -188,7 +215,7 @@ __device__ __forceinline__ void corr_tile(const float* __restrict__ a, int lda,
 #pragma unroll
         for (int v = 0; v < K; ++v) {
 #pragma unroll
-          for (int j = 0; j < CW; ++j) G[u * K + v] = fmaf(gr[orow][j], xv[j + v], G[u * K + v]);
+          for (int j = 0; j < CW; ++j) G[u * K + v] = fmaf(gr[orow][j], xv[j + v + OFF], G[u * K + v]);
         }
       }
     }

@@ -27,7 +27,7 @@ namespace wt {
 
 constexpr int MAIN_NT = 128;
 constexpr int MAIN_HEADER = 4;       // floats: mbarrier (8 bytes), abort flag
-constexpr int DEEP_NT = 256;
+constexpr int DEEP_NT = 512;
 
 // ------------------------------------------------------------ mbarriers
 __device__ __forceinline__ unsigned smem_u32(const void* p) { return (unsigned)__cvta_generic_to_shared(p); }
@@ -430,46 +430,48 @@ __device__ __forceinline__ void main_issue(const MainPlan& P, float* slot, uint6
   }
 }
 
-// Level-0 fp32 planes at least 32 wide: one unit's bulk copies straight into
-// row buffer `buf` (row y of plane j at (y - y0 + r) * ld + 4, 16-byte
-// aligned), no staging pass; issued by the lanes of warp 0 after lane 0 has
-// set the phase's byte count.  The folded weights come as for the other
-// paths.
-__device__ __forceinline__ void main_issue_direct(const MainPlan& P, float* slot, uint64_t* full, const UnitGeo& g,
-                                                  int buf, const float* __restrict__ x,
+// One tile-mode tensor copy (TMA) of the box at element coordinates
+// (x, y, c, n) of a 4-D tensor map into shared memory at dst (128-byte
+// aligned), completing on mbarrier `bar`.  Elements of the box outside the
+// tensor arrive as zeros.
+__device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, int x, int y, int c, int n,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5}], "
+      "[%6];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(c), "r"(n), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Level-0 fp32 planes: one unit's input rows straight into row buffer `buf`
+// by one tensor copy of the map over x viewed as [N][C][H][W]: the box of
+// PB planes x (rup(TH, R3) + 2r) rows x (W + 8) columns at (column -4, row
+// y0 - r, channel c, batch entry nb0), so that row y of plane j lands at
+// (y - y0 + r) * ld + x + 4 and the rows and columns outside the plane
+// (the zero padding) arrive as zeros; no staging pass.  The folded weights
+// come by a bulk copy as for the other paths.  Thread 0 issues.
+__device__ __forceinline__ void main_issue_tensor(const MainPlan& P, float* slot, uint64_t* full, const UnitGeo& g,
+                                                  int buf, const CUtensorMap* xmap,
                                                   const float* __restrict__ wfold) {
-  const int lane = threadIdx.x & 31;
-  const int nrows = g.y_hi - g.y_lo;
-  const unsigned brow = (unsigned)(P.W * 4);
-  if (lane == 0) {
-    const unsigned bw = (unsigned)(P.wblk * 4);
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(full)),
-                 "r"(bw + brow * nrows * g.npb)
-                 : "memory");
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-            smem_u32(slot + P.wraw_off)),
-        "l"(wfold + (size_t)g.c * P.wblk), "r"(bw), "r"(smem_u32(full))
-        : "memory");
-  }
-  __syncwarp();
-  for (int q = lane; q < g.npb * nrows; q += 32) {
-    const int j = q / nrows, yy = g.y_lo + (q - j * nrows);
-    float* dst = slot + P.xf.off + buf * P.xbuf + j * P.xf.ps + (yy - g.y0 + P.r) * P.xf.ld + 4;
-    const float* src = x + plane_index(P, g, j) * P.H * P.W + (size_t)yy * P.W;
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                     smem_u32(dst)),
-                 "l"(src), "r"(brow), "r"(smem_u32(full))
-                 : "memory");
-  }
+  const unsigned bw = (unsigned)(P.wblk * 4);
+  const unsigned bx = (unsigned)(P.xf.ld * P.xf.rows * P.PB * 4);
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(full)), "r"(bw + bx)
+               : "memory");
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(slot + P.wraw_off)),
+      "l"(wfold + (size_t)g.c * P.wblk), "r"(bw), "r"(smem_u32(full))
+      : "memory");
+  tma_load_4d(slot + P.xf.off + buf * P.xbuf, xmap, -4, g.y0 - P.r, g.c, g.nb0, full);
 }
 
 template <int K, int R3, typename IO, bool FUSED, bool DIRECT>
 __global__ void __launch_bounds__(MAIN_NT, 4)
     wtconv_main_kernel(const MainPlan P, const IO* __restrict__ x, const float* __restrict__ t1g,
-                       const float* __restrict__ wfold, IO* __restrict__ y, int* __restrict__ status) {
-  extern __shared__ float4 smem4[];
+                       const float* __restrict__ wfold, IO* __restrict__ y, int* __restrict__ status,
+                       const __grid_constant__ CUtensorMap xmap) {
+  extern __shared__ __align__(128) float4 smem4[];
   float* sm = reinterpret_cast<float*>(smem4);
   uint64_t* full = reinterpret_cast<uint64_t*>(sm);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + 2);
@@ -484,8 +486,7 @@ __global__ void __launch_bounds__(MAIN_NT, 4)
   const int myunits = (int)blockIdx.x < P.units ? (P.units - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
   float* slot = sm + P.slot0;
   if constexpr (DIRECT) {
-    if (tid < 32 && myunits > 0)
-      main_issue_direct(P, slot, full, unit_geo(P, blockIdx.x), 0, reinterpret_cast<const float*>(x), wfold);
+    if (tid == 0 && myunits > 0) main_issue_tensor(P, slot, full, unit_geo(P, blockIdx.x), 0, &xmap, wfold);
   } else {
     if (tid == 0 && myunits > 0) main_issue<IO>(P, slot, full, unit_geo(P, blockIdx.x), x, t1g, wfold);
   }
@@ -495,25 +496,6 @@ __global__ void __launch_bounds__(MAIN_NT, 4)
     // every thread waits on every phase in order, so a parity wait is exact
     mb_wait(full, k & 1, abort_flag);
     const int n = (FUSED || DIRECT) ? 0 : g.npb * P.stage_pp;
-    if constexpr (DIRECT) {
-      // The halo rows of the first and last band lie outside the image and
-      // must read as zero, but the buffer may hold another band's rows there
-      // (bands divide H, so no other row is outside; whole planes never
-      // write those rows at all).  The fence orders these generic stores
-      // before the bulk copies that later refill the rows.
-      constexpr int hx = K / 2;
-      if (P.nbands > 1 && (g.y0 == 0 || g.y0 + P.TH == P.H)) {
-        const int rr0 = g.y0 == 0 ? 0 : P.TH + hx;
-        const int q = P.xf.ld >> 2;
-        for (int it = tid; it < g.npb * hx * q; it += MAIN_NT) {
-          const int j = it / (hx * q), rem = it - j * hx * q;
-          const int rr = rem / q, cx = (rem - rr * q) << 2;
-          *reinterpret_cast<float4*>(slot + P.xf.off + (k & 1) * P.xbuf + j * P.xf.ps + (rr0 + rr) * P.xf.ld + cx) =
-              make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      }
-    }
     if constexpr (FUSED) {
       const int nb = g.npb * P.f_bpp.d;
       for (int it = tid; it < nb; it += MAIN_NT) {
@@ -563,9 +545,8 @@ __global__ void __launch_bounds__(MAIN_NT, 4)
     __syncthreads();
     if (*abort_flag) break;  // uniform: read after the barrier
     if constexpr (DIRECT) {
-      if (tid < 32 && k + 1 < myunits)
-        main_issue_direct(P, slot, full, unit_geo(P, blockIdx.x + (k + 1) * gridDim.x), (k + 1) & 1,
-                          reinterpret_cast<const float*>(x), wfold);
+      if (tid == 0 && k + 1 < myunits)
+        main_issue_tensor(P, slot, full, unit_geo(P, blockIdx.x + (k + 1) * gridDim.x), (k + 1) & 1, &xmap, wfold);
     } else {
       if (tid == 0 && k + 1 < myunits)
         main_issue<IO>(P, slot, full, unit_geo(P, blockIdx.x + (k + 1) * gridDim.x), x, t1g, wfold);

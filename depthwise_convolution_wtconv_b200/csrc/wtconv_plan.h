@@ -156,6 +156,39 @@ struct BwPlan {
   BwBranch br[BW_MAXB];
   int red_off;                     // final reduction: BW_NT * (kk4 + 1) + BW_NT floats (over the slab)
   int smem_floats;
+  int dys;                         // dy buffers shifted like x's (the fused backward reads them as conv inputs)
+  int w_off;                       // fused backward: the channel's adjoint folded weights
+};
+
+// Plan of the fused backward kernel (whole planes): the weight-gradient plan
+// B (with dy staged in the shifted layout) and, for the backward-data pass
+// over the same staged dy, an output-kernel plan M whose input buffers are
+// B's dy buffers and whose Z planes reuse B's x-side buffers once the
+// correlations are done.
+struct BwdPlan {
+  BwPlan B;
+  MainPlan M;
+  // ranges of each plane's slab the adjoint writes over x's buffers (zb over
+  // xf, the deep Z planes over s1): cleared before the next unit, since x's
+  // staging writes only the interiors and relies on zero borders
+  int za_off, za_len, zb_off, zb_len;
+};
+
+// Plan of the level-0 fp32 weight-gradient kernel fed by tensor copies: a
+// CTA owns channel c and planes [g*ppc, (g+1)*ppc), PB planes per unit, in
+// two buffer sets (the next unit's copies land in one while the CTA works on
+// the other).  x arrives zero-padded: row y of plane j at
+// xoff + j*xps + (y + r) * xld + x + 4 (xld = W + 8, 128-byte aligned
+// destination); dy plain: goff + j*gps + y * gld + x (gld = W).  The final
+// reduction uses BW_NT * (kk4 + 1) + BW_NT floats at red_off.
+struct BwDirectPlan {
+  int N, C, H, W, K, r, kk4, V;
+  int PB, ppc, ngroups;
+  int xld, xrows, xps, gld, grows, gps;
+  int xoff[2], goff[2];
+  int tiles_pp;
+  FDiv f_tiles, f_tx;  // 4x4 tiles per plane, per tile row
+  int red_off, smem_floats;
 };
 
 }  // namespace wt

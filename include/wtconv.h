@@ -49,7 +49,8 @@
  *     forward and backward-data passes keep the folded weights of every
  *     channel and, for L >= 2, the synthesis of levels >= 2 at level-1
  *     resolution (fp32, N*C*(H/2)*(W/2)); the weight-gradient passes keep
- *     their per-CTA partial sums.  For sides that are not multiples of 2^L
+ *     their per-CTA partial sums (the fused backward: the partial sums and
+ *     the adjoint's folded weights).  For sides that are not multiples of 2^L
  *     it also holds zero-padded copies of the call's input planes (x or dy;
  *     both for the weight-gradient passes).  The workspace is required.
  *   - Arithmetic is fp32 throughout; bf16 I/O is rounded to nearest even on
@@ -162,10 +163,19 @@ wtconv_status wtconv_backward_weight(const wtconv_desc* desc, const void* x,
                                      float* dwl, float* dsl, void* ws,
                                      size_t ws_bytes, void* stream);
 
-/* Both backward passes in one call (dx and every parameter gradient):
- * wtconv_backward_data, then wtconv_backward_weight, launched in that order
- * on `stream` with one workspace; the results equal those of the two calls.
- * Needs wtconv_workspace_size(desc, 3) bytes of ws. */
+/* Both backward passes in one call (dx and every parameter gradient).
+ * Source: arXiv:2608.10805, abstract (training): the adjoint of the forward
+ * map in x runs the analysis on dy, which is the same Haar pyramid of dy
+ * the weight gradients correlate against, so for planes held whole in one
+ * SM (k <= 5) one fused pass stages x and dy once per unit and computes the
+ * correlations, then the adjoint data pass, from the same on-chip pyramids
+ * (launches: the adjoint weight fold, the fused pass, the finalize).  Other
+ * shapes (row-band planes, k = 7) run wtconv_backward_data, then
+ * wtconv_backward_weight, in that order on `stream`.  dx equals what
+ * wtconv_backward_data gives, bit for bit; the parameter gradients agree
+ * with wtconv_backward_weight up to the order of the per-CTA partial sums.
+ * Needs wtconv_workspace_size(desc, 3) bytes of ws (for the fused pass: the
+ * header, the partial sums and the adjoint folded block). */
 wtconv_status wtconv_backward(const wtconv_desc* desc, const void* x,
                               const void* dy, const float* w0, const float* b0,
                               const float* s0, const float* wl, const float* sl,

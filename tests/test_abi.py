@@ -55,7 +55,10 @@ def test_workspace_sizes(lib):
     assert lib.wtconv_workspace_size(ctypes.byref(d), 0) == 16 + t1 + folded
     assert lib.wtconv_workspace_size(ctypes.byref(d), 1) == 16 + t1 + folded
     assert lib.wtconv_workspace_size(ctypes.byref(d), 2) == 16 + 2 * 3 * V * 4
-    assert lib.wtconv_workspace_size(ctypes.byref(d), 3) == 16 + max(2 * 3 * V * 4, t1 + folded)
+    # both backward passes: whole 16x16 planes take the fused pass, whose
+    # workspace holds the partial sums and the adjoint folded block at once
+    assert lib.wtconv_workspace_size(ctypes.byref(d), 3) == 16 + max(2 * 3 * V * 4, t1 + folded,
+                                                                     2 * 3 * V * 4 + folded)
     assert lib.wtconv_workspace_size(ctypes.byref(_desc(L=1)), 0) == 16 + 3 * (5 * 28 + 4) * 4
     assert lib.wtconv_workspace_size(ctypes.byref(_desc(L=0)), 0) == 16 + 3 * (28 + 4) * 4
     assert lib.wtconv_workspace_size(ctypes.byref(_desc(k=4)), 2) == 0
@@ -79,11 +82,13 @@ def test_workspace_of_the_row_band_weight_gradient_path(lib):
 
 def test_kernel_launch_counts(lib):
     """Whole 56x56 planes with L = 3: fold + output kernel per data pass, the
-    weight-gradient kernel + finalize; 256x256 planes with L = 5 run as row
-    bands: fold + deep + output kernel, and one launch per level + finalize."""
+    weight-gradient kernel + finalize, and both backward passes fused (fold,
+    fused pass, finalize); 256x256 planes with L = 5 run as row bands: fold +
+    deep + output kernel, and one launch per level + finalize (the backward
+    passes one after the other)."""
     n = lambda d, op: lib.wtconv_kernel_launches(ctypes.byref(d), op)
     whole = _lib.WTConvDesc(32, 96, 56, 56, 5, 3, 0)
-    assert [n(whole, op) for op in range(4)] == [2, 2, 2, 4]
+    assert [n(whole, op) for op in range(4)] == [2, 2, 2, 3]
     bands = _lib.WTConvDesc(16, 64, 256, 256, 5, 5, 1)
     assert [n(bands, op) for op in range(4)] == [3, 3, 6, 9]
     assert n(_lib.WTConvDesc(2, 3, 16, 16, 4, 2, 0), 0) == 0
@@ -102,10 +107,11 @@ def test_workspace_of_ragged_sides(lib):
     V = 25 * (1 + 4 * 2) + 1
     fwd = 16 + t1 + folded                           # 5008, a multiple of 16
     bw = 16 + 2 * 3 * V * 4
+    fused = bw + folded                              # partial sums and the adjoint block together
     assert lib.wtconv_workspace_size(ctypes.byref(d), 0) == fwd + act
     assert lib.wtconv_workspace_size(ctypes.byref(d), 1) == fwd + act
     assert lib.wtconv_workspace_size(ctypes.byref(d), 2) == bw + 2 * act
-    assert lib.wtconv_workspace_size(ctypes.byref(d), 3) == (max(bw, fwd) + 15) // 16 * 16 + 2 * act
+    assert lib.wtconv_workspace_size(ctypes.byref(d), 3) == (max(bw, fwd, fused) + 15) // 16 * 16 + 2 * act
     assert lib.wtconv_workspace_size(ctypes.byref(d), 4) == 16 + t1 + act
     bf = _desc(H=7, W=5, L=1, io=1)                  # 8 x 6 bf16: 2*3*8*6*2 = 576 bytes
     assert lib.wtconv_workspace_size(ctypes.byref(bf), 0) == 16 + 3 * (5 * 28 + 4) * 4 + 576
@@ -115,8 +121,8 @@ def test_ragged_launch_counts_and_noalloc(lib):
     """Ragged sides add one pad launch per input; the no-allocation weight
     gradients refuse them (no room for the copies)."""
     n = lambda d, op: lib.wtconv_kernel_launches(ctypes.byref(d), op)
-    d = _lib.WTConvDesc(32, 96, 55, 54, 5, 3, 0)      # padded to 56 x 56
-    assert [n(d, op) for op in range(6)] == [3, 3, 4, 6, 2, 1]
+    d = _lib.WTConvDesc(32, 96, 55, 54, 5, 3, 0)      # padded to 56 x 56; backward fused
+    assert [n(d, op) for op in range(6)] == [3, 3, 4, 5, 2, 1]
     args = [FAKE] * 12
     assert lib.wtconv_backward_weight_noalloc(ctypes.byref(d), *args, None) == SHAPE
 

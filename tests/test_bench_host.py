@@ -58,11 +58,22 @@ def test_step_and_pass_rooflines_pick_the_slower_bound():
 
 
 def test_launches_per_step_of_the_stage1_workload():
-    """fold + output kernel for each data pass, weight-gradient kernel +
-    finalize: six library kernels per step."""
+    """fold + output kernel for the forward, then the fused backward (fold,
+    fused pass, finalize): five library kernels per step."""
     wl = WORKLOADS["stage1_f32_k5_L3"]
     desc = wt.make_desc(wl.N, wl.C, wl.H, wl.W, wl.k, wl.L, wl.io)
-    assert bench.launches_per_step(wt, desc) == 6
+    assert bench.fused_backward(wt, desc)
+    assert bench.launches_per_step(wt, desc) == 5
+
+
+def test_launches_per_step_of_the_deep_workload():
+    """Row-band planes: the backward passes run apart (forward: fold, deep
+    kernel, output kernel; backward-data the same; weight gradients: one
+    launch per level and the finalize)."""
+    wl = WORKLOADS["deep_bf16_k5_L5"]
+    desc = wt.make_desc(wl.N, wl.C, wl.H, wl.W, wl.k, wl.L, wl.io)
+    assert not bench.fused_backward(wt, desc)
+    assert bench.launches_per_step(wt, desc) == 3 + 3 + 6
 
 
 def test_source_hash_ignores_comments_and_layout_only():

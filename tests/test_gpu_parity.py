@@ -111,6 +111,17 @@ EDGE = [
     Workload("rows_L0_k5_batched", 5, 4, 8, 64, 5, 0, "f32"),
     Workload("rows_L0_k3_reuse", 6, 1000, 8, 64, 3, 0, "f32"),
     Workload("rows_L0_k1", 2, 3, 12, 64, 1, 0, "f32"),
+    # level-0 fp32 planes by tensor copies (zero-padded boxes): the output
+    # kernel and, where two buffer sets fit, the weight-gradient kernel with
+    # no staging pass; heights not multiples of 4, the widest box (W + 8 =
+    # 256), batched small planes with a partial last unit, k = 1 and 7
+    Workload("tma_L0_k3_20x12", 3, 5, 20, 12, 3, 0, "f32"),
+    Workload("tma_L0_k5_h7", 2, 4, 7, 16, 5, 0, "f32"),
+    Workload("tma_L0_k7_8x8_batched", 7, 3, 8, 8, 7, 0, "f32"),
+    Workload("tma_L0_k3_w248", 1, 2, 40, 248, 3, 0, "f32"),
+    Workload("tma_L0_k1_30x40", 2, 2, 30, 40, 1, 0, "f32"),
+    Workload("tma_L0_k5_reuse", 3, 700, 12, 20, 5, 0, "f32"),
+    Workload("tma_L0_k5_bands_300", 1, 2, 300, 64, 5, 0, "f32"),
     # sides not multiples of 2^L (zero-padded copies, cropped results)
     Workload("ragged_13x11_L2", 2, 3, 13, 11, 5, 2, "f32"),
     Workload("ragged_7x9_L3_bf16", 1, 2, 7, 9, 3, 3, "bf16"),
@@ -205,6 +216,51 @@ def test_fused_backward_matches_separate_calls(cuda_ok, wl):
     assert torch.equal(dx, sep["dX"])
     for k, kk in (("dw0", "dW0"), ("db0", "db0"), ("ds0", "ds0"), ("dwl", "dWl"), ("dsl", "dsl")):
         assert torch.allclose(g[k], sep[kk], rtol=1e-6, atol=1e-6), k
+
+
+FUSED_BWD = [
+    Workload("fbwd_stage1_n3", 3, 5, 56, 56, 5, 3, "f32"),
+    Workload("fbwd_bf16_L2", 4, 3, 28, 28, 5, 2, "bf16"),
+    Workload("fbwd_L1_k3", 5, 2, 24, 20, 3, 1, "f32"),
+    Workload("fbwd_L0_k5_small", 9, 3, 14, 14, 5, 0, "f32"),
+    Workload("fbwd_L0_k3_bf16", 3, 2, 24, 24, 3, 0, "bf16"),
+    # k = 7 runs the two passes apart (too many registers for the fused pass)
+    Workload("bwd_L1_k7_apart", 3, 2, 24, 24, 7, 1, "bf16"),
+    Workload("fbwd_L4_k1", 2, 3, 32, 48, 1, 4, "f32"),
+    Workload("fbwd_L3_k3", 2, 2, 40, 40, 3, 3, "f32"),
+    Workload("fbwd_ragged_L3", 3, 2, 53, 45, 3, 3, "f32"),
+    Workload("fbwd_many_units", 13, 300, 16, 16, 5, 2, "f32"),
+    # several units per CTA: the Z planes written over x's buffers must not
+    # leak into the next unit's zero borders
+    Workload("fbwd_units_L1", 40, 3, 16, 16, 3, 1, "f32"),
+    Workload("fbwd_units_L3", 6, 3, 32, 32, 5, 3, "f32"),
+    Workload("fbwd_units_L2_bf16", 9, 2, 24, 24, 5, 2, "bf16"),
+]
+
+
+@pytest.mark.parametrize("wl", FUSED_BWD, ids=[w.name for w in FUSED_BWD])
+def test_fused_backward_against_oracle(cuda_ok, wl):
+    """wtconv_backward (one staging of x and dy per unit on whole planes: the
+    correlations, then the adjoint data pass from the same dy pyramid)
+    against the oracle: dx and every parameter gradient."""
+    inp = make_inputs(wl, 7)
+    d = _dev(inp, wl.io)
+    desc = wt.make_desc(wl.N, wl.C, wl.H, wl.W, wl.k, wl.L, wl.io)
+    dx, g = wt.backward(d["X"], d["dY"], d["W0"], d["b0"], d["s0"], d["Wl"], d["sl"])
+    torch.cuda.synchronize()
+    p = as_float64(inp)
+    ref = oracle.backward(p["X"], p["dY"], p["W0"], p["b0"], p["s0"], p["Wl"], p["sl"])
+    pairs = [(dx, "dX"), (g["dw0"], "dW0"), (g["db0"], "db0"), (g["ds0"], "ds0")]
+    if wl.L:
+        pairs += [(g["dwl"], "dWl"), (g["dsl"], "dsl")]
+    for got, key in pairs:
+        err = _rel(_np(got), ref[key])
+        assert err <= TOL[wl.io], (wl.name, key, err)
+    # k <= 5 takes the fused pass: fold, fused kernel, finalize (plus one pad
+    # per input for sides not multiples of 2^L)
+    pads = 2 if (wl.H % (1 << wl.L) or wl.W % (1 << wl.L)) else 0
+    apart = wt.kernel_launches(desc, 1) + wt.kernel_launches(desc, 2)
+    assert wt.kernel_launches(desc, 3) == (3 + pads if wl.k <= 5 else apart)
 
 
 def test_delta_kernels_on_gpu(cuda_ok):
