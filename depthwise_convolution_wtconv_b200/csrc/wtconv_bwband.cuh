@@ -76,6 +76,80 @@ __device__ __forceinline__ float stage_band_rows(const IN* __restrict__ src, con
   return sum;
 }
 
+// 4 consecutive elements of a staged row in shared memory as one vector
+// load (the row width is a multiple of 4 and x a multiple of 4).
+__device__ __forceinline__ float4 lds4v(const float* p) { return *reinterpret_cast<const float4*>(p); }
+__device__ __forceinline__ float4 lds4v(const __nv_bfloat16* p) {
+  const uint2 raw = *reinterpret_cast<const uint2*>(p);
+  return make_float4(__uint_as_float(raw.x << 16), __uint_as_float(raw.x & 0xffff0000u),
+                     __uint_as_float(raw.y << 16), __uint_as_float(raw.y & 0xffff0000u));
+}
+
+// Levels >= 1 with bulk-copied rows of width W % 4 == 0: staging and the Haar
+// step in one pass.  Each item takes two rows x four columns of one input
+// (the x window: TB + 2r level rows from i0 - r, rows outside the image as
+// zeros; or the dy band: TB level rows), stores the two fp32 rows (x
+// shifted by r columns, dy plain), their two 2x2 blocks' subbands (x: into
+// s, shifted; dy: into d, plain) and the raw LL to the next level; returns
+// this thread's sum of the dy values.
+template <int K, typename IN>
+__device__ __forceinline__ float band_stage_haar(const BandPlan& P, const IN* rawa, const IN* rawb, float* sa, float* sb,
+                                                 float* ss, float* sd, int y0, size_t ll0, float* __restrict__ llx,
+                                                 float* __restrict__ lld) {
+  constexpr int r = K / 2;
+  const int q4 = P.f_q4.d;  // W / 4
+  const int nx = (P.TB + 2 * r) * q4, ny = P.TB * q4;
+  const int s_band = P.s_ld * P.s_rows, d_band = P.d_ld * P.d_rows, wl = P.Wl;
+  const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
+  float sum = 0.f;
+  for (int it = threadIdx.x; it < nx + ny; it += NT) {
+    const bool isx = it < nx;
+    const int e = isx ? it : it - nx;
+    const int q = P.f_q4.div(e), x = (e - q * q4) << 2;
+    const int jj = x >> 1;
+    float l0, h0, g0, k0, l1, h1, g1, k1;
+    if (isx) {
+      const int y = y0 - P.ha + 2 * q;  // rows y, y + 1 of the image are rows 2q, 2q + 1 of the window
+      const float4 v0 = (y >= 0 && y < P.H) ? lds4v(rawa + (size_t)(2 * q) * P.W + x) : zero;
+      const float4 v1 = (y + 1 >= 0 && y + 1 < P.H) ? lds4v(rawa + (size_t)(2 * q + 1) * P.W + x) : zero;
+      float* o = sa + 2 * q * P.a_ld + r + x;
+      sts4<r>(o, v0);
+      sts4<r>(o + P.a_ld, v1);
+      haar4(v0.x, v0.y, v1.x, v1.y, l0, h0, g0, k0);
+      haar4(v0.z, v0.w, v1.z, v1.w, l1, h1, g1, k1);
+      float* so = ss + q * P.s_ld + r + jj;
+      sts2<r>(so, l0, l1);
+      sts2<r>(so + s_band, h0, h1);
+      sts2<r>(so + 2 * s_band, g0, g1);
+      sts2<r>(so + 3 * s_band, k0, k1);
+      const int qi = q - r;
+      if (P.write_ll && qi >= 0 && qi < P.TB) {
+        llx[ll0 + (size_t)qi * wl + jj] = l0;
+        llx[ll0 + (size_t)qi * wl + jj + 1] = l1;
+      }
+    } else {
+      const float4 v0 = lds4v(rawb + (size_t)(2 * q) * P.W + x);
+      const float4 v1 = lds4v(rawb + (size_t)(2 * q + 1) * P.W + x);
+      float* o = sb + 2 * q * P.b_ld + x;
+      *reinterpret_cast<float4*>(o) = v0;
+      *reinterpret_cast<float4*>(o + P.b_ld) = v1;
+      sum += ((v0.x + v0.y) + (v0.z + v0.w)) + ((v1.x + v1.y) + (v1.z + v1.w));
+      haar4(v0.x, v0.y, v1.x, v1.y, l0, h0, g0, k0);
+      haar4(v0.z, v0.w, v1.z, v1.w, l1, h1, g1, k1);
+      float* dd = sd + q * P.d_ld + jj;
+      *reinterpret_cast<float2*>(dd) = make_float2(l0, l1);
+      *reinterpret_cast<float2*>(dd + d_band) = make_float2(h0, h1);
+      *reinterpret_cast<float2*>(dd + 2 * d_band) = make_float2(g0, g1);
+      *reinterpret_cast<float2*>(dd + 3 * d_band) = make_float2(k0, k1);
+      if (P.write_ll) {
+        lld[ll0 + (size_t)q * wl + jj] = l0;
+        lld[ll0 + (size_t)q * wl + jj + 1] = l1;
+      }
+    }
+  }
+  return sum;
+}
+
 template <int K, typename IN>
 __global__ void __launch_bounds__(NT, 2) wtconv_bwband_kernel(const BandPlan P, const IN* __restrict__ A,
                                                               const IN* __restrict__ B, float* __restrict__ llx,
@@ -141,7 +215,13 @@ __global__ void __launch_bounds__(NT, 2) wtconv_bwband_kernel(const BandPlan P, 
     const IN* a = A + ((size_t)n * P.C + c) * plane;
     const IN* bb = B + ((size_t)n * P.C + c) * plane;
     float sdy;
-    if (P.bulk) {
+    const size_t ll0 = ((size_t)n * P.C + c) * P.Hl * P.Wl + (size_t)i0 * P.Wl;
+    // levels >= 1, bulk-copied rows of width W % 4 == 0: staging and Haar step in one pass
+    const bool joint = P.lvl >= 1 && P.bulk && P.vec && (P.W % 4) == 0;
+    if (joint) {
+      mb_wait(full, k & 1, abort_flag);
+      sdy = band_stage_haar<K, IN>(P, rawa, rawb, sa, sb, ss, sd, y0, ll0, llx, lld);
+    } else if (P.bulk) {
       mb_wait(full, k & 1, abort_flag);
       stage_band_rows<IN, false, true, r>(a, rawa, P.H, P.W, y0 - P.ha, P.FR + 2 * P.ha, sa, P.a_ld, P.vec, P.f_q4);
       sdy = stage_band_rows<IN, true, true, 0>(bb, rawb, P.H, P.W, y0, P.FR, sb, P.b_ld, P.vec, P.f_q4);
@@ -153,13 +233,12 @@ __global__ void __launch_bounds__(NT, 2) wtconv_bwband_kernel(const BandPlan P, 
     __syncthreads();
     if (*abort_flag) break;  // uniform: read after the barrier
     if (P.bulk && threadIdx.x == 0 && u + P.ngroups < P.units) issue(u + P.ngroups);
-    if (P.lvl >= 1) {
+    if (P.lvl >= 1 && !joint) {
       // subbands of x over TB + 2r level rows (the halo rows outside the
       // image come out zero from the zero rows staged above) and of dy over
       // the TB band rows; raw LL of the band rows to the next level
       const int wl = P.Wl;
       const int nsub = (P.TB + 2 * r) * wl;
-      const size_t ll0 = ((size_t)n * P.C + c) * P.Hl * wl + (size_t)i0 * wl;
       for (int it = threadIdx.x; it < nsub; it += NT) {
         const int q = P.f_wl.div(it), jj = it - q * wl;
         const float* src = sa + 2 * q * P.a_ld + r + 2 * jj;
