@@ -941,6 +941,28 @@ def ffma_probe():
             **{k: {**v, "frac_of_nominal": v["tfma_per_s"] / peak} for k, v in res.items()}, "clocks": clocks}
 
 
+def passes_once(wl_name, reps, batch=0):
+    """Runs every pass of a workload `reps` times, eagerly and untimed (for
+    profiler captures: each pass's kernels appear in order forward,
+    backward-data, weight gradients, and the fused backward where the
+    library fuses the shape's backward passes); `batch` > 0 replaces N
+    (a smaller case of the same kernels)."""
+    import depthwise_convolution_wtconv_b200 as wt
+    device = torch.device("cuda", 0)
+    wl = WORKLOADS[wl_name]
+    if batch:
+        wl = dataclasses.replace(wl, N=batch)
+    layer = Layer(wt, wl, device, 0)
+    st = torch.cuda.current_stream(device)
+    for _ in range(reps):
+        for name in layer.passes:
+            getattr(layer, name)(st)
+    torch.cuda.synchronize(device)
+    return {"workload": wl_name, "N": wl.N, "passes": list(layer.passes), "reps": reps,
+            "launches": {name: wt.kernel_launches(layer.desc, op) for name, op in
+                         (("fwd", 0), ("bwd_data", 1), ("bwd_weight", 2), ("bwd", 3))}}
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -954,9 +976,15 @@ def main(argv=None):
     ap.add_argument("--no-per-config", action="store_true", help="time the headline workload only")
     ap.add_argument("--no-comparators", action="store_true", help="skip the same-GPU PyTorch comparators")
     ap.add_argument("--ffma-probe", action="store_true", help="measure the FP32 FMA rate and exit")
+    ap.add_argument("--passes-once", type=int, default=0, metavar="R",
+                    help="run every pass of --workload R times, untimed (for profiler captures), and exit")
+    ap.add_argument("--batch", type=int, default=0, help="with --passes-once: batch size N in place of the workload's")
     args = ap.parse_args(argv)
     if args.ffma_probe:
         print(json.dumps(ffma_probe()), flush=True)
+        return
+    if args.passes_once:
+        print(json.dumps(passes_once(args.workload, args.passes_once, args.batch)), flush=True)
         return
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

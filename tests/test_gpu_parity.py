@@ -263,6 +263,37 @@ def test_fused_backward_against_oracle(cuda_ok, wl):
     assert wt.kernel_launches(desc, 3) == (3 + pads if wl.k <= 5 else apart)
 
 
+BANDED = [
+    Workload("band_k3_L1", 8, 64, 192, 192, 3, 1, "f32"),
+    Workload("band_k5_L2_bf16", 4, 64, 192, 192, 5, 2, "bf16"),
+    Workload("band_k7_L1_bf16", 8, 64, 160, 160, 7, 1, "bf16"),
+    Workload("band_k3_L3", 4, 64, 256, 256, 3, 3, "f32"),
+]
+
+
+@pytest.mark.parametrize("wl", BANDED, ids=[w.name for w in BANDED])
+def test_row_bands_on_sampled_planes(cuda_ok, wl):
+    """Row-band shapes with thousands of bands (more than the resident CTAs
+    take in one round) and every odd kernel size.  The layer is independent
+    across (n, c) planes, so the forward and backward-data outputs of
+    sampled planes are checked against the oracle run on those planes
+    alone."""
+    inp = make_inputs(wl, 11)
+    d = _dev(inp, wl.io)
+    y = wt.forward(d["X"], d["W0"], d["b0"], d["s0"], d["Wl"], d["sl"])
+    dx = wt.backward_data(d["dY"], d["W0"], d["s0"], d["Wl"], d["sl"])
+    torch.cuda.synchronize()
+    p = as_float64(inp)
+    for n, c in ((0, 0), (wl.N - 1, wl.C - 1), (wl.N // 2, wl.C // 3)):
+        one = {key: p[key][n:n + 1, c:c + 1] for key in ("X", "dY")}
+        one.update(W0=p["W0"][c:c + 1], b0=p["b0"][c:c + 1], s0=p["s0"][c:c + 1],
+                   Wl=p["Wl"][:, c:c + 1], sl=p["sl"][:, c:c + 1])
+        Y = oracle.forward(one["X"], one["W0"], one["b0"], one["s0"], one["Wl"], one["sl"])
+        dX = oracle.backward(one["X"], one["dY"], one["W0"], one["b0"], one["s0"], one["Wl"], one["sl"])["dX"]
+        assert _rel(_np(y[n:n + 1, c:c + 1]), Y) <= TOL[wl.io], (wl.name, n, c, "Y")
+        assert _rel(_np(dx[n:n + 1, c:c + 1]), dX) <= TOL[wl.io], (wl.name, n, c, "dX")
+
+
 def test_delta_kernels_on_gpu(cuda_ok):
     """Closed form Y = s0 X + sum_l s_l U_{l-1}(X) through the CUDA path."""
     N, C, H, W, k, L = 2, 3, 32, 32, 5, 3
