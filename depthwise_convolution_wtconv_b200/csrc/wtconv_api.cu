@@ -294,9 +294,14 @@ bool build_deep_plan(DeepPlan& D, const wtconv_desc* d, int max_smem) {
     D.f_l_tx[l] = make_fdiv(tx);
     D.f_l_per[l] = make_fdiv(4 * tiles);
   }
+  for (int l = 3; l <= D.L; ++l) {
+    const int px = (D.W >> (l - 1)) / 2;
+    D.f_up_x[l] = make_fdiv(px);
+    D.f_up_per[l] = make_fdiv((D.H >> (l - 1)) * px);
+  }
   const int tq = cdiv_h(D.W1, 4);
   D.f_t1_x = make_fdiv(tq);
-  D.f_t1_per = make_fdiv(D.H1 * tq);
+  D.f_t1_per = make_fdiv((D.H1 / 2) * tq);  // items of two t1 rows by four columns
   return true;
 }
 
@@ -1099,18 +1104,34 @@ bool build_band_plan(BandPlan& B, const wtconv_desc* d, int lvl) {
 int band_first_level(const wtconv_desc* d) { return d->L == 0 ? 0 : 1; }
 
 // CTAs per channel of every band launch (the same for all, so that the
-// partials keep the whole-plane layout): enough CTAs for four per SM, at
-// most one per unit of the launch with the fewest units.  0 if a level
-// does not fit.
+// partials keep the whole-plane layout), at most one per unit of the launch
+// with the fewest units.  The count minimises the first level's time (it
+// carries most of the work): rounds of resident CTAs (two per SM, the
+// kernel's launch bound, or fewer where a level's shared memory allows
+// fewer) times units per CTA plus one for the CTA's fixed costs (clearing
+// its shared memory, the first copy, the reduction), the smallest count on
+// a tie.  0 if a level does not fit.
 int band_groups(const wtconv_desc* d) {
-  int umin = 1 << 30;
+  int umin = 1 << 30, ufirst = 0, per_sm = 2;
   for (int lvl = band_first_level(d); lvl <= d->L; ++lvl) {
     BandPlan B;
     if (!build_band_plan(B, d, lvl)) return 0;
     umin = std::min(umin, B.units);
+    if (lvl == band_first_level(d)) ufirst = B.units;
+    per_sm = std::min(per_sm, (int)(SM_SMEM / ((size_t)B.smem_floats * 4 + 1024)));
   }
-  const int target = (4 * PLAN_SMS + d->C - 1) / d->C;
-  return std::max(1, std::min(umin, target));
+  const long slots = (long)std::max(1, per_sm) * PLAN_SMS;
+  int best = 1;
+  long best_cost = -1;
+  for (int G = 1; G <= umin; ++G) {
+    const long rounds = ((long)d->C * G + slots - 1) / slots;
+    const long cost = rounds * ((ufirst + G - 1) / G + 1);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best = G;
+    }
+  }
+  return best;
 }
 
 // Floats of the raw LL planes of x and dy that level l (1 <= l < L) hands

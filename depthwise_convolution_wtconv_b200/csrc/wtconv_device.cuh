@@ -110,7 +110,9 @@ __device__ __forceinline__ float warp_sum(float v) {
 
 // acc[R][CW] += sum_{u,v<K} w[u*K+v] * in[(orow+u)*ld + (j+v)]
 // `in` points at the input element (y0-r, x0-r) of the tile and must be
-// 16-byte aligned; ld is a multiple of 4 floats.  Each input row is read
+// 16-byte aligned; ld is a multiple of 4 floats.  w is 16-byte aligned and
+// readable up to the next multiple of 4 floats after K*K (the folded
+// blocks reserve kk4 floats per kernel): it is read as float4s.  Each input row is read
 // once (NV float4 loads) and used by every output row it touches.  With
 // OFF > 0, `in` points OFF elements before (y0-r, x0-r) (an aligned window
 // start when the row layout's column padding is not r).
@@ -119,9 +121,16 @@ __device__ __forceinline__ void conv_tile(const float* __restrict__ in, int ld,
                                           const float* __restrict__ w, float (&acc)[R][CW]) {
   constexpr int NIN = CW + K - 1 + OFF;
   constexpr int NV = (NIN + 3) / 4;
-  float wr[K * K];
+  constexpr int NW = (K * K + 3) / 4;
+  float wr[NW * 4];
 #pragma unroll
-  for (int i = 0; i < K * K; ++i) wr[i] = w[i];
+  for (int q = 0; q < NW; ++q) {
+    const float4 t = reinterpret_cast<const float4*>(w)[q];
+    wr[4 * q + 0] = t.x;
+    wr[4 * q + 1] = t.y;
+    wr[4 * q + 2] = t.z;
+    wr[4 * q + 3] = t.w;
+  }
 #pragma unroll
   for (int row = 0; row < R + K - 1; ++row) {
     float xv[NV * 4];

@@ -18,7 +18,8 @@
 //
 // Deep kernel: levels 2..L of a batch of planes on chip (pyramid, every level
 // conv, then the closed-form synthesis of all levels >= 2 at level-1
-// resolution indexed by coordinate bits -- reformulation (2)), written as t1.
+// resolution indexed by coordinate bits -- reformulation (2) -- summed level
+// by level from the deepest), written as t1.
 #pragma once
 
 #include "wtconv_kernels.cuh"
@@ -59,6 +60,12 @@ __device__ __forceinline__ bool mb_wait(uint64_t* b, unsigned parity, volatile i
 __device__ __forceinline__ void mb_drain(uint64_t* b, unsigned parity) {
   for (int i = 0; i < (1 << 22); ++i)
     if (mb_try(b, parity)) return;
+}
+// Starts moving [p, p + bytes) into L2; no completion to wait for.  Issued
+// only for 16-byte aligned ranges whose size is a multiple of 16 bytes.
+__device__ __forceinline__ void l2_prefetch(const void* p, unsigned bytes) {
+  if (((reinterpret_cast<uintptr_t>(p) | bytes) & 15) == 0)
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
 // ------------------------------------------------------------ unit geometry
 // A unit is one band of one plane (nbands > 1) or a batch of npb planes of
@@ -603,6 +610,12 @@ __global__ void __launch_bounds__(DEEP_NT) wtconv_deep_kernel(const DeepPlan P, 
     const int c = u - bt * P.C;
     const int nb0 = bt * P.PB;
     const int npb = (P.N - nb0) < P.PB ? (P.N - nb0) : P.PB;
+    // the next unit's planes start towards L2 while this one is processed
+    // (each plane is contiguous: H*W elements, a multiple of 16 bytes here)
+    if (threadIdx.x < P.PB && u + (int)gridDim.x < units) {
+      const int un = u + gridDim.x, btn = un / P.C, cn = un - btn * P.C, nbn = btn * P.PB + (int)threadIdx.x;
+      if (nbn < P.N) l2_prefetch(x + ((size_t)nbn * P.C + cn) * plane, (unsigned)(plane * sizeof(IO)));
+    }
     // the channel's folded level-2..L weights (contiguous in its block)
     for (int i = threadIdx.x; i < (P.L - 1) * 4 * kk4; i += DEEP_NT) sw[i] = wfold[(size_t)c * P.wblk + P.wdeep + i];
     // level-2 subbands straight from 4x4 blocks of x (two blocks in flight)
@@ -663,13 +676,20 @@ __global__ void __launch_bounds__(DEEP_NT) wtconv_deep_kernel(const DeepPlan P, 
     }
     // every level's band convs (no barrier between levels: each reads its own
     // subbands and writes its own Z planes); the per-level plan entries are
-    // read once per level, outside the tile loop
+    // read once per level, outside the tile loop.  The tiles of all levels
+    // are dealt out as one sequence (thread t takes tiles t, t + DEEP_NT, ...
+    // of it), so the few tiles of the deep levels go to threads with fewer
+    // level-2 tiles.
+    int before = 0;  // tiles of the levels already dealt
     for (int l = 2; l <= P.L; ++l) {
       const BufDesc d = P.sd[l];
       const BufDesc z = P.zd[l];
       const FDiv ft = P.f_l_tiles[l], fx = P.f_l_tx[l], fp = P.f_l_per[l];
       const float* wlv = sw + (l - 2) * 4 * kk4;
-      for (int it = threadIdx.x; it < npb * fp.d; it += DEEP_NT) {
+      int it = (int)threadIdx.x - before % DEEP_NT;
+      if (it < 0) it += DEEP_NT;
+      before += npb * fp.d;
+      for (; it < npb * fp.d; it += DEEP_NT) {
         const int pb = fp.div(it);
         int rem = it - pb * fp.d;
         const int s = ft.div(rem);
@@ -690,52 +710,63 @@ __global__ void __launch_bounds__(DEEP_NT) wtconv_deep_kernel(const DeepPlan P, 
       }
     }
     __syncthreads();
+    // t1(i, j) = sum_{l>=2} sum_s sigma_s(bit_{l-2}(i), bit_{l-2}(j)) Zd_l^s(i >> (l-1), j >> (l-1)).
+    // The terms of levels >= 3 are the same sum one level down, at
+    // (i >> 1, j >> 1), and the LL sign is always +, so the sum is taken
+    // level by level from the deepest: the synthesis of level l's four Z
+    // planes is added into level l-1's LL Z plane, then t1 is the synthesis
+    // of level 2's four planes.  Pixels of level l-1 go in pairs (2j', 2j'+1)
+    // that share their level-l parent (i >> 1, j').
+    for (int l = P.L; l >= 3; --l) {
+      const BufDesc zs = P.zd[l], zt = P.zd[l - 1];
+      const FDiv fx = P.f_up_x[l], fp = P.f_up_per[l];
+      const int bz = zs.ld * zs.rows;
+      for (int it = threadIdx.x; it < npb * fp.d; it += DEEP_NT) {
+        const int pb = fp.div(it);
+        const int rem = it - pb * fp.d;
+        const int i = fx.div(rem);
+        const int jp = rem - i * fx.d;
+        const float* q = sm + zs.off + pb * zs.ps + (i >> 1) * zs.ld + jp;
+        const float sy = (i & 1) ? -1.f : 1.f;
+        const float A = fmaf(sy, q[bz], q[0]), B = fmaf(sy, q[3 * bz], q[2 * bz]);
+        float2* t = reinterpret_cast<float2*>(sm + zt.off + pb * zt.ps + i * zt.ld + 2 * jp);
+        float2 v = *t;
+        v.x += A + B;
+        v.y += A - B;
+        *t = v;
+      }
+      __syncthreads();
+    }
     {
-      // t1(i, j) = sum_{l>=2} sum_s sigma_s(bit_{l-2}(i), bit_{l-2}(j)) Zd_l^s(i >> (l-1), j >> (l-1))
+      // t1 rows 2i' and 2i' + 1, columns j0 .. j0 + 3: parents (i', j0/2) and (i', j0/2 + 1)
       const int tq = P.f_t1_x.d, per1 = P.f_t1_per.d;
       const BufDesc& z2 = P.zd[2];
       const int bz2 = z2.ld * z2.rows;
       for (int it = threadIdx.x; it < npb * per1; it += DEEP_NT) {
         const int pb = P.f_t1_per.div(it);
         const int rem = it - pb * per1;
-        const int i = P.f_t1_x.div(rem);
-        const int j0 = (rem - i * tq) << 2;
-        const float* q = sm + z2.off + pb * z2.ps + (i >> 1) * z2.ld + (j0 >> 1);
+        const int ip = P.f_t1_x.div(rem);
+        const int j0 = (rem - ip * tq) << 2;
+        const float* q = sm + z2.off + pb * z2.ps + ip * z2.ld + (j0 >> 1);
         const float2 zl = *reinterpret_cast<const float2*>(q);
         const float2 zh = *reinterpret_cast<const float2*>(q + bz2);
         const float2 zg = *reinterpret_cast<const float2*>(q + 2 * bz2);
         const float2 zk = *reinterpret_cast<const float2*>(q + 3 * bz2);
-        const float sy = (i & 1) ? -1.f : 1.f;
-        const float a0 = fmaf(sy, zh.x, zl.x), c0 = fmaf(sy, zk.x, zg.x);
-        const float a1 = fmaf(sy, zh.y, zl.y), c1 = fmaf(sy, zk.y, zg.y);
-        float o[4] = {a0 + c0, a0 - c0, a1 + c1, a1 - c1};
-        for (int l = 3; l <= P.L; ++l) {
-          const BufDesc& z = P.zd[l];
-          const int bz = z.ld * z.rows;
-          const float* pz = sm + z.off + pb * z.ps + (i >> (l - 1)) * z.ld + (j0 >> (l - 1));
-          const float syl = ((i >> (l - 2)) & 1) ? -1.f : 1.f;
-          const float A = fmaf(syl, pz[bz], pz[0]), B = fmaf(syl, pz[3 * bz], pz[2 * bz]);
-          if (l == 3) {  // bit1 of j: 0 for j0, j0+1 and 1 for j0+2, j0+3
-            o[0] += A + B;
-            o[1] += A + B;
-            o[2] += A - B;
-            o[3] += A - B;
-          } else {
-            const float sxl = ((j0 >> (l - 2)) & 1) ? -1.f : 1.f;
-            const float v = fmaf(sxl, B, A);
-            o[0] += v;
-            o[1] += v;
-            o[2] += v;
-            o[3] += v;
-          }
-        }
-        float* dst = t1g + ((size_t)(nb0 + pb) * P.C + c) * P.H1 * P.W1 + (size_t)i * P.W1 + j0;
-        if ((P.W1 & 3) == 0) {
-          *reinterpret_cast<float4*>(dst) = make_float4(o[0], o[1], o[2], o[3]);
-        } else {
+        float* dst = t1g + ((size_t)(nb0 + pb) * P.C + c) * P.H1 * P.W1 + (size_t)(2 * ip) * P.W1 + j0;
 #pragma unroll
-          for (int e = 0; e < 4; ++e)
-            if (j0 + e < P.W1) dst[e] = o[e];
+        for (int h = 0; h < 2; ++h) {
+          const float sy = h ? -1.f : 1.f;
+          const float a0 = fmaf(sy, zh.x, zl.x), c0 = fmaf(sy, zk.x, zg.x);
+          const float a1 = fmaf(sy, zh.y, zl.y), c1 = fmaf(sy, zk.y, zg.y);
+          const float o[4] = {a0 + c0, a0 - c0, a1 + c1, a1 - c1};
+          float* row = dst + (size_t)h * P.W1;
+          if ((P.W1 & 3) == 0) {
+            *reinterpret_cast<float4*>(row) = make_float4(o[0], o[1], o[2], o[3]);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              if (j0 + e < P.W1) row[e] = o[e];
+          }
         }
       }
     }

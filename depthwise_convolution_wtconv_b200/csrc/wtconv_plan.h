@@ -95,6 +95,7 @@ struct DeepPlan {
   BufDesc sd[MAXL + 1], zd[MAXL + 1];
   FDiv f_stage_per, f_stage_x, f_t1_per, f_t1_x;
   FDiv f_l_tiles[MAXL + 1], f_l_tx[MAXL + 1], f_l_per[MAXL + 1];  // per level: tiles per band, per row, per plane
+  FDiv f_up_x[MAXL + 1], f_up_per[MAXL + 1];  // l >= 3: pixel pairs of level l-1 per row, per plane
   int smem_floats;
 };
 

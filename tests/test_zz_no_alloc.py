@@ -49,7 +49,7 @@ CASES = [
     # planes too large for one SM: the row-band path, LL planes in the array too
     Workload("band_path_L2", 1, 2, 192, 192, 5, 2, "f32"),
     # row-band path whose LL planes (7.9 MB) leave room for 10 groups of
-    # partial sums where the workspace entry point would use 24: the array
+    # partial sums where the workspace entry point would use 20: the array
     # forces fewer CTAs per channel on the row-band path
     Workload("band_fewer_groups", 2, 14, 384, 384, 5, 2, "f32"),
 ]
