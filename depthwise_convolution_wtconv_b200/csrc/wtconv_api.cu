@@ -16,6 +16,7 @@
 #include "wtconv_main.cuh"
 #include "wtconv_bwband.cuh"
 #include "wtconv_bwdw.cuh"
+#include "wtconv_small.cuh"
 
 namespace wt {
 namespace {
@@ -610,6 +611,70 @@ wtconv_status launch_forward_k(const wtconv_desc* d, const Device& dev, const vo
   return launch_forward_t<K, __nv_bfloat16>(d, dev, x, wfold, y, status, t1, out, st);
 }
 
+// ---- level 0 on small planes: a warp per plane (wtconv_small.cuh)
+
+// Level-0 planes of at most 32x32 (at most 64 4x4 tiles).
+bool small_planes(const wtconv_desc* d) { return d->L == 0 && d->W <= 32 && d->H <= 32; }
+
+void build_small_plan(SmallPlan& S, const wtconv_desc* d) {
+  S = SmallPlan{};
+  S.N = d->N; S.C = d->C; S.H = d->H; S.W = d->W; S.K = d->k; S.r = d->k / 2;
+  S.hw = d->H * d->W;
+  S.TY = cdiv_h(d->H, 4);
+  S.TX = cdiv_h(d->W, 4);
+  S.T = S.TY * S.TX;
+  S.PW = std::max(1, std::min(8, 32 / S.T));
+  // the 4x4 tile reads rows 4 ty .. 4 ty + 3 + 2r and 16-byte groups of
+  // columns up to 4 tx + 4 + 2r (rounded up to 4)
+  S.ld = rup(4 * S.TX + 2 * S.r, 4);
+  S.rows = 4 * S.TY + 2 * S.r;
+  S.xs_pp = S.ld * S.rows;
+  S.kk4 = rup(d->k * d->k, 4);
+  S.tab_off = S.PW * S.xs_pp;  // the plane buffers, then the element table, then weights and biases
+  S.w_off = rup(S.tab_off + S.PW * S.hw, 4);
+  S.buf = rup(S.w_off + S.PW * (S.kk4 + 1), 4);
+  S.wblk = main_wblk(d);
+  S.f_w = make_fdiv(d->W);
+  S.f_hw = make_fdiv(S.hw);
+  S.f_C = make_fdiv(d->C);
+}
+
+// Forward (flip = 0) or backward-data (flip = 1) from the raw parameters
+// (wfold null) or from a folded block.
+template <int K, typename IO>
+wtconv_status launch_small_t(const wtconv_desc* d, const Device& dev, const void* x, const float* wfold,
+                             const float* w0, const float* b0, const float* s0, int flip, void* y, cudaStream_t st) {
+  SmallPlan S;
+  build_small_plan(S, d);
+  const size_t smem = (size_t)(SMALL_NT / 32) * S.buf * sizeof(float);
+  auto k = wtconv_small_kernel<K, IO>;
+  int occ = 0;
+  wtconv_status e = prepare(k, smem, occ, SMALL_NT);
+  if (e != WTCONV_OK) return e;
+  const long long warps = ((long long)d->N * d->C + S.PW - 1) / S.PW;
+  const int grid = (int)std::min<long long>((warps + SMALL_NT / 32 - 1) / (SMALL_NT / 32), (long long)dev.sms * occ);
+  k<<<grid, SMALL_NT, smem, st>>>(S, static_cast<const IO*>(x), wfold, w0, b0, s0, flip, static_cast<IO*>(y));
+  return cudaGetLastError() == cudaSuccess ? WTCONV_OK : WTCONV_ERR_CUDA;
+}
+
+wtconv_status launch_small(const wtconv_desc* d, const void* x, const float* wfold, const float* w0,
+                           const float* b0, const float* s0, int flip, void* y, cudaStream_t st) {
+  Device dev;
+  wtconv_status e = query_device(dev);
+  if (e != WTCONV_OK) return e;
+  const bool f32 = d->io == WTCONV_F32;
+  switch (d->k) {
+    case 1: return f32 ? launch_small_t<1, float>(d, dev, x, wfold, w0, b0, s0, flip, y, st)
+                       : launch_small_t<1, __nv_bfloat16>(d, dev, x, wfold, w0, b0, s0, flip, y, st);
+    case 3: return f32 ? launch_small_t<3, float>(d, dev, x, wfold, w0, b0, s0, flip, y, st)
+                       : launch_small_t<3, __nv_bfloat16>(d, dev, x, wfold, w0, b0, s0, flip, y, st);
+    case 5: return f32 ? launch_small_t<5, float>(d, dev, x, wfold, w0, b0, s0, flip, y, st)
+                       : launch_small_t<5, __nv_bfloat16>(d, dev, x, wfold, w0, b0, s0, flip, y, st);
+    default: return f32 ? launch_small_t<7, float>(d, dev, x, wfold, w0, b0, s0, flip, y, st)
+                        : launch_small_t<7, __nv_bfloat16>(d, dev, x, wfold, w0, b0, s0, flip, y, st);
+  }
+}
+
 // Folds the weights into `wfold` (flip = 1: the adjoint's block).
 wtconv_status run_fold(const wtconv_desc* d, const float* w0, const float* b0, const float* s0, const float* wl,
                        const float* sl, int flip, float* wfold, cudaStream_t st) {
@@ -635,6 +700,7 @@ wtconv_status run_folded(const wtconv_desc* d, const void* x, const float* wfold
   // the workspace layout (deep kernel or recursion) is planned for sm_100a's
   // shared memory per CTA
   if (dev.max_smem < PLAN_SMEM) return WTCONV_ERR_UNSUPPORTED;
+  if (small_planes(d) && !out) return launch_small(d, x, wfold, nullptr, nullptr, nullptr, 0, y, st);
   // the smaller layer's kernels report to the caller's status word
   int* status = status_word ? status_word : static_cast<int*>(ws);
   float* t1 = reinterpret_cast<float*>(static_cast<char*>(ws) + 16);
@@ -671,6 +737,8 @@ wtconv_status run_folded(const wtconv_desc* d, const void* x, const float* wfold
 wtconv_status run_forward(const wtconv_desc* d, const void* x, const float* w0, const float* b0, const float* s0,
                           const float* wl, const float* sl, void* y, int flip, void* ws, cudaStream_t st,
                           const wtconv_desc* out = nullptr) {
+  // level-0 small planes fold s0 into W0 and b0 inside their one kernel
+  if (small_planes(d) && !out) return launch_small(d, x, nullptr, w0, b0, s0, flip, y, st);
   float* wfold = reinterpret_cast<float*>(static_cast<char*>(ws) + pass_ws_bytes(d));
   wtconv_status e = run_fold(d, w0, b0, s0, wl, sl, flip, wfold, st);
   if (e != WTCONV_OK) return e;
@@ -1006,6 +1074,7 @@ bool build_bwd_plan(BwdPlan& Q, const wtconv_desc* d, const wtconv_desc* out, in
 }
 
 bool bwd_fused(const wtconv_desc* d) {
+  if (small_planes(d)) return false;  // backward-data on the small-plane kernel instead
   BwdPlan Q;
   return build_bwd_plan(Q, d, d, PLAN_SMEM);
 }
@@ -1737,7 +1806,7 @@ int wtconv_kernel_launches(const wtconv_desc* desc, int op) {
     return inner + op_acts(op);  // the pads of the inputs
   }
   const int pass = pass_launches(desc);
-  const int data = pass ? 1 + pass : 0;  // fold first
+  const int data = small_planes(desc) ? 1 : pass ? 1 + pass : 0;  // fold first, except on small level-0 planes
   const int weight = bwdw_whole_plane(desc) ? 2 : (desc->L == 0 ? 1 : desc->L) + 1;  // kernel(s), finalize
   switch (op) {
     case WTCONV_OP_FORWARD:

@@ -53,6 +53,9 @@
  *     the adjoint's folded weights).  For sides that are not multiples of 2^L
  *     it also holds zero-padded copies of the call's input planes (x or dy;
  *     both for the weight-gradient passes).  The workspace is required.
+ *     Level-0 layers (L = 0) on planes of at most 32x32 run one kernel per
+ *     data pass, a few planes per warp, scaling W0 and b0 by s0 as it loads
+ *     them (no fold launch; the folded weights in the workspace unused).
  *   - Arithmetic is fp32 throughout; bf16 I/O is rounded to nearest even on
  *     output.  Results are deterministic run to run (fixed reduction order).
  *   - Gradients are overwritten, not accumulated.
@@ -170,7 +173,8 @@ wtconv_status wtconv_backward_weight(const wtconv_desc* desc, const void* x,
  * SM (k <= 5) one fused pass stages x and dy once per unit and computes the
  * correlations, then the adjoint data pass, from the same on-chip pyramids
  * (launches: the adjoint weight fold, the fused pass, the finalize).  Other
- * shapes (row-band planes, k = 7) run wtconv_backward_data, then
+ * shapes (row-band planes, k = 7, level-0 planes of at most 32x32) run
+ * wtconv_backward_data, then
  * wtconv_backward_weight, in that order on `stream`.  dx equals what
  * wtconv_backward_data gives, bit for bit; the parameter gradients agree
  * with wtconv_backward_weight up to the order of the per-CTA partial sums.

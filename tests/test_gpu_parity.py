@@ -122,6 +122,19 @@ EDGE = [
     Workload("tma_L0_k1_30x40", 2, 2, 30, 40, 1, 0, "f32"),
     Workload("tma_L0_k5_reuse", 3, 700, 12, 20, 5, 0, "f32"),
     Workload("tma_L0_k5_bands_300", 1, 2, 300, 64, 5, 0, "f32"),
+    Workload("tma_L0_k7_36x36_batched", 7, 3, 36, 36, 7, 0, "f32"),
+    Workload("tma_L0_k5_reuse_40x36", 3, 300, 40, 36, 5, 0, "f32"),
+    # level 0 on planes of at most 32x32: a warp takes up to 8 planes at a
+    # time, a 4x4 tile per lane (two for 64-tile planes), the next planes
+    # prefetched into registers (planes past 512 elements per warp load the
+    # rest directly)
+    Workload("small_L0_k1_14", 5, 7, 14, 14, 1, 0, "f32"),
+    Workload("small_L0_k3_7x5_bf16", 3, 4, 7, 5, 3, 0, "bf16"),
+    Workload("small_L0_k7_16x16", 9, 2, 16, 16, 7, 0, "f32"),
+    Workload("small_L0_k5_32x16_bf16", 2, 3, 32, 16, 5, 0, "bf16"),
+    Workload("small_L0_k3_1x1", 4, 3, 1, 1, 3, 0, "f32"),
+    Workload("small_L0_k5_3x30", 6, 5, 3, 30, 5, 0, "f32"),
+    Workload("small_L0_k5_many", 37, 129, 14, 14, 5, 0, "f32"),
     # sides not multiples of 2^L (zero-padded copies, cropped results)
     Workload("ragged_13x11_L2", 2, 3, 13, 11, 5, 2, "f32"),
     Workload("ragged_7x9_L3_bf16", 1, 2, 7, 9, 3, 3, "bf16"),
