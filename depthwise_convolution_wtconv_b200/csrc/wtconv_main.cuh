@@ -616,9 +616,14 @@ __global__ void __launch_bounds__(DEEP_NT) wtconv_deep_kernel(const DeepPlan P, 
       const int un = u + gridDim.x, btn = un / P.C, cn = un - btn * P.C, nbn = btn * P.PB + (int)threadIdx.x;
       if (nbn < P.N) l2_prefetch(x + ((size_t)nbn * P.C + cn) * plane, (unsigned)(plane * sizeof(IO)));
     }
-    // the channel's folded level-2..L weights (contiguous in its block)
-    for (int i = threadIdx.x; i < (P.L - 1) * 4 * kk4; i += DEEP_NT) sw[i] = wfold[(size_t)c * P.wblk + P.wdeep + i];
-    // level-2 subbands straight from 4x4 blocks of x (two blocks in flight)
+    // the channel's folded level-2..L weights (contiguous in its block): the
+    // first DEEP_NT of them are loaded here and stored after the staging
+    // loads below are issued, so that the staging does not wait behind them
+    const int nw = (P.L - 1) * 4 * kk4;
+    const float* wsrc = wfold + (size_t)c * P.wblk + P.wdeep;
+    const float w_first = (int)threadIdx.x < nw ? wsrc[threadIdx.x] : 0.f;
+    for (int i = threadIdx.x + DEEP_NT; i < nw; i += DEEP_NT) sw[i] = wsrc[i];
+    // level-2 subbands straight from 4x4 blocks of x (four blocks in flight)
     {
       const int bw = P.W >> 2, per = (P.H >> 2) * bw, n = npb * per;
       const BufDesc& d = P.sd[2];
@@ -666,6 +671,7 @@ __global__ void __launch_bounds__(DEEP_NT) wtconv_deep_kernel(const DeepPlan P, 
         }
       }
     }
+    if ((int)threadIdx.x < nw) sw[threadIdx.x] = w_first;
     __syncthreads();
     for (int l = 3; l <= P.L; ++l) {
       const BufDesc& sb = P.sd[l - 1];
