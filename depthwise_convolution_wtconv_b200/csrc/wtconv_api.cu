@@ -551,7 +551,7 @@ wtconv_status launch_fold(const wtconv_desc* d, const Device& dev, const float* 
 // weights `wfold`.
 template <int K, typename IO>
 wtconv_status launch_forward_t(const wtconv_desc* d, const Device& dev, const void* x, const float* wfold, void* y,
-                               int* status, float* t1, const wtconv_desc* out, cudaStream_t st) {
+                               int* status, float* t1, const wtconv_desc* out, cudaStream_t st, const RawW& rw) {
   MainPlan M;
   if (!build_main_plan(M, d, dev.max_smem)) return WTCONV_ERR_UNSUPPORTED;
   if (out) {  // y is the image inside the padded planes x holds
@@ -587,7 +587,7 @@ wtconv_status launch_forward_t(const wtconv_desc* d, const Device& dev, const vo
     wtconv_status e = prepare(km, smem, occ, MAIN_NT);                                                  \
     if (e != WTCONV_OK) return e;                                                                       \
     km<<<std::min(M.units, dev.sms * occ), MAIN_NT, smem, st>>>(M, static_cast<const IO*>(x), t1, wfold, \
-                                                                static_cast<IO*>(y), status, xmap);     \
+                                                                static_cast<IO*>(y), status, xmap, rw); \
   }
   if (M.fused) {
     if (M.R3 == 8) WT_MAIN(8, true, false) else WT_MAIN(4, true, false)
@@ -606,9 +606,18 @@ wtconv_status launch_forward_t(const wtconv_desc* d, const Device& dev, const vo
 
 template <int K>
 wtconv_status launch_forward_k(const wtconv_desc* d, const Device& dev, const void* x, const float* wfold, void* y,
-                               int* status, float* t1, const wtconv_desc* out, cudaStream_t st) {
-  if (d->io == WTCONV_F32) return launch_forward_t<K, float>(d, dev, x, wfold, y, status, t1, out, st);
-  return launch_forward_t<K, __nv_bfloat16>(d, dev, x, wfold, y, status, t1, out, st);
+                               int* status, float* t1, const wtconv_desc* out, cudaStream_t st,
+                               const RawW& rw = RawW{nullptr, nullptr, nullptr, 0}) {
+  if (d->io == WTCONV_F32) return launch_forward_t<K, float>(d, dev, x, wfold, y, status, t1, out, st, rw);
+  return launch_forward_t<K, __nv_bfloat16>(d, dev, x, wfold, y, status, t1, out, st, rw);
+}
+
+// Level-0 fp32 planes whose output kernel takes the tensor-copy (DIRECT)
+// path: their data passes scale the raw taps in the kernel (no fold launch).
+bool direct_raw(const wtconv_desc* d) {
+  if (d->L != 0 || d->io != WTCONV_F32) return false;
+  MainPlan M;
+  return build_main_plan(M, d, PLAN_SMEM) && M.direct;
 }
 
 // ---- level 0 on small planes: a warp per plane (wtconv_small.cuh)
@@ -737,8 +746,23 @@ wtconv_status run_folded(const wtconv_desc* d, const void* x, const float* wfold
 wtconv_status run_forward(const wtconv_desc* d, const void* x, const float* w0, const float* b0, const float* s0,
                           const float* wl, const float* sl, void* y, int flip, void* ws, cudaStream_t st,
                           const wtconv_desc* out = nullptr) {
-  // level-0 small planes fold s0 into W0 and b0 inside their one kernel
+  // level-0 small planes, and level-0 planes on the tensor-copy path, scale
+  // W0 and b0 by s0 inside their one kernel
   if (small_planes(d) && !out) return launch_small(d, x, nullptr, w0, b0, s0, flip, y, st);
+  if (direct_raw(d) && !out) {
+    Device dev;
+    wtconv_status e = query_device(dev);
+    if (e != WTCONV_OK) return e;
+    if (dev.max_smem < PLAN_SMEM) return WTCONV_ERR_UNSUPPORTED;  // planned for sm_100a's shared memory
+    const RawW rw{w0, b0, s0, flip};
+    int* status = static_cast<int*>(ws);
+    switch (d->k) {
+      case 1: return launch_forward_k<1>(d, dev, x, nullptr, y, status, nullptr, nullptr, st, rw);
+      case 3: return launch_forward_k<3>(d, dev, x, nullptr, y, status, nullptr, nullptr, st, rw);
+      case 5: return launch_forward_k<5>(d, dev, x, nullptr, y, status, nullptr, nullptr, st, rw);
+      default: return launch_forward_k<7>(d, dev, x, nullptr, y, status, nullptr, nullptr, st, rw);
+    }
+  }
   float* wfold = reinterpret_cast<float*>(static_cast<char*>(ws) + pass_ws_bytes(d));
   wtconv_status e = run_fold(d, w0, b0, s0, wl, sl, flip, wfold, st);
   if (e != WTCONV_OK) return e;
@@ -1806,7 +1830,8 @@ int wtconv_kernel_launches(const wtconv_desc* desc, int op) {
     return inner + op_acts(op);  // the pads of the inputs
   }
   const int pass = pass_launches(desc);
-  const int data = small_planes(desc) ? 1 : pass ? 1 + pass : 0;  // fold first, except on small level-0 planes
+  // fold first, except on level-0 planes that scale the taps in their one kernel
+  const int data = (small_planes(desc) || direct_raw(desc)) ? 1 : pass ? 1 + pass : 0;
   const int weight = bwdw_whole_plane(desc) ? 2 : (desc->L == 0 ? 1 : desc->L) + 1;  // kernel(s), finalize
   switch (op) {
     case WTCONV_OP_FORWARD:

@@ -456,20 +456,22 @@ __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, i
 // y0 - r, channel c, batch entry nb0), so that row y of plane j lands at
 // (y - y0 + r) * ld + x + 4 and the rows and columns outside the plane
 // (the zero padding) arrive as zeros; no staging pass.  The folded weights
-// come by a bulk copy as for the other paths.  Thread 0 issues.
+// come by a bulk copy as for the other paths, unless the kernel scales the
+// raw ones itself (wfold null).  Thread 0 issues.
 __device__ __forceinline__ void main_issue_tensor(const MainPlan& P, float* slot, uint64_t* full, const UnitGeo& g,
                                                   int buf, const CUtensorMap* xmap,
                                                   const float* __restrict__ wfold) {
-  const unsigned bw = (unsigned)(P.wblk * 4);
+  const unsigned bw = wfold ? (unsigned)(P.wblk * 4) : 0u;
   const unsigned bx = (unsigned)(P.xf.ld * P.xf.rows * P.PB * 4);
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(full)), "r"(bw + bx)
                : "memory");
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-          smem_u32(slot + P.wraw_off)),
-      "l"(wfold + (size_t)g.c * P.wblk), "r"(bw), "r"(smem_u32(full))
-      : "memory");
+  if (wfold)
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(slot + P.wraw_off)),
+        "l"(wfold + (size_t)g.c * P.wblk), "r"(bw), "r"(smem_u32(full))
+        : "memory");
   tma_load_4d(slot + P.xf.off + buf * P.xbuf, xmap, -4, g.y0 - P.r, g.c, g.nb0, full);
 }
 
@@ -477,7 +479,7 @@ template <int K, int R3, typename IO, bool FUSED, bool DIRECT>
 __global__ void __launch_bounds__(MAIN_NT, 4)
     wtconv_main_kernel(const MainPlan P, const IO* __restrict__ x, const float* __restrict__ t1g,
                        const float* __restrict__ wfold, IO* __restrict__ y, int* __restrict__ status,
-                       const __grid_constant__ CUtensorMap xmap) {
+                       const __grid_constant__ CUtensorMap xmap, const RawW rw) {
   extern __shared__ __align__(128) float4 smem4[];
   float* sm = reinterpret_cast<float*>(smem4);
   uint64_t* full = reinterpret_cast<uint64_t*>(sm);
@@ -492,8 +494,22 @@ __global__ void __launch_bounds__(MAIN_NT, 4)
   __syncthreads();
   const int myunits = (int)blockIdx.x < P.units ? (P.units - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
   float* slot = sm + P.slot0;
+  // level-0 direct path without a folded block (wfold null): thread t <= kk4
+  // holds the next unit's raw tap t (the bias at t = kk4) and its channel's
+  // scale, loaded one unit ahead and scaled into the weight slots when that
+  // unit starts
+  float w_next = 0.f, s_next = 0.f;
+  auto fetch_w = [&](int c) {
+    constexpr int KK = K * K;
+    if (tid <= P.kk4) {
+      s_next = rw.s0[c];
+      w_next = tid < KK ? rw.w0[(size_t)c * KK + (rw.flip ? KK - 1 - tid : tid)]
+                        : (tid == P.kk4 && !rw.flip ? rw.b0[c] : 0.f);
+    }
+  };
   if constexpr (DIRECT) {
     if (tid == 0 && myunits > 0) main_issue_tensor(P, slot, full, unit_geo(P, blockIdx.x), 0, &xmap, wfold);
+    if (!wfold && myunits > 0) fetch_w(unit_geo(P, blockIdx.x).c);
   } else {
     if (tid == 0 && myunits > 0) main_issue<IO>(P, slot, full, unit_geo(P, blockIdx.x), x, t1g, wfold);
   }
@@ -532,8 +548,12 @@ __global__ void __launch_bounds__(MAIN_NT, 4)
     }
     // folded weights and t1 rows leave the raw region, which the next
     // unit's copies overwrite while this unit computes
-    for (int i = tid; i < (P.wblk >> 2); i += MAIN_NT)
-      reinterpret_cast<float4*>(slot + P.w_off)[i] = reinterpret_cast<const float4*>(slot + P.wraw_off)[i];
+    if (DIRECT && !wfold) {
+      if (tid <= P.kk4) slot[P.w_off + tid] = s_next * w_next;
+    } else {
+      for (int i = tid; i < (P.wblk >> 2); i += MAIN_NT)
+        reinterpret_cast<float4*>(slot + P.w_off)[i] = reinterpret_cast<const float4*>(slot + P.wraw_off)[i];
+    }
     if (!FUSED && P.L >= 2) {
       const int q4 = P.f_t1q.d, per = P.f_t1pp.d;  // (W1 + 3) / 4, TH/2 rows of them
       for (int it = tid; it < g.npb * per; it += MAIN_NT) {
@@ -554,6 +574,7 @@ __global__ void __launch_bounds__(MAIN_NT, 4)
     if constexpr (DIRECT) {
       if (tid == 0 && k + 1 < myunits)
         main_issue_tensor(P, slot, full, unit_geo(P, blockIdx.x + (k + 1) * gridDim.x), (k + 1) & 1, &xmap, wfold);
+      if (!wfold && k + 1 < myunits) fetch_w(unit_geo(P, blockIdx.x + (k + 1) * gridDim.x).c);
     } else {
       if (tid == 0 && k + 1 < myunits)
         main_issue<IO>(P, slot, full, unit_geo(P, blockIdx.x + (k + 1) * gridDim.x), x, t1g, wfold);

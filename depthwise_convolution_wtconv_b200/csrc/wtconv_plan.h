@@ -87,6 +87,15 @@ struct MainPlan {
 // Plan of the deep-level kernel: levels 2..L of PB planes of one channel,
 // written as t1 (the synthesis of levels >= 2 at level-1 resolution,
 // already scaled by the level-1 synthesis factor) to global memory.
+// Raw parameters for the level-0 direct output kernel, which can scale the
+// taps and the bias itself instead of reading a folded block.
+struct RawW {
+  const float* w0;
+  const float* b0;
+  const float* s0;
+  int flip;
+};
+
 struct DeepPlan {
   int N, C, H, W, K, r, L, H1, W1, kk4, io_bytes, vec_in;
   int PB, nbatch;

@@ -53,9 +53,11 @@
  *     the adjoint's folded weights).  For sides that are not multiples of 2^L
  *     it also holds zero-padded copies of the call's input planes (x or dy;
  *     both for the weight-gradient passes).  The workspace is required.
- *     Level-0 layers (L = 0) on planes of at most 32x32 run one kernel per
- *     data pass, a few planes per warp, scaling W0 and b0 by s0 as it loads
- *     them (no fold launch; the folded weights in the workspace unused).
+ *     Level-0 layers (L = 0) on planes of at most 32x32 (a few planes per
+ *     warp), and fp32 level-0 layers whose rows are a multiple of 4 and at
+ *     most 248 elements (one tensor copy per unit), run one kernel per data
+ *     pass that scales W0 and b0 by s0 as it loads them (no fold launch; the
+ *     folded weights in the workspace unused).
  *   - Arithmetic is fp32 throughout; bf16 I/O is rounded to nearest even on
  *     output.  Results are deterministic run to run (fixed reduction order).
  *   - Gradients are overwritten, not accumulated.

@@ -95,20 +95,22 @@ def test_kernel_launch_counts(lib):
     assert n(whole, 7) == 0
 
 
-def test_small_level0_planes_take_one_kernel_per_data_pass(lib):
-    """Level-0 planes of at most 32x32 run on warps of their own: one launch
-    per data pass (the scale is applied as the kernel loads the weights, no
-    fold launch), the weight-gradient kernel + finalize, and the backward as
-    the two passes in turn; larger level-0 planes keep fold + output kernel."""
+def test_level0_data_passes_take_one_kernel(lib):
+    """Level-0 planes of at most 32x32 (on warps of their own) and fp32
+    level-0 planes on the tensor-copy path run one launch per data pass (the
+    scale is applied as the kernel loads the weights, no fold launch), then
+    the weight-gradient kernel + finalize, and the backward as the two passes
+    in turn; other level-0 planes (bf16 rows too wide for one tensor copy
+    per unit here) keep fold + output kernel."""
     n = lambda d, op: lib.wtconv_kernel_launches(ctypes.byref(d), op)
     small = _lib.WTConvDesc(64, 384, 14, 14, 5, 0, 0)
     assert [n(small, op) for op in range(6)] == [1, 1, 2, 3, 1, 1]
     edge = _lib.WTConvDesc(2, 3, 32, 32, 7, 0, 1)     # 64 tiles: two per lane
     assert [n(edge, op) for op in range(4)] == [1, 1, 2, 3]
-    tall = _lib.WTConvDesc(2, 3, 40, 16, 7, 0, 1)     # taller than 32: the CTA-wide kernels
+    tall = _lib.WTConvDesc(2, 3, 40, 16, 7, 0, 1)     # bf16, taller than 32: fold + output kernel
     assert [n(tall, op) for op in range(4)] == [2, 2, 2, 4]
-    large = _lib.WTConvDesc(64, 32, 112, 112, 3, 0, 0)
-    assert [n(large, op) for op in range(4)] == [2, 2, 2, 4]
+    large = _lib.WTConvDesc(64, 32, 112, 112, 3, 0, 0)  # fp32, 112-float rows: one tensor copy per unit
+    assert [n(large, op) for op in range(4)] == [1, 1, 2, 3]
 
 
 def test_workspace_of_ragged_sides(lib):
