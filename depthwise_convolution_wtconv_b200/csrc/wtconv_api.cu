@@ -952,35 +952,56 @@ bool build_bw_direct_plan(BwDirectPlan& B, const wtconv_desc* d, int max_smem) {
   B.kk4 = rup(d->k * d->k, 4);
   B.V = d->k * d->k + 1;
   B.xld = d->W + 8;
-  B.xrows = rup(d->H, 4) + 2 * B.r;
-  if (B.xld > 256 || B.xrows > 256) return false;
-  B.xps = B.xld * B.xrows;
   B.gld = d->W;
-  B.grows = rup(d->H, 4);
-  B.gps = B.gld * B.grows;
-  B.tiles_pp = (B.grows / 4) * (d->W / 4);
-  B.f_tiles = make_fdiv(B.tiles_pp);
-  B.f_tx = make_fdiv(d->W / 4);
-  const int pb0 = std::max(1, std::min({d->N, cdiv_h(BW_NT, B.tiles_pp), 256}));
-  for (const int budget : {(int)(SM_SMEM / 2 - 1024), max_smem}) {
-    for (int pb = pb0; pb >= 1; --pb) {
-      // header: two mbarriers and the abort flag; buffers on 128-byte boundaries
-      int cur = 32;
-      for (int b = 0; b < 2; ++b) {
-        B.xoff[b] = cur;
-        cur += rup(pb * B.xps, 32);
-        B.goff[b] = cur;
-        cur += rup(pb * B.gps, 32);
-      }
-      B.red_off = B.xoff[0];
-      const int need = std::max(cur, B.red_off + BW_NT * (B.kk4 + 1) + BW_NT);
-      if ((size_t)rup(need, 4) * 4 <= (size_t)std::min(budget, max_smem)) {
-        B.PB = pb;
-        B.smem_floats = rup(need, 4);
+  if (B.xld > 256) return false;
+  // Lays out two buffer sets for units of pb planes of `rows` rows (whole
+  // planes: rup(H, 4); row bands: TB) within `budget` bytes.
+  auto fit = [&](int pb, int rows, int budget) {
+    B.xrows = rows + 2 * B.r;
+    B.grows = rows;
+    if (B.xrows > 256) return false;
+    B.xps = B.xld * B.xrows;
+    B.gps = B.gld * B.grows;
+    B.tiles_pp = (B.grows / 4) * (d->W / 4);
+    // header: two mbarriers and the abort flag; buffers on 128-byte boundaries
+    int cur = 32;
+    for (int b = 0; b < 2; ++b) {
+      B.xoff[b] = cur;
+      cur += rup(pb * B.xps, 32);
+      B.goff[b] = cur;
+      cur += rup(pb * B.gps, 32);
+    }
+    B.red_off = B.xoff[0];
+    const int need = std::max(cur, B.red_off + BW_NT * (B.kk4 + 1) + BW_NT);
+    if ((size_t)rup(need, 4) * 4 > (size_t)std::min(budget, max_smem)) return false;
+    B.PB = pb;
+    B.smem_floats = rup(need, 4);
+    B.f_tiles = make_fdiv(B.tiles_pp);
+    B.f_tx = make_fdiv(d->W / 4);
+    return true;
+  };
+  const int half = (int)(SM_SMEM / 2 - 1024);
+  const int whole = rup(d->H, 4);
+  const int pb0 = std::max(1, std::min({d->N, cdiv_h(BW_NT, (whole / 4) * (d->W / 4)), 256}));
+  // whole planes at two CTAs per SM; else row bands at two CTAs per SM (the
+  // largest band, a multiple of 4 rows dividing H, of at least 16 rows);
+  // else whole planes at one CTA per SM
+  B.nb = 1;
+  B.TB = whole;
+  for (int pb = pb0; pb >= 1; --pb)
+    if (fit(pb, whole, half)) return true;
+  if (d->H % 4 == 0)
+    for (int nb = 2; d->H / nb >= 16; ++nb) {
+      const int tb = d->H / nb;
+      if (d->H % nb || tb % 4) continue;
+      if (fit(1, tb, half)) {
+        B.nb = nb;
+        B.TB = tb;
         return true;
       }
     }
-  }
+  for (int pb = pb0; pb >= 1; --pb)
+    if (fit(pb, whole, max_smem)) return true;
   return false;
 }
 
@@ -1268,9 +1289,9 @@ wtconv_status launch_finalize(const wtconv_desc* d, int groups, const float* par
 // fewest sequential units per CTA slot, counting one more unit per CTA for
 // its fixed costs (clearing its shared memory, the first copy that nothing
 // overlaps, the final reduction and partial write); ties broken towards
-// longer CTAs (fewer partial sums).  0 when no choice has at most
-// max_groups CTAs per channel.
-int planes_per_cta(int N, int C, int units_pb, int slots, int max_groups) {
+// longer CTAs (fewer partial sums); a plane in `bands` row bands is that many
+// units.  0 when no choice has at most max_groups CTAs per channel.
+int planes_per_cta(int N, int C, int units_pb, int slots, int max_groups, int bands = 1) {
   long best = -1;
   int ppc = 0;
   for (int q = units_pb; q < N + units_pb; q += units_pb) {
@@ -1278,7 +1299,7 @@ int planes_per_cta(int N, int C, int units_pb, int slots, int max_groups) {
     const int groups = (N + p - 1) / p;
     if (groups > max_groups) continue;
     const long ctas = (long)C * groups;
-    const long cost = ((ctas + slots - 1) / slots) * ((p + units_pb - 1) / units_pb + 1);
+    const long cost = ((ctas + slots - 1) / slots) * ((long)(p + units_pb - 1) / units_pb * bands + 1);
     if (best < 0 || cost <= best) {
       best = cost;
       ppc = p;
@@ -1328,7 +1349,7 @@ wtconv_status launch_bw_direct(BwDirectPlan& B, const Device& dev, const wtconv_
   int occ = 0;
   wtconv_status e = prepare(kern, smem, occ, BW_NT);
   if (e != WTCONV_OK) return e;
-  B.ppc = planes_per_cta(B.N, B.C, B.PB, dev.sms * occ, max_groups);
+  B.ppc = planes_per_cta(B.N, B.C, B.PB, dev.sms * occ, max_groups, B.nb);
   if (B.ppc == 0) return WTCONV_ERR_SCRATCH_LIMIT;
   B.ngroups = (B.N + B.ppc - 1) / B.ppc;
   CUtensorMap xmap;

@@ -502,21 +502,33 @@ __global__ void __launch_bounds__(BW_NT, 1) wtconv_bwdw_direct_kernel(const __gr
   __syncthreads();
   const int c = blockIdx.x % P.C, grp = blockIdx.x / P.C;
   const int n_begin = grp * P.ppc, n_end = min(P.N, n_begin + P.ppc);
-  const int nunits = n_end > n_begin ? (n_end - n_begin + P.PB - 1) / P.PB : 0;
-  const unsigned gbytes = (unsigned)((size_t)P.H * P.W * 4);
+  // units: PB planes at a time (nb == 1), or one row band of one plane
+  const int nunits = n_end <= n_begin ? 0 : P.nb == 1 ? (n_end - n_begin + P.PB - 1) / P.PB : (n_end - n_begin) * P.nb;
+  const unsigned gbytes = (unsigned)((size_t)(P.nb == 1 ? P.H : P.TB) * P.W * 4);
   auto issue = [&](int u) {
-    const int b = u & 1, nb0 = n_begin + u * P.PB, cnt = min(P.PB, n_end - nb0);
+    const int b = u & 1;
+    int nb0, cnt, y0;
+    if (P.nb == 1) {
+      nb0 = n_begin + u * P.PB;
+      cnt = min(P.PB, n_end - nb0);
+      y0 = 0;
+    } else {
+      const int pl = u / P.nb;
+      nb0 = n_begin + pl;
+      cnt = 1;
+      y0 = (u - pl * P.nb) * P.TB;
+    }
     const unsigned xbytes = (unsigned)(P.xps * P.PB * 4);
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(full + b)),
                  "r"(xbytes + gbytes * (unsigned)cnt)
                  : "memory");
-    tma_load_4d(sm + P.xoff[b], &xmap, -4, -r, c, nb0, full + b);
+    tma_load_4d(sm + P.xoff[b], &xmap, -4, y0 - r, c, nb0, full + b);
     for (int jj = 0; jj < cnt; ++jj)
       asm volatile(
           "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
               smem_u32(sm + P.goff[b] + jj * P.gps)),
-          "l"(dy + ((size_t)(nb0 + jj) * P.C + c) * P.H * P.W), "r"(gbytes), "r"(smem_u32(full + b))
+          "l"(dy + (((size_t)(nb0 + jj) * P.C + c) * P.H + y0) * P.W), "r"(gbytes), "r"(smem_u32(full + b))
           : "memory");
   };
   if (tid == 0) {
@@ -532,7 +544,7 @@ __global__ void __launch_bounds__(BW_NT, 1) wtconv_bwdw_direct_kernel(const __gr
     mb_wait(full + b, (k >> 1) & 1, abort_flag);
     __syncthreads();
     if (*abort_flag) break;  // uniform: read after the barrier
-    const int npb = min(P.PB, n_end - (n_begin + k * P.PB));
+    const int npb = P.nb == 1 ? min(P.PB, n_end - (n_begin + k * P.PB)) : 1;
     const float* xs = sm + P.xoff[b];
     const float* gs = sm + P.goff[b];
     for (int t = tid; t < npb * P.tiles_pp; t += BW_NT) {

@@ -194,6 +194,7 @@ struct BwdPlan {
 struct BwDirectPlan {
   int N, C, H, W, K, r, kk4, V;
   int PB, ppc, ngroups;
+  int nb, TB;           // row bands per plane (1: whole planes) and rows per band (PB = 1 then)
   int xld, xrows, xps, gld, grows, gps;
   int xoff[2], goff[2];
   int tiles_pp;
