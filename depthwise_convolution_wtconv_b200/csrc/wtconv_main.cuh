@@ -610,6 +610,21 @@ __global__ void __launch_bounds__(MAIN_NT, 4)
 }
 
 // ------------------------------------------------------------ deep kernel
+// Four elements as loaded (converted to fp32 where used).
+template <typename IO> struct Raw4;
+template <> struct Raw4<float> {
+  using T = float4;
+  static __device__ __forceinline__ T ld(const float* p) { return __ldg(reinterpret_cast<const float4*>(p)); }
+  static __device__ __forceinline__ float4 cvt(T v) { return v; }
+};
+template <> struct Raw4<__nv_bfloat16> {
+  using T = uint2;
+  static __device__ __forceinline__ T ld(const __nv_bfloat16* p) { return __ldg(reinterpret_cast<const uint2*>(p)); }
+  static __device__ __forceinline__ float4 cvt(T r) {
+    return make_float4(__uint_as_float(r.x << 16), __uint_as_float(r.x & 0xffff0000u), __uint_as_float(r.y << 16),
+                       __uint_as_float(r.y & 0xffff0000u));
+  }
+};
 // Levels 2..L of the planes of a batch: level-2 subbands from 4x4 blocks of
 // x, the rest of the pyramid, every level conv (folded weights
 // 2^-l s_l W_l), then t1 by the closed form, stored to global memory.
@@ -618,6 +633,7 @@ __global__ void __launch_bounds__(DEEP_NT) wtconv_deep_kernel(const DeepPlan P, 
                                                               const float* __restrict__ wfold,
                                                               float* __restrict__ t1g) {
   constexpr int r = K / 2;
+  constexpr int DQ = sizeof(IO) == 2 ? 8 : 4;  // 4x4 blocks in flight per thread
   extern __shared__ float4 smem4[];
   float* sm = reinterpret_cast<float*>(smem4);
   for (int i = threadIdx.x; i < (P.smem_floats >> 2); i += DEEP_NT) smem4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -644,15 +660,16 @@ __global__ void __launch_bounds__(DEEP_NT) wtconv_deep_kernel(const DeepPlan P, 
     const float* wsrc = wfold + (size_t)c * P.wblk + P.wdeep;
     const float w_first = (int)threadIdx.x < nw ? wsrc[threadIdx.x] : 0.f;
     for (int i = threadIdx.x + DEEP_NT; i < nw; i += DEEP_NT) sw[i] = wsrc[i];
-    // level-2 subbands straight from 4x4 blocks of x (four blocks in flight)
+    // level-2 subbands straight from 4x4 blocks of x (DQ blocks in flight per
+    // thread, held as loaded and converted where used)
     {
       const int bw = P.W >> 2, per = (P.H >> 2) * bw, n = npb * per;
       const BufDesc& d = P.sd[2];
       const int bs = d.ld * d.rows;
-      for (int it0 = threadIdx.x; it0 < n; it0 += 4 * DEEP_NT) {
-        float4 v[4][4];
+      for (int it0 = threadIdx.x; it0 < n; it0 += DQ * DEEP_NT) {
+        typename Raw4<IO>::T v[DQ][4];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
+        for (int q = 0; q < DQ; ++q) {
           const int it = it0 + q * DEEP_NT;
           if (it < n) {
             const int pb = P.f_stage_per.div(it);
@@ -661,23 +678,26 @@ __global__ void __launch_bounds__(DEEP_NT) wtconv_deep_kernel(const DeepPlan P, 
             const int x0 = (rem - by * bw) << 2;
             const IO* src = x + ((size_t)(nb0 + pb) * P.C + c) * plane + (size_t)(by << 2) * P.W + x0;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) v[q][i] = load4v(src + (size_t)i * P.W);  // W % 4 == 0 here
+            for (int i = 0; i < 4; ++i) v[q][i] = Raw4<IO>::ld(src + (size_t)i * P.W);  // W % 4 == 0 here
           }
         }
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
+        for (int q = 0; q < DQ; ++q) {
           const int it = it0 + q * DEEP_NT;
           if (it < n) {
             const int pb = P.f_stage_per.div(it);
             const int rem = it - pb * per;
             const int by = P.f_stage_x.div(rem);
             const int bxi = rem - by * bw;
+            float4 w[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) w[i] = Raw4<IO>::cvt(v[q][i]);
             float ll[2][2];
 #pragma unroll
             for (int a = 0; a < 2; ++a) {
               float l0, h0, g0, k0, l1, h1, g1, k1;
-              haar4(v[q][2 * a].x, v[q][2 * a].y, v[q][2 * a + 1].x, v[q][2 * a + 1].y, l0, h0, g0, k0);
-              haar4(v[q][2 * a].z, v[q][2 * a].w, v[q][2 * a + 1].z, v[q][2 * a + 1].w, l1, h1, g1, k1);
+              haar4(w[2 * a].x, w[2 * a].y, w[2 * a + 1].x, w[2 * a + 1].y, l0, h0, g0, k0);
+              haar4(w[2 * a].z, w[2 * a].w, w[2 * a + 1].z, w[2 * a + 1].w, l1, h1, g1, k1);
               ll[a][0] = l0;
               ll[a][1] = l1;
             }
