@@ -620,7 +620,7 @@ bool direct_raw(const wtconv_desc* d) {
   return build_main_plan(M, d, PLAN_SMEM) && M.direct;
 }
 
-// ---- level 0 on small planes: a warp per plane (wtconv_small.cuh)
+// ---- level 0 on small planes: a few planes per warp (wtconv_small.cuh)
 
 // Level-0 planes of at most 32x32 (at most 64 4x4 tiles).
 bool small_planes(const wtconv_desc* d) { return d->L == 0 && d->W <= 32 && d->H <= 32; }
